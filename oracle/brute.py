@@ -1,0 +1,74 @@
+"""Pure-Python brute force for tiny inputs: explicit loops, ``math.fsum``, ``sorted``.
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/oracle.py``).  Independent of the NumPy oracle: no
+NumPy arithmetic, no shared helpers; it exists to pin the oracle on inputs small enough to
+loop over.  The quantities are those of the Mosaic page's mask-only logits step and the
+confidence-driven unmasking of the dLLM survey page ("Main Findings").
+"""
+from __future__ import annotations
+
+import math
+import struct
+
+
+def bf16_to_float(bits: int) -> float:
+    """bfloat16 bit pattern -> Python float (exact): it is the upper 16 bits of a float32."""
+    return struct.unpack("<f", struct.pack("<I", (int(bits) & 0xFFFF) << 16))[0]
+
+
+def compact(mask_rows):
+    """mask_rows: list of B lists of 0/1 -> (row_idx, seq_off) by explicit enumeration."""
+    row_idx, seq_off = [], [0]
+    L = len(mask_rows[0]) if mask_rows else 0
+    for b, row in enumerate(mask_rows):
+        for l, v in enumerate(row):
+            if v:
+                row_idx.append(b * L + l)
+        seq_off.append(len(row_idx))
+    return row_idx, seq_off
+
+
+def dot(h, w):
+    """Correctly rounded dot product of two float lists (math.fsum of exact products)."""
+    return math.fsum(a * b for a, b in zip(h, w))
+
+
+def row_logits(h, W):
+    return [dot(h, w) for w in W]
+
+
+def stats(z):
+    """(tok, m, lse, conf) of one logit row z by definition."""
+    m = max(z)
+    tok = next(i for i, x in enumerate(z) if x == m)
+    s = math.fsum(math.exp(x - m) for x in z)
+    lse = m + math.log(s)
+    conf = math.exp(m - lse)
+    return tok, m, lse, conf
+
+
+def topk(cands, k):
+    """cands: list of (conf, pos); the k best by (conf desc, pos asc)."""
+    return [p for _, p in sorted(cands, key=lambda cp: (-cp[0], cp[1]))[:k]]
+
+
+def step(H, W, mask_rows, k, win=None):
+    """Whole decode step on lists: H [B*L][d] floats, W [V][d] floats, mask [B][L] 0/1."""
+    B = len(mask_rows)
+    L = len(mask_rows[0])
+    row_idx, seq_off = compact(mask_rows)
+    per_row = [stats(row_logits(H[p], W)) for p in row_idx]
+    idx, n_sel = [], []
+    for b in range(B):
+        cands = []
+        for r in range(seq_off[b], seq_off[b + 1]):
+            pos = row_idx[r] - b * L
+            if win is None or (win[0][b] <= pos < win[1][b]):
+                cands.append((per_row[r][3], pos))
+        sel = topk(cands, k)
+        n_sel.append(len(sel))
+        idx.append(sel + [-1] * (k - len(sel)))
+    return dict(row_idx=row_idx, seq_off=seq_off,
+                tok=[s[0] for s in per_row], m=[s[1] for s in per_row],
+                lse=[s[2] for s in per_row], conf=[s[3] for s in per_row],
+                idx=idx, n_sel=n_sel)

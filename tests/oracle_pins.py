@@ -1,0 +1,215 @@
+"""Pin checks for the CPU oracle, written against an oracle-like namespace.
+
+Each check raises AssertionError when the oracle disagrees with something fixed outside it:
+a hand-worked fixture, a closed form, a library routine, an invariant or brute force.  The
+checks take the namespace as an argument so that ``test_oracle_mutations.py`` can run them
+against copies of the oracle with a planted mistake and show that some check fails.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import scipy.special
+import torch
+
+from oracle import brute
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _bits(a) -> np.ndarray:
+    """Exact bf16 bit patterns of small float arrays (values chosen bf16-representable)."""
+    t = torch.tensor(np.asarray(a, dtype=np.float32)).to(torch.bfloat16)
+    assert torch.equal(t.float(), torch.tensor(np.asarray(a, dtype=np.float32))), "not bf16-exact"
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def _rand_bits(rng: np.random.Generator, shape, scale=1.0) -> np.ndarray:
+    x = torch.tensor(rng.standard_normal(shape).astype(np.float32) * scale).to(torch.bfloat16)
+    return x.view(torch.int16).numpy().view(np.uint16)
+
+
+def _bf16_list(bits) -> list:
+    return [[brute.bf16_to_float(b) for b in row] for row in np.asarray(bits)]
+
+
+# ----------------------------------------------------------------------------------------
+def check_handworked(o):
+    g = json.load(open(os.path.join(GOLDEN, "handworked_step.json")))
+    H, W, M = _bits(g["H"]), _bits(g["W"]), np.array(g["M"], dtype=np.uint8)
+    out = o.oracle_step(H, W, M, g["k"])
+    assert out["row_idx"].tolist() == g["row_idx"]
+    assert out["seq_off"].tolist() == g["seq_off"]
+    assert out["tok"].tolist() == g["tok"]
+    np.testing.assert_allclose(out["m"], g["m"], rtol=0, atol=0)
+    np.testing.assert_allclose(out["lse"], g["lse"], rtol=1e-14)
+    np.testing.assert_allclose(out["conf"], g["conf"], rtol=1e-14)
+    assert out["idx"].tolist() == g["idx"]
+    assert out["n_sel"].tolist() == g["n_sel"]
+    out1 = o.oracle_step(H, W, M, 1)
+    assert out1["idx"].tolist() == g["k1_idx"]
+    lo, hi = np.array(g["window_lo"]), np.array(g["window_hi"])
+    outw = o.oracle_step(H, W, M, 2, lo, hi)
+    assert outw["idx"].tolist() == g["window_k2_idx"]
+    assert outw["n_sel"].tolist() == g["window_k2_n_sel"]
+    # the logits themselves
+    Z = o.logits_rows(o.bf16_bits_to_f64(H[out["row_idx"]]), o.bf16_bits_to_f64(W))
+    np.testing.assert_array_equal(Z, np.array(g["logits"], dtype=np.float64))
+
+
+def check_topk_ties(o):
+    g = json.load(open(os.path.join(GOLDEN, "topk_ties.json")))
+    M = np.array(g["M"], dtype=np.uint8)
+    row_idx, seq_off, count = o.mask_compact(M)
+    assert row_idx.tolist() == g["positions"]
+    for dt in (np.float32, np.float64):
+        conf = np.array(g["conf"], dtype=dt)
+        for c in g["cases"]:
+            lo = np.array([c["lo"]]) if "lo" in c else None
+            hi = np.array([c["hi"]]) if "hi" in c else None
+            idx, n_sel = o.select_unmask(conf, row_idx, seq_off, g["L"], c["k"], lo, hi)
+            assert idx[0].tolist() == c["idx"], (c, idx)
+            assert int(n_sel[0]) == c["n_sel"]
+
+
+def check_compact(o, seeds=range(8)):
+    rng = np.random.default_rng(123)
+    cases = [np.zeros((1, 5), np.uint8), np.ones((2, 3), np.uint8),
+             np.array([[0, 7, 0, 255, 1]], np.uint8)]
+    for s in seeds:
+        B, L = int(rng.integers(1, 5)), int(rng.integers(1, 40))
+        cases.append((rng.random((B, L)) < rng.random()).astype(np.uint8))
+    for M in cases:
+        row_idx, seq_off, count = o.mask_compact(M)
+        r2, s2 = brute.compact([[1 if v else 0 for v in row] for row in M.tolist()])
+        assert row_idx.tolist() == r2 and seq_off.tolist() == s2 and count == len(r2)
+        assert row_idx.dtype == np.int32 and seq_off.dtype == np.int32
+
+
+def check_brute_random(o, n_cases=12):
+    rng = np.random.default_rng(7)
+    for _ in range(n_cases):
+        B, L = int(rng.integers(1, 3)), int(rng.integers(1, 17))
+        d, V = int(rng.integers(1, 9)), int(rng.integers(1, 33))
+        k = int(rng.integers(1, 6))
+        H, W = _rand_bits(rng, (B * L, d)), _rand_bits(rng, (V, d), 0.5)
+        M = (rng.random((B, L)) < 0.6).astype(np.uint8)
+        win = None
+        if rng.random() < 0.5:
+            lo = rng.integers(0, L, size=B)
+            hi = np.minimum(L, lo + rng.integers(1, L + 1, size=B))
+            win = (lo, hi)
+        out = o.oracle_step(H, W, M, k, *(win if win else (None, None)))
+        ref = brute.step(_bf16_list(H), _bf16_list(W), M.tolist(), k,
+                         (win[0].tolist(), win[1].tolist()) if win else None)
+        assert out["row_idx"].tolist() == ref["row_idx"]
+        assert out["seq_off"].tolist() == ref["seq_off"]
+        assert out["tok"].tolist() == ref["tok"]
+        np.testing.assert_allclose(out["m"], ref["m"], rtol=1e-13, atol=1e-300)
+        np.testing.assert_allclose(out["lse"], ref["lse"], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(out["conf"], ref["conf"], rtol=1e-12)
+        assert out["idx"].tolist() == ref["idx"]
+        assert out["n_sel"].tolist() == ref["n_sel"]
+
+
+def check_closed_forms(o):
+    # (1) all vocabulary rows equal -> all logits equal: tok 0, conf 1/V, lse = z + ln V
+    rng = np.random.default_rng(3)
+    d, V = 16, 37
+    w = _rand_bits(rng, (1, d))
+    W = np.repeat(w, V, axis=0)
+    H = _rand_bits(rng, (5, d))
+    M = np.ones((1, 5), np.uint8)
+    out = o.oracle_rows(H, W, M)
+    z = o.bf16_bits_to_f64(H) @ o.bf16_bits_to_f64(w)[0]
+    assert out["tok"].tolist() == [0] * 5
+    np.testing.assert_allclose(out["conf"], 1.0 / V, rtol=1e-13)
+    np.testing.assert_allclose(out["lse"], z + math.log(V), rtol=1e-13, atol=1e-13)
+    # (2) W = [I_d; 0], H = c e_j -> tok j, lse = log(e^c + V - 1), conf = e^c / (e^c + V - 1)
+    d, V = 8, 20
+    Wf = np.zeros((V, d), np.float32)
+    Wf[:d, :d] = np.eye(d)
+    for j, c in [(0, 3.0), (5, 1.5), (7, 8.0), (3, 0.25)]:
+        Hf = np.zeros((1, d), np.float32)
+        Hf[0, j] = c
+        out = o.oracle_rows(_bits(Hf), _bits(Wf), np.ones((1, 1), np.uint8))
+        assert out["tok"].tolist() == [j]
+        np.testing.assert_allclose(out["lse"], [math.log(math.exp(c) + V - 1)], rtol=1e-14)
+        np.testing.assert_allclose(out["conf"], [math.exp(c) / (math.exp(c) + V - 1)], rtol=1e-14)
+    # (3) V = 1 -> conf 1, lse = the single logit, tok 0
+    H = _rand_bits(rng, (4, 8))
+    W = _rand_bits(rng, (1, 8))
+    out = o.oracle_rows(H, W, np.ones((1, 4), np.uint8))
+    np.testing.assert_allclose(out["conf"], 1.0, rtol=0, atol=0)
+    np.testing.assert_allclose(out["lse"], o.bf16_bits_to_f64(H) @ o.bf16_bits_to_f64(W)[0],
+                               rtol=1e-15)
+    assert out["tok"].tolist() == [0] * 4
+
+
+def check_library_routines(o):
+    """lse against scipy.special.logsumexp, conf against max of scipy.special.softmax,
+    tok against torch.argmax, the bf16 decoding against torch's bf16 -> float64 cast."""
+    rng = np.random.default_rng(11)
+    H, W = _rand_bits(rng, (24, 64)), _rand_bits(rng, (300, 64), 0.3)
+    M = np.ones((2, 12), np.uint8)
+    out = o.oracle_rows(H, W, M)
+    Ht = torch.from_numpy(H.view(np.int16)).view(torch.bfloat16).double()
+    Wt = torch.from_numpy(W.view(np.int16)).view(torch.bfloat16).double()
+    np.testing.assert_array_equal(o.bf16_bits_to_f64(H), Ht.numpy())
+    Z = (Ht @ Wt.T).numpy()
+    np.testing.assert_allclose(out["lse"], scipy.special.logsumexp(Z, axis=1), rtol=1e-12)
+    np.testing.assert_allclose(out["conf"], scipy.special.softmax(Z, axis=1).max(axis=1),
+                               rtol=1e-12)
+    assert out["tok"].tolist() == torch.argmax(torch.from_numpy(Z), dim=1).tolist()
+
+
+def check_invariants(o):
+    rng = np.random.default_rng(5)
+    H, W = _rand_bits(rng, (64, 32)), _rand_bits(rng, (500, 32), 0.5)
+    M = (rng.random((2, 32)) < 0.5).astype(np.uint8)
+    out = o.oracle_rows(H, W, M)
+    V = W.shape[0]
+    conf, m, lse = out["conf"], out["m"], out["lse"]
+    assert np.all(conf >= 1.0 / V * (1 - 1e-12)) and np.all(conf <= 1.0 + 1e-15)
+    assert np.all(m <= lse + 1e-12) and np.all(lse <= m + math.log(V) + 1e-12)
+    Z = o.bf16_bits_to_f64(H[out["row_idx"]]) @ o.bf16_bits_to_f64(W).T
+    np.testing.assert_allclose(np.exp(Z - lse[:, None]).sum(axis=1), 1.0, rtol=1e-12)
+    np.testing.assert_allclose(conf * np.exp(Z - m[:, None]).sum(axis=1), 1.0, rtol=1e-12)
+    np.testing.assert_array_equal(m, Z.max(axis=1))
+
+
+def check_mask_only_equals_full(o):
+    rng = np.random.default_rng(9)
+    for B, L, d, V in [(1, 40, 16, 70), (3, 9, 8, 33)]:
+        H, W = _rand_bits(rng, (B * L, d)), _rand_bits(rng, (V, d))
+        M = (rng.random((B, L)) < 0.5).astype(np.uint8)
+        a = o.oracle_rows(H, W, M)
+        b = o.full_then_gather(H, W, M)
+        for key in ("tok", "m", "lse", "conf"):
+            np.testing.assert_array_equal(a[key], b[key])
+
+
+def check_merge_split_invariance(o):
+    rng = np.random.default_rng(13)
+    Z = rng.standard_normal((20, 257)) * 3
+    Z[3, 10] = Z[3, 200] = Z[3].max() + 1.0        # an exact tie across splits
+    tok0, m0, lse0, conf0 = o.row_stats(Z)
+    V = Z.shape[1]
+    for n_split in (1, 2, 3, 7, 64, 257):
+        cuts = np.sort(rng.choice(np.arange(1, V), size=n_split - 1, replace=False))
+        bounds = np.concatenate([[0], cuts, [V]])
+        parts = [o.partial_stats(Z, int(a), int(b)) for a, b in zip(bounds[:-1], bounds[1:])]
+        tok, m, lse, conf = o.lse_merge(parts)
+        assert tok.tolist() == tok0.tolist()
+        np.testing.assert_array_equal(m, m0)
+        np.testing.assert_allclose(lse, lse0, rtol=1e-13)
+        np.testing.assert_allclose(conf, conf0, rtol=1e-12)
+    assert tok0[3] == 10
+
+
+ALL_CHECKS = [check_handworked, check_topk_ties, check_compact, check_brute_random,
+              check_closed_forms, check_library_routines, check_invariants,
+              check_mask_only_equals_full, check_merge_split_invariance]
