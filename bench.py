@@ -1,0 +1,353 @@
+"""Benchmark of the diffusion-LLM decode step: mask-only logits + confidence unmasking.
+
+One step = the whole hot path on one batch: mask compaction, masked-row gather, the
+tensor-core LM head with the fused softmax-statistics epilogue, lse_merge and the
+per-sequence top-k unmask selection (``dllm_decode_step``).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config cfg1] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0).  ``value`` = masked rows per second over the whole job
+(device time, inputs resident in HBM); ``e2e`` = the same through ``DecodeStep.run_host``
+with the step's H and mask copied from pinned host memory and the selection copied back,
+every step.  Under torchrun each rank runs its own replica of the workload (weak scaling,
+no data-path collective): the decode steps of independent batches share nothing.
+``--impl reference`` times the fp64 CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads as WL  # noqa: E402
+
+METRIC = "masked rows/sec & TFLOP/s (frac of roofline) for mask-only logits+unmask"
+UNIT = "masked_rows/s"
+
+
+def load_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return dict(hbm_gbs=p["hbm_gbs"], bf16_tflops=p["bf16_tflops"],
+                    bf16_tflops_sustained=p.get("bf16_tflops_sustained"), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def algorithmic(cfg, M: int) -> dict:
+    """Work of one step: flops of the dense contraction and bytes that must move once."""
+    flops = 2.0 * M * cfg.V * cfg.d
+    bytes_ = (2.0 * cfg.V * cfg.d          # W once
+              + 2.0 * M * cfg.d            # masked rows of H once
+              + cfg.B * cfg.L              # mask
+              + 12.0 * M                   # tok, conf, lse
+              + 4.0 * cfg.B * (2 * cfg.k + 1))   # idx, tok_sel, n_sel
+    return dict(flops=flops, bytes=bytes_)
+
+
+def roofline_s(cfg, M: int, peaks: dict) -> float:
+    a = algorithmic(cfg, M)
+    return max(a["flops"] / (peaks["bf16_tflops"] * 1e12), a["bytes"] / (peaks["hbm_gbs"] * 1e9))
+
+
+# ------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, period_ms: int = 100):
+        self.gpu = gpu_index
+        self.period = period_ms
+        self.proc = None
+        self.lines: list[str] = []
+        self._t = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", f"-lms={self.period}"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self._t is not None:
+                self._t.join(timeout=5)
+
+    def summary(self) -> dict:
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, flag in zip(names, parts[5:9]):
+                if flag.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=[], samples=0)
+        return dict(sm_mhz=statistics.median(sm), sm_max_mhz=max(mx), reasons=sorted(reasons),
+                    samples=len(sm))
+
+
+# ---------------------------------------------------------------------------- oracle leg
+def oracle_rate(inp: dict, rows: np.ndarray) -> tuple[float, float]:
+    """Seconds the fp64 oracle takes for the given compacted rows (logits statistics) plus
+    the unmask selection over them; returns (seconds, rows)."""
+    import oracle.oracle as O
+    Hb, Wb, M = WL.bf16_bits(inp["H"]), WL.bf16_bits(inp["W"]), inp["M"].numpy()
+    row_idx, seq_off, count = O.mask_compact(M)
+    t0 = time.perf_counter()
+    ref = O.rows_stats_chunked(Hb[row_idx[rows]], Wb)
+    O.select_unmask(ref[3], row_idx[rows], np.array([0, rows.size]), M.shape[1], inp["k"])
+    return time.perf_counter() - t0, float(rows.size)
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max((i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"), default=1)
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(inp: dict, budget_s: float = 12.0) -> dict:
+    cfg = inp["cfg"]
+    count = int(inp["M"].sum())
+    rng = np.random.default_rng(0)
+    t, n = oracle_rate(inp, np.sort(rng.choice(count, size=min(count, 16), replace=False)))
+    per_row = t / n
+    n_rows = int(max(16, min(count, budget_s / max(per_row, 1e-6))))
+    rows = np.sort(rng.choice(count, size=n_rows, replace=False))
+    t, n = oracle_rate(inp, rows)
+    return dict(value=n / t, unit=UNIT, cores=blas_threads(), kind="oracle",
+                sample=f"{n_rows} of {count} masked rows of {cfg.name} (fp64 NumPy logits over all "
+                       f"V={cfg.V}, statistics, top-k over the sample), {t:.1f} s")
+
+
+def run_reference(args, cfg) -> None:
+    """The oracle as the reference arm: rank 0 only, on the host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    inp = WL.make_inputs(cfg, seed=0)
+    count = int(inp["M"].sum())
+    rng = np.random.default_rng(0)
+    t, n = oracle_rate(inp, np.sort(rng.choice(count, size=min(count, 8), replace=False)))
+    per_row = t / n
+    # size each step so that warmup + steps take about two minutes in total
+    per_step = 120.0 / max(1, args.steps + args.warmup)
+    rows_per_step = int(max(1, min(count, per_step / max(per_row, 1e-6))))
+    for _ in range(args.warmup):
+        oracle_rate(inp, np.sort(rng.choice(count, size=rows_per_step, replace=False)))
+    tot_t, tot_n = 0.0, 0.0
+    for _ in range(args.steps):
+        t, n = oracle_rate(inp, np.sort(rng.choice(count, size=rows_per_step, replace=False)))
+        tot_t += t
+        tot_n += n
+    value = tot_n / tot_t
+    line = dict(metric=METRIC, value=value, unit=UNIT, n_gpus=args.gpus, steps=args.steps,
+                warmup=args.warmup, ms_per_step=1e3 * tot_t / args.steps, higher_is_better=True,
+                scaling="weak", vs_baseline=None, dtype="f64", data="synthetic", impl="reference",
+                config=workload_config(cfg, count),
+                cpu_baseline=dict(value=value, unit=UNIT, cores=blas_threads(), kind="oracle",
+                                  sample=f"{rows_per_step} random masked rows per step of {cfg.name}"),
+                e2e=dict(value=value, unit=UNIT, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(cfg, count: int) -> dict:
+    return dict(workload=f"{cfg.name}: {cfg.description}", B=cfg.B, L=cfg.L, d=cfg.d, V=cfg.V,
+                k=cfg.k, masked_rows=count,
+                l2="inputs larger than L2: W (%.2f GB) is streamed every step" % (2 * cfg.V * cfg.d / 1e9)
+                if 2 * cfg.V * cfg.d > 126e6 else "L2-resident inputs (no flush)",
+                parallelism="one independent replica per GPU")
+
+
+# ------------------------------------------------------------------------------ our arm
+def main() -> None:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="cfg1")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    cfg = WL.CONFIGS[args.config]
+
+    if args.impl == "reference":
+        run_reference(args, cfg)
+        return
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    # inputs (each rank its own seeded batch), and the oracle baseline before any GPU work
+    inp = WL.make_inputs(cfg, seed=rank)
+    count = int(inp["M"].sum())
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(inp)
+
+    import mask_only_logits_b200 as dl
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    H = inp["H"].to(dev)
+    M = inp["M"].to(dev)
+    W = inp["W"].to(dev)
+    win_lo = None if inp["win_lo"] is None else torch.from_numpy(inp["win_lo"]).to(dev)
+    win_hi = None if inp["win_hi"] is None else torch.from_numpy(inp["win_hi"]).to(dev)
+    torch.cuda.reset_peak_memory_stats(dev)
+    base_mem = torch.cuda.memory_allocated(dev)
+    step = dl.DecodeStep(cfg.B, cfg.L, cfg.d, cfg.V, cfg.k, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(args.warmup):
+        step.run(H, M, W, win_lo, win_hi, stream)
+    torch.cuda.synchronize(dev)
+    status = dl.get_status(stream)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after warm-up")
+    step_peak = torch.cuda.max_memory_allocated(dev) - base_mem
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    # ---- device-resident timed region ----
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        barrier()
+        dl.prof_begin()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step.run(H, M, W, win_lo, win_hi, stream)
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        gemm_ms, gemm_launches, launches = dl.prof_end()
+        barrier()
+    t_ms = ev0.elapsed_time(ev1)
+    status = dl.get_status(stream)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+    if dist is not None:
+        tt = torch.tensor([t_ms, gemm_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_ms, gemm_ms = float(tt[0]), float(tt[1])
+
+    # ---- end to end from pinned host memory ----
+    e2e_steps = args.e2e_steps or max(10, min(args.steps, 200))
+    H_host = inp["H"].pin_memory()
+    M_host = inp["M"].pin_memory()
+    for _ in range(3):
+        step.run_host(H_host, M_host, W, win_lo, win_hi, stream)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        step.run_host(H_host, M_host, W, win_lo, win_hi, stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    if dist is not None:
+        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt[0])
+        barrier()
+
+    if rank == 0:
+        peaks = load_peaks()
+        a = algorithmic(cfg, count)
+        ms_step = t_ms / args.steps
+        rows_s = count * world * args.steps / (t_ms / 1e3)
+        gemm_avg_s = gemm_ms / max(1, gemm_launches) / 1e3
+        tflops_gemm = a["flops"] / gemm_avg_s / 1e12
+        roof = roofline_s(cfg, count, peaks)
+        step_tflops = a["flops"] / (ms_step / 1e3) / 1e12
+        step_gbs = a["bytes"] / (ms_step / 1e3) / 1e9
+        full_logits = cfg.B * cfg.L * cfg.V * 4
+        line = dict(
+            metric=METRIC, value=rows_s, unit=UNIT, n_gpus=world, steps=args.steps,
+            warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True, scaling="weak",
+            vs_baseline=None, dtype="bf16", data="synthetic",
+            config=workload_config(cfg, count),
+            tflops=step_tflops, gbs=step_gbs,
+            roofline_frac_step=roof / (ms_step / 1e3),
+            roofline_ms=roof * 1e3,
+            roofline=dict(bound="tensor" if a["flops"] / (peaks["bf16_tflops"] * 1e12) >=
+                          a["bytes"] / (peaks["hbm_gbs"] * 1e9) else "hbm",
+                          kernel="masked_lmhead (lmhead_kernel)",
+                          achieved=tflops_gemm, peak=peaks["bf16_tflops"], unit="TFLOP/s",
+                          frac=tflops_gemm / peaks["bf16_tflops"],
+                          frac_of_sustained=(tflops_gemm / peaks["bf16_tflops_sustained"]
+                                             if peaks.get("bf16_tflops_sustained") else None),
+                          peak_source=peaks["source"] + " (burst bf16 GEMM)",
+                          gemm_ms_avg=gemm_avg_s * 1e3, traffic=None),
+            gpu_launches=launches,
+            memory=dict(peak_step_bytes=int(step_peak),
+                        full_logits_fp32_bytes=int(full_logits),
+                        note="peak = torch allocations of the step (outputs + workspace) over the "
+                             "resident inputs; the full-logits baseline is B*L*V fp32 logits, "
+                             "analytic"),
+            e2e=dict(value=count * world * e2e_steps / (e2e_ms / 1e3), unit=UNIT,
+                     h2d_bytes_per_step=step.h2d_bytes(), d2h_bytes_per_step=step.d2h_bytes(),
+                     ms_per_step=e2e_ms / e2e_steps),
+            clocks=clk.summary(),
+        )
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

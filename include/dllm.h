@@ -1,0 +1,206 @@
+/*
+ * dllm.h - C ABI of the mask-only logits + confidence-unmasking decode step for B200 (sm_100a).
+ *
+ * One denoising step of a diffusion LLM takes hidden states H[B*L, d] and a mask M[B, L]
+ * (nonzero = the position still holds [MASK]).  The Mosaic page ("Mosaic: Unlocking
+ * Long-Context Inference for Diffusion LLMs via Global Memory Planning and Dynamic Peak
+ * Taming", TL;DR and Abstract) builds a mask-only logits kernel: the LM head is applied to
+ * the masked rows only, so the [L, V] logits tensor of a plain implementation is never
+ * needed.  This library
+ *   1. compacts the masked positions with a prefix sum            (dllm_mask_compact),
+ *   2. multiplies only those rows by the vocabulary projection W[V, d] on the tensor cores
+ *      and reduces every row to (predicted token, log-sum-exp, confidence) in the GEMM
+ *      epilogue, without ever storing a logit                       (dllm_masked_logits),
+ *   3. picks, per sequence, the k most confident masked positions to unmask
+ *      (confidence-driven unmasking, dLLM inference survey page, "Main Findings";
+ *      an optional per-sequence window restricts candidates to the current
+ *      semi-autoregressive block, Sparse-dLLM page, "Experiment")  (dllm_select_unmask).
+ *
+ * Conventions for every call:
+ *   - Pointers marked "device" must point to memory of the current CUDA device; the caller
+ *     owns every buffer.  The library never allocates device memory: scratch space is the
+ *     caller's workspace, sized by dllm_workspace_bytes().
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  All
+ *     work is enqueued asynchronously on it; no call synchronises the host except
+ *     dllm_get_status() and dllm_prof_end().
+ *   - Arguments are validated on the host before anything is launched; an invalid call
+ *     returns a negative status and enqueues nothing.
+ *   - Errors detected on the device (a wait that gave up, a failed bound check) are
+ *     recorded in a per-device status word; dllm_get_status() reports and clears it.
+ *   - bf16 tensors are passed as their raw 16-bit patterns (uint16_t).
+ *   - Device pointers must be 16-byte aligned.
+ */
+#ifndef DLLM_H
+#define DLLM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t dllm_status;
+
+#define DLLM_OK              0
+#define DLLM_ERR_NULL       -1   /* a required pointer is NULL                              */
+#define DLLM_ERR_ALIGN      -2   /* a device pointer is not 16-byte aligned                 */
+#define DLLM_ERR_SHAPE      -3   /* B, L, d, V or k out of range (see each call)            */
+#define DLLM_ERR_WORKSPACE  -4   /* workspace smaller than dllm_workspace_bytes()           */
+#define DLLM_ERR_CUDA       -5   /* a CUDA runtime/driver call failed                       */
+#define DLLM_ERR_TIMEOUT    -6   /* a device-side wait exceeded its limit (kernel returned) */
+#define DLLM_ERR_DEVICE     -7   /* the current device is not an sm_100 GPU                 */
+#define DLLM_ERR_BOUNDS     -8   /* a device-side bound check failed (access skipped)       */
+
+/* Limits. */
+#define DLLM_MAX_K          1024 /* largest k accepted by dllm_select_unmask                */
+#define DLLM_D_MULTIPLE     64   /* d must be a positive multiple of this                   */
+
+/* Version of this ABI (major * 10000 + minor * 100 + patch). */
+int32_t dllm_version(void);
+
+/* Human-readable text for a status code (static storage; never NULL). */
+const char* dllm_status_string(dllm_status s);
+
+/*
+ * Workspace size in bytes for a step with these shapes: an upper bound that does not depend
+ * on how many positions are masked.  It covers the compaction tile counts, the gathered
+ * masked hidden rows (B*L*d bf16 at most) and the per-row vocabulary-split partials.
+ * Returns 0 if the shapes are invalid (B, L, d, V < 1, d % 64 != 0 or B*L >= 2^31).
+ * Needs no GPU.
+ */
+size_t dllm_workspace_bytes(int32_t B, int32_t L, int32_t d, int32_t V);
+
+/*
+ * dllm_mask_compact - prefix-sum compaction of the mask (Mosaic page, Abstract: logits are
+ * computed for masked positions only).
+ *
+ *   M        device, uint8 [B, L] row-major; nonzero = masked.
+ *   row_idx  device, int32 [B*L] capacity; on return row_idx[0:count] holds the flattened
+ *            positions b*L + l of the masked entries in ascending order.  Entries at and
+ *            past `count` are left untouched.
+ *   seq_off  device, int32 [B + 1]; seq_off[b] = number of masked positions in sequences
+ *            0..b-1, so sequence b owns compacted rows seq_off[b] .. seq_off[b+1]-1.
+ *   count    device, int32 [1]; the number of masked positions.  It stays on the device:
+ *            later calls size their work from it without a host round trip.
+ *   ws       device workspace of at least dllm_workspace_bytes(B, L, 64, 1) bytes.
+ * Errors: DLLM_ERR_NULL, DLLM_ERR_ALIGN (M, row_idx, seq_off, ws), DLLM_ERR_SHAPE
+ * (B < 1, L < 1, B*L >= 2^31), DLLM_ERR_WORKSPACE, DLLM_ERR_CUDA, DLLM_ERR_DEVICE.
+ */
+dllm_status dllm_mask_compact(const uint8_t* M, int32_t B, int32_t L,
+                              int32_t* row_idx, int32_t* seq_off, int32_t* count,
+                              void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * dllm_masked_logits - mask-only LM head with a fused online softmax epilogue (Mosaic page,
+ * TL;DR and Abstract: the mask-only logits kernel).
+ *
+ * Runs dllm_mask_compact on M, gathers the masked rows of H, and computes for every masked
+ * row i (in compacted order, i < count):
+ *     z_v    = sum_k H[row_idx[i], k] * W[v, k]          (bf16 inputs, fp32 accumulation)
+ *     tok[i] = the smallest v with z_v = max_v z_v
+ *     lse[i] = log sum_v exp(z_v)                        (natural log)
+ *     conf[i]= exp(max_v z_v - lse[i])                   (largest softmax probability)
+ * No logit is ever written to memory: the GEMM epilogue keeps a running max, sum of
+ * exponentials and argmax per row over vocabulary tiles, and a merge kernel (lse_merge)
+ * combines the per-split partials.
+ *
+ *   H        device, bf16 [B*L, d] row-major.
+ *   M        device, uint8 [B, L] row-major.
+ *   W        device, bf16 [V, d] row-major (the vocabulary projection; no bias).
+ *   tok, conf, lse   device, int32 / float32 / float32, each of capacity B*L; entries
+ *            0..count-1 are written, the rest untouched.
+ *   row_idx, seq_off, count   device outputs exactly as in dllm_mask_compact.
+ *   ws       device workspace of at least dllm_workspace_bytes(B, L, d, V) bytes.
+ * Constraints: B, L, V >= 1; d a positive multiple of 64; B*L < 2^31; every pointer
+ * 16-byte aligned.  Errors: as dllm_mask_compact.
+ */
+dllm_status dllm_masked_logits(const uint16_t* H, const uint8_t* M, const uint16_t* W,
+                               int32_t B, int32_t L, int32_t d, int32_t V,
+                               int32_t* tok, float* conf, float* lse,
+                               int32_t* row_idx, int32_t* seq_off, int32_t* count,
+                               void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * dllm_select_unmask - per-sequence top-k over confidences (confidence-driven unmasking,
+ * dLLM inference survey page, "Main Findings").
+ *
+ * For each sequence b, the candidates are its masked positions l = row_idx[i] - b*L for
+ * i in [seq_off[b], seq_off[b+1]), restricted to win_lo[b] <= l < win_hi[b] when windows
+ * are given.  The k candidates of largest conf are selected, ordered by conf descending,
+ * then by position ascending (this order also breaks exact ties).
+ *
+ *   conf, row_idx, seq_off   device, as produced by dllm_masked_logits (compacted order).
+ *   win_lo, win_hi   device int32 [B] or both NULL (no window).
+ *   tok      device int32 (compacted order) or NULL.
+ *   idx      device int32 [B, k]: selected positions l in [0, L); -1 past n_sel[b].
+ *   n_sel    device int32 [B]: min(k, number of candidates of sequence b).
+ *   tok_sel  device int32 [B, k] or NULL: tok of each selected position (-1 padding);
+ *            requires tok.
+ *   conf_sel device float32 [B, k] or NULL: conf of each selected position (0 padding).
+ * Constraints: 1 <= k <= DLLM_MAX_K.  Errors: DLLM_ERR_NULL, DLLM_ERR_ALIGN,
+ * DLLM_ERR_SHAPE, DLLM_ERR_CUDA, DLLM_ERR_DEVICE.
+ */
+dllm_status dllm_select_unmask(const float* conf, const int32_t* row_idx,
+                               const int32_t* seq_off, int32_t B, int32_t L, int32_t k,
+                               const int32_t* win_lo, const int32_t* win_hi,
+                               const int32_t* tok,
+                               int32_t* idx, int32_t* n_sel,
+                               int32_t* tok_sel, float* conf_sel, void* stream);
+
+/*
+ * dllm_decode_step - the whole hot path in one call: dllm_masked_logits followed by
+ * dllm_select_unmask on the same stream.  Arguments as in those two calls.
+ */
+dllm_status dllm_decode_step(const uint16_t* H, const uint8_t* M, const uint16_t* W,
+                             int32_t B, int32_t L, int32_t d, int32_t V, int32_t k,
+                             const int32_t* win_lo, const int32_t* win_hi,
+                             int32_t* tok, float* conf, float* lse,
+                             int32_t* row_idx, int32_t* seq_off, int32_t* count,
+                             int32_t* idx, int32_t* n_sel, int32_t* tok_sel, float* conf_sel,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * dllm_get_status - synchronise `stream`, then return (and clear) the device-side status
+ * word of the current device: DLLM_OK, DLLM_ERR_TIMEOUT or DLLM_ERR_BOUNDS; DLLM_ERR_CUDA
+ * if the synchronisation itself failed.
+ */
+dllm_status dllm_get_status(void* stream);
+
+/*
+ * Test hook: run the tensor-core GEMM of dllm_masked_logits on already compacted inputs and
+ * store the raw fp32 logits instead of reducing them.  For small-shape tests only: the
+ * caller provides logits_out, float32 [B*L, V] capacity (rows 0..count-1 written).  The
+ * other arguments are as in dllm_masked_logits; row_idx/seq_off/count are outputs.
+ */
+dllm_status dllm_debug_lmhead_logits(const uint16_t* H, const uint8_t* M, const uint16_t* W,
+                                     int32_t B, int32_t L, int32_t d, int32_t V,
+                                     float* logits_out,
+                                     int32_t* row_idx, int32_t* seq_off, int32_t* count,
+                                     void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Test hook: the lse_merge step alone.  Partials are given per vocabulary split j and row i
+ * at index j * n_rows + i: running max m, sum of exp(z - m) s, and argmax a.  Writes tok,
+ * conf and lse for i < n_rows, merging splits 0..n_split-1 in order (lowest split wins a
+ * tie of maxima).
+ */
+dllm_status dllm_debug_lse_merge(const float* part_m, const float* part_s,
+                                 const int32_t* part_a, int32_t n_rows, int32_t n_split,
+                                 int32_t* tok, float* conf, float* lse, void* stream);
+
+/*
+ * Kernel-time accounting for benchmarks.  dllm_prof_begin() starts recording a CUDA event
+ * pair around every tensor-core GEMM launch and counting every kernel launch made by this
+ * library (all devices, all streams).  dllm_prof_end() synchronises those events, returns
+ * the summed GEMM time in milliseconds, the number of GEMM launches and the number of
+ * kernel launches since dllm_prof_begin(), and stops recording.  Not thread-safe.
+ */
+dllm_status dllm_prof_begin(void);
+dllm_status dllm_prof_end(double* gemm_ms, int32_t* gemm_launches, int32_t* kernel_launches);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DLLM_H */

@@ -1,0 +1,238 @@
+"""Mask-only logits + confidence unmasking for diffusion-LLM decoding on B200 (sm_100a).
+
+Python face of the C ABI in ``include/dllm.h``.  Every step of the path runs in the
+library's CUDA kernels; this module only turns torch tensors into pointers and picks the
+current CUDA stream.  PyTorch supplies device memory and streams.  There is no CPU
+fallback: if ``libdllm.so`` is missing, loading fails loudly.
+
+Low-level calls (same names and arguments as the C ABI, tensors instead of pointers):
+``workspace_bytes``, ``mask_compact``, ``masked_logits``, ``select_unmask``,
+``decode_step``, ``get_status``.  ``DecodeStep`` owns the buffers of one shape and runs a
+whole step on device tensors (``run``) or on host tensors with the copies included
+(``run_host``).
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _abi
+
+__all__ = [
+    "DllmError", "lib", "version", "workspace_bytes", "mask_compact", "masked_logits",
+    "select_unmask", "decode_step", "get_status", "debug_lmhead_logits", "debug_lse_merge",
+    "prof_begin", "prof_end", "DecodeStep", "MAX_K",
+]
+
+MAX_K = 1024
+
+STATUS = {0: "DLLM_OK", -1: "DLLM_ERR_NULL", -2: "DLLM_ERR_ALIGN", -3: "DLLM_ERR_SHAPE",
+          -4: "DLLM_ERR_WORKSPACE", -5: "DLLM_ERR_CUDA", -6: "DLLM_ERR_TIMEOUT",
+          -7: "DLLM_ERR_DEVICE", -8: "DLLM_ERR_BOUNDS"}
+
+
+class DllmError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib().dllm_status_string(status).decode()
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({msg})")
+
+
+def lib() -> ctypes.CDLL:
+    return _abi.load()
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise DllmError(status, where)
+
+
+def _ptr(t: torch.Tensor | None, dtype: torch.dtype | None = None, name: str = "") -> ctypes.c_void_p:
+    if t is None:
+        return ctypes.c_void_p(None)
+    if not t.is_cuda:
+        raise ValueError(f"{name}: expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name}: expected {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def version() -> int:
+    return int(lib().dllm_version())
+
+
+def workspace_bytes(B: int, L: int, d: int, V: int) -> int:
+    return int(lib().dllm_workspace_bytes(B, L, d, V))
+
+
+def mask_compact(M, row_idx, seq_off, count, ws, stream=None) -> None:
+    B, L = M.shape
+    _check(lib().dllm_mask_compact(_ptr(M, torch.uint8, "M"), B, L,
+                                   _ptr(row_idx, torch.int32, "row_idx"),
+                                   _ptr(seq_off, torch.int32, "seq_off"),
+                                   _ptr(count, torch.int32, "count"), _ptr(ws, None, "ws"),
+                                   ws.numel() * ws.element_size(), _stream(stream)),
+           "dllm_mask_compact")
+
+
+def masked_logits(H, M, W, tok, conf, lse, row_idx, seq_off, count, ws, stream=None) -> None:
+    B, L = M.shape
+    V, d = W.shape
+    _check(lib().dllm_masked_logits(
+        _ptr(H, torch.bfloat16, "H"), _ptr(M, torch.uint8, "M"), _ptr(W, torch.bfloat16, "W"),
+        B, L, d, V, _ptr(tok, torch.int32, "tok"), _ptr(conf, torch.float32, "conf"),
+        _ptr(lse, torch.float32, "lse"), _ptr(row_idx, torch.int32, "row_idx"),
+        _ptr(seq_off, torch.int32, "seq_off"), _ptr(count, torch.int32, "count"),
+        _ptr(ws, None, "ws"), ws.numel() * ws.element_size(), _stream(stream)),
+        "dllm_masked_logits")
+
+
+def select_unmask(conf, row_idx, seq_off, B, L, k, idx, n_sel, win_lo=None, win_hi=None,
+                  tok=None, tok_sel=None, conf_sel=None, stream=None) -> None:
+    _check(lib().dllm_select_unmask(
+        _ptr(conf, torch.float32, "conf"), _ptr(row_idx, torch.int32, "row_idx"),
+        _ptr(seq_off, torch.int32, "seq_off"), B, L, k, _ptr(win_lo, torch.int32, "win_lo"),
+        _ptr(win_hi, torch.int32, "win_hi"), _ptr(tok, torch.int32, "tok"),
+        _ptr(idx, torch.int32, "idx"), _ptr(n_sel, torch.int32, "n_sel"),
+        _ptr(tok_sel, torch.int32, "tok_sel"), _ptr(conf_sel, torch.float32, "conf_sel"),
+        _stream(stream)), "dllm_select_unmask")
+
+
+def decode_step(H, M, W, k, tok, conf, lse, row_idx, seq_off, count, idx, n_sel, ws,
+                win_lo=None, win_hi=None, tok_sel=None, conf_sel=None, stream=None) -> None:
+    B, L = M.shape
+    V, d = W.shape
+    _check(lib().dllm_decode_step(
+        _ptr(H, torch.bfloat16, "H"), _ptr(M, torch.uint8, "M"), _ptr(W, torch.bfloat16, "W"),
+        B, L, d, V, k, _ptr(win_lo, torch.int32, "win_lo"), _ptr(win_hi, torch.int32, "win_hi"),
+        _ptr(tok, torch.int32, "tok"), _ptr(conf, torch.float32, "conf"),
+        _ptr(lse, torch.float32, "lse"), _ptr(row_idx, torch.int32, "row_idx"),
+        _ptr(seq_off, torch.int32, "seq_off"), _ptr(count, torch.int32, "count"),
+        _ptr(idx, torch.int32, "idx"), _ptr(n_sel, torch.int32, "n_sel"),
+        _ptr(tok_sel, torch.int32, "tok_sel"), _ptr(conf_sel, torch.float32, "conf_sel"),
+        _ptr(ws, None, "ws"), ws.numel() * ws.element_size(), _stream(stream)),
+        "dllm_decode_step")
+
+
+def get_status(stream=None) -> int:
+    return int(lib().dllm_get_status(_stream(stream)))
+
+
+def debug_lmhead_logits(H, M, W, logits_out, row_idx, seq_off, count, ws, stream=None) -> None:
+    B, L = M.shape
+    V, d = W.shape
+    _check(lib().dllm_debug_lmhead_logits(
+        _ptr(H, torch.bfloat16, "H"), _ptr(M, torch.uint8, "M"), _ptr(W, torch.bfloat16, "W"),
+        B, L, d, V, _ptr(logits_out, torch.float32, "logits_out"),
+        _ptr(row_idx, torch.int32, "row_idx"), _ptr(seq_off, torch.int32, "seq_off"),
+        _ptr(count, torch.int32, "count"), _ptr(ws, None, "ws"), ws.numel() * ws.element_size(),
+        _stream(stream)), "dllm_debug_lmhead_logits")
+
+
+def debug_lse_merge(part_m, part_s, part_a, tok, conf, lse, stream=None) -> None:
+    n_split, n_rows = part_m.shape
+    _check(lib().dllm_debug_lse_merge(
+        _ptr(part_m, torch.float32, "part_m"), _ptr(part_s, torch.float32, "part_s"),
+        _ptr(part_a, torch.int32, "part_a"), n_rows, n_split, _ptr(tok, torch.int32, "tok"),
+        _ptr(conf, torch.float32, "conf"), _ptr(lse, torch.float32, "lse"), _stream(stream)),
+        "dllm_debug_lse_merge")
+
+
+def prof_begin() -> None:
+    _check(lib().dllm_prof_begin(), "dllm_prof_begin")
+
+
+def prof_end() -> tuple[float, int, int]:
+    ms = ctypes.c_double(0.0)
+    g = ctypes.c_int32(0)
+    kcount = ctypes.c_int32(0)
+    _check(lib().dllm_prof_end(ctypes.byref(ms), ctypes.byref(g), ctypes.byref(kcount)),
+           "dllm_prof_end")
+    return ms.value, g.value, kcount.value
+
+
+class DecodeStep:
+    """Buffers for one decode-step shape (B, L, d, V, k) on one device, and the step itself.
+
+    Outputs are views into buffers owned by this object; their first ``count`` entries are
+    valid (``count`` stays on the device unless read).
+    """
+
+    def __init__(self, B: int, L: int, d: int, V: int, k: int, device="cuda"):
+        if k < 1 or k > MAX_K:
+            raise ValueError(f"k must be in [1, {MAX_K}]")
+        self.B, self.L, self.d, self.V, self.k = B, L, d, V, k
+        self.device = torch.device(device)
+        n = B * L
+        i32 = dict(dtype=torch.int32, device=self.device)
+        self.tok = torch.empty(n, **i32)
+        self.conf = torch.empty(n, dtype=torch.float32, device=self.device)
+        self.lse = torch.empty(n, dtype=torch.float32, device=self.device)
+        self.row_idx = torch.empty(n, **i32)
+        self.seq_off = torch.empty(B + 1, **i32)
+        self.count = torch.empty(4, **i32)          # 16 bytes: keeps the next buffer aligned
+        self.idx = torch.empty(B, k, **i32)
+        self.n_sel = torch.empty(B, **i32)
+        self.tok_sel = torch.empty(B, k, **i32)
+        self.conf_sel = torch.empty(B, k, dtype=torch.float32, device=self.device)
+        nbytes = workspace_bytes(B, L, d, V)
+        if nbytes == 0:
+            raise ValueError("invalid shapes (d must be a positive multiple of 64)")
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        self._host = None
+
+    def run(self, H, M, W, win_lo=None, win_hi=None, stream=None) -> dict:
+        decode_step(H, M, W, self.k, self.tok, self.conf, self.lse, self.row_idx, self.seq_off,
+                    self.count, self.idx, self.n_sel, self.ws, win_lo, win_hi, self.tok_sel,
+                    self.conf_sel, stream)
+        return dict(tok=self.tok, conf=self.conf, lse=self.lse, row_idx=self.row_idx,
+                    seq_off=self.seq_off, count=self.count[:1], idx=self.idx, n_sel=self.n_sel,
+                    tok_sel=self.tok_sel, conf_sel=self.conf_sel)
+
+    # -- end-to-end from host memory ---------------------------------------------------------
+    def _host_buffers(self):
+        if self._host is None:
+            B, L, d, k = self.B, self.L, self.d, self.k
+            pin = dict(pin_memory=True)
+            self._host = dict(
+                H=torch.empty(B * L, d, dtype=torch.bfloat16, device=self.device),
+                M=torch.empty(B, L, dtype=torch.uint8, device=self.device),
+                idx=torch.empty(B, k, dtype=torch.int32, **pin),
+                n_sel=torch.empty(B, dtype=torch.int32, **pin),
+                tok_sel=torch.empty(B, k, dtype=torch.int32, **pin),
+                conf_sel=torch.empty(B, k, dtype=torch.float32, **pin))
+        return self._host
+
+    def run_host(self, H_host, M_host, W, win_lo=None, win_hi=None, stream=None) -> dict:
+        """One step from pinned host H and M: copy them in, run, copy the selection back.
+
+        W (the resident vocabulary projection) and the windows are device tensors.  Returns
+        host tensors idx, n_sel, tok_sel, conf_sel; synchronises the stream.
+        """
+        hb = self._host_buffers()
+        s = stream if stream is not None else torch.cuda.current_stream()
+        with torch.cuda.stream(s):
+            hb["H"].copy_(H_host, non_blocking=True)
+            hb["M"].copy_(M_host, non_blocking=True)
+            self.run(hb["H"], hb["M"], W, win_lo, win_hi, s)
+            hb["idx"].copy_(self.idx, non_blocking=True)
+            hb["n_sel"].copy_(self.n_sel, non_blocking=True)
+            hb["tok_sel"].copy_(self.tok_sel, non_blocking=True)
+            hb["conf_sel"].copy_(self.conf_sel, non_blocking=True)
+        s.synchronize()
+        return dict(idx=hb["idx"], n_sel=hb["n_sel"], tok_sel=hb["tok_sel"], conf_sel=hb["conf_sel"])
+
+    def h2d_bytes(self) -> int:
+        return self.B * self.L * self.d * 2 + self.B * self.L
+
+    def d2h_bytes(self) -> int:
+        return self.B * self.k * 4 * 3 + self.B * 4

@@ -1,0 +1,52 @@
+"""ctypes declarations of the C ABI in include/dllm.h (argument marshalling only)."""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG_DIR, "libdllm.so")
+
+_p = ctypes.c_void_p
+_i32 = ctypes.c_int32
+_sz = ctypes.c_size_t
+_st = ctypes.c_int32
+
+# name -> (restype, argtypes); every symbol declared in include/dllm.h
+PROTOTYPES = {
+    "dllm_version": (_i32, []),
+    "dllm_status_string": (ctypes.c_char_p, [_st]),
+    "dllm_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32]),
+    "dllm_mask_compact": (_st, [_p, _i32, _i32, _p, _p, _p, _p, _sz, _p]),
+    "dllm_masked_logits": (_st, [_p, _p, _p, _i32, _i32, _i32, _i32, _p, _p, _p, _p, _p, _p,
+                                 _p, _sz, _p]),
+    "dllm_select_unmask": (_st, [_p, _p, _p, _i32, _i32, _i32, _p, _p, _p, _p, _p, _p, _p, _p]),
+    "dllm_decode_step": (_st, [_p, _p, _p, _i32, _i32, _i32, _i32, _i32, _p, _p, _p, _p, _p,
+                               _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
+    "dllm_get_status": (_st, [_p]),
+    "dllm_debug_lmhead_logits": (_st, [_p, _p, _p, _i32, _i32, _i32, _i32, _p, _p, _p, _p, _p,
+                                       _sz, _p]),
+    "dllm_debug_lse_merge": (_st, [_p, _p, _p, _i32, _i32, _p, _p, _p, _p]),
+    "dllm_prof_begin": (_st, []),
+    "dllm_prof_end": (_st, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i32),
+                            ctypes.POINTER(_i32)]),
+}
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libdllm.so from the package directory; raise if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m mask_only_logits_b200.build` "
+                "(there is no fallback implementation)")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in PROTOTYPES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib

@@ -1,0 +1,408 @@
+// dllm_api.cu - the C ABI (include/dllm.h): argument validation, workspace layout, TMA
+// tensor maps, launches on the caller's stream, device status word and kernel timing.
+//
+// All kernels are compiled in this one translation unit so that they share the device
+// status word without relocatable device code.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+#include <vector>
+
+#include "dllm.h"
+#include "ptx.cuh"
+#include "compact.cuh"
+#include "lmhead.cuh"
+#include "merge.cuh"
+#include "select.cuh"
+
+namespace dllm {
+
+// Device-side error bits (kStatusTimeout, kStatusBounds); one word per device.
+__device__ int g_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool ready = false;
+  dllm_status err = DLLM_OK;
+  int sms = 0;
+  int* status = nullptr;        // device address of g_status on this device
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+// Kernel-time accounting (dllm_prof_begin / dllm_prof_end).
+struct Prof {
+  bool on = false;
+  std::vector<cudaEvent_t> ev;  // pairs: start, stop
+  size_t used = 0;
+  int gemm_launches = 0;
+  std::atomic<int> kernel_launches{0};
+};
+Prof g_prof;
+
+inline void count_launch(int n = 1) {
+  if (g_prof.on) g_prof.kernel_launches += n;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Per-device setup, once: check the architecture, find g_status, raise the GEMM's shared
+// memory limit, resolve the tensor-map encoder.
+dllm_status device_state(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DLLM_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return DLLM_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState& st = g_dev[dev];
+  if (!st.ready) {
+    st.err = DLLM_OK;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) {
+      st.err = DLLM_ERR_CUDA;
+    } else if (prop.major != 10 || prop.minor != 0) {
+      st.err = DLLM_ERR_DEVICE;
+    } else {
+      st.sms = prop.multiProcessorCount;
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) st.err = DLLM_ERR_CUDA;
+      st.status = static_cast<int*>(p);
+      if (st.err == DLLM_OK &&
+          (cudaFuncSetAttribute(lm::lmhead_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                lm::SMEM_BYTES) != cudaSuccess ||
+           cudaFuncSetAttribute(lm::lmhead_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                lm::SMEM_BYTES) != cudaSuccess))
+        st.err = DLLM_ERR_CUDA;
+      if (st.err == DLLM_OK && g_encode == nullptr) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr)
+          st.err = DLLM_ERR_CUDA;
+        else
+          g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+      }
+    }
+    st.ready = true;
+  }
+  if (st.err != DLLM_OK) return st.err;
+  *out = &st;
+  return DLLM_OK;
+}
+
+// Workspace layout: [tile counts | gathered rows Hm | part_m | part_s | part_a].
+struct WsLayout {
+  size_t tiles_off, hm_off, pm_off, ps_off, pa_off, total;
+  long long part_cap;
+};
+
+WsLayout ws_layout(int B, int L, int d, int V) {
+  WsLayout w{};
+  const long long n = static_cast<long long>(B) * L;
+  const long long ntiles = (n + kCompactTile - 1) / kCompactTile;
+  // partial entries: worst case over the masked count (all positions masked) with the
+  // largest CTA count; fewer masked rows never need more.
+  const lm::Plan worst = lm::Plan::make(static_cast<int>(n), V, lm::kMaxCtas, lm::kGroupM);
+  long long cap = worst.ngroups * static_cast<long long>(lm::kMaxCtas) * lm::BM;
+  if (cap < 1) cap = 1;
+  w.part_cap = cap;
+  size_t off = 0;
+  w.tiles_off = off; off = round_up(off + sizeof(int) * ntiles, 256);
+  w.hm_off = off;    off = round_up(off + static_cast<size_t>(n) * d * 2, 256);
+  w.pm_off = off;    off = round_up(off + sizeof(float) * cap, 256);
+  w.ps_off = off;    off = round_up(off + sizeof(float) * cap, 256);
+  w.pa_off = off;    off = round_up(off + sizeof(int) * cap, 256);
+  w.total = off;
+  return w;
+}
+
+bool shapes_ok(int B, int L) {
+  return B >= 1 && L >= 1 && static_cast<long long>(B) * L < (1ll << 31);
+}
+
+dllm_status launch_compact(const uint8_t* M, int B, int L, int* row_idx, int* seq_off, int* count,
+                           int* tiles, int* status, cudaStream_t s) {
+  const long long n = static_cast<long long>(B) * L;
+  const unsigned ntiles = static_cast<unsigned>((n + kCompactTile - 1) / kCompactTile);
+  compact_count_kernel<<<ntiles, kCompactThreads, 0, s>>>(M, n, tiles);
+  compact_scatter_kernel<<<ntiles, kCompactThreads, 0, s>>>(M, B, L, tiles, row_idx, seq_off, count,
+                                                            status);
+  count_launch(2);
+  return cudaPeekAtLastError() == cudaSuccess ? DLLM_OK : DLLM_ERR_CUDA;
+}
+
+dllm_status make_tmap(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(lm::BK), box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DLLM_OK : DLLM_ERR_CUDA;
+}
+
+struct LogitsArgs {
+  const uint16_t* H; const uint8_t* M; const uint16_t* W;
+  int B, L, d, V;
+  int* tok; float* conf; float* lse; float* dbg;
+  int* row_idx; int* seq_off; int* count;
+  void* ws; size_t ws_bytes; cudaStream_t s;
+};
+
+dllm_status validate_logits(const LogitsArgs& a, bool debug) {
+  if (!a.H || !a.M || !a.W || !a.row_idx || !a.seq_off || !a.count || !a.ws) return DLLM_ERR_NULL;
+  if (!debug && (!a.tok || !a.conf || !a.lse)) return DLLM_ERR_NULL;
+  if (debug && !a.dbg) return DLLM_ERR_NULL;
+  if (!shapes_ok(a.B, a.L) || a.V < 1 || a.d < DLLM_D_MULTIPLE || a.d % DLLM_D_MULTIPLE != 0)
+    return DLLM_ERR_SHAPE;
+  const void* ptrs[] = {a.H, a.M, a.W, a.row_idx, a.seq_off, a.count, a.ws, a.tok, a.conf, a.lse, a.dbg};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return DLLM_ERR_ALIGN;
+  if (a.ws_bytes < ws_layout(a.B, a.L, a.d, a.V).total) return DLLM_ERR_WORKSPACE;
+  return DLLM_OK;
+}
+
+dllm_status run_logits(const LogitsArgs& a, bool debug) {
+  dllm_status st = validate_logits(a, debug);
+  if (st != DLLM_OK) return st;
+  DeviceState* ds = nullptr;
+  if ((st = device_state(&ds)) != DLLM_OK) return st;
+  const WsLayout w = ws_layout(a.B, a.L, a.d, a.V);
+  uint8_t* ws = static_cast<uint8_t*>(a.ws);
+  int* tiles = reinterpret_cast<int*>(ws + w.tiles_off);
+  uint16_t* Hm = reinterpret_cast<uint16_t*>(ws + w.hm_off);
+  float* pm = reinterpret_cast<float*>(ws + w.pm_off);
+  float* ps = reinterpret_cast<float*>(ws + w.ps_off);
+  int* pa = reinterpret_cast<int*>(ws + w.pa_off);
+  const long long n = static_cast<long long>(a.B) * a.L;
+
+  const int ctas = ds->sms < lm::kMaxCtas ? ds->sms : lm::kMaxCtas;
+  const lm::Plan worst = lm::Plan::make(static_cast<int>(n), a.V, ctas, lm::kGroupM);
+  if (worst.part_entries() > w.part_cap) return DLLM_ERR_WORKSPACE;   // cannot happen on B200
+
+  if ((st = launch_compact(a.M, a.B, a.L, a.row_idx, a.seq_off, a.count, tiles, ds->status, a.s)) != DLLM_OK)
+    return st;
+
+  gather_rows_kernel<<<ds->sms * 4, kGatherThreads, 0, a.s>>>(a.H, a.row_idx, a.count, n, a.d, Hm,
+                                                               ds->status);
+  count_launch();
+
+  CUtensorMap tmA, tmB;
+  if (make_tmap(&tmA, Hm, static_cast<uint64_t>(n), a.d, lm::BM) != DLLM_OK) return DLLM_ERR_CUDA;
+  if (make_tmap(&tmB, a.W, static_cast<uint64_t>(a.V), a.d, lm::BN) != DLLM_OK) return DLLM_ERR_CUDA;
+
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  if (g_prof.on) {
+    if (g_prof.used + 2 > g_prof.ev.size()) {
+      for (int i = 0; i < 64; ++i) {
+        cudaEvent_t e;
+        if (cudaEventCreate(&e) != cudaSuccess) return DLLM_ERR_CUDA;
+        g_prof.ev.push_back(e);
+      }
+    }
+    e0 = g_prof.ev[g_prof.used];
+    e1 = g_prof.ev[g_prof.used + 1];
+    g_prof.used += 2;
+    cudaEventRecord(e0, a.s);
+  }
+  if (debug)
+    lm::lmhead_kernel<true><<<ctas, lm::kThreads, lm::SMEM_BYTES, a.s>>>(
+        tmA, tmB, a.count, static_cast<int>(n), a.V, a.d, lm::kGroupM, pm, ps, pa, w.part_cap, a.dbg, ds->status);
+  else
+    lm::lmhead_kernel<false><<<ctas, lm::kThreads, lm::SMEM_BYTES, a.s>>>(
+        tmA, tmB, a.count, static_cast<int>(n), a.V, a.d, lm::kGroupM, pm, ps, pa, w.part_cap, nullptr, ds->status);
+  count_launch();
+  if (g_prof.on) {
+    cudaEventRecord(e1, a.s);
+    g_prof.gemm_launches++;
+  }
+  if (!debug) {
+    int mblocks = static_cast<int>((n + kMergeThreads - 1) / kMergeThreads);
+    if (mblocks > ds->sms * 8) mblocks = ds->sms * 8;
+    lse_merge_kernel<<<mblocks, kMergeThreads, 0, a.s>>>(a.count, static_cast<int>(n), a.V, ctas, lm::kGroupM, pm, ps, pa,
+                                                        a.tok, a.conf, a.lse);
+    count_launch();
+  }
+  return cudaPeekAtLastError() == cudaSuccess ? DLLM_OK : DLLM_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace dllm
+
+using namespace dllm;
+
+extern "C" {
+
+int32_t dllm_version(void) { return 10000; }
+
+const char* dllm_status_string(dllm_status s) {
+  switch (s) {
+    case DLLM_OK: return "ok";
+    case DLLM_ERR_NULL: return "a required pointer is NULL";
+    case DLLM_ERR_ALIGN: return "a device pointer is not 16-byte aligned";
+    case DLLM_ERR_SHAPE: return "shape out of range";
+    case DLLM_ERR_WORKSPACE: return "workspace too small";
+    case DLLM_ERR_CUDA: return "CUDA error";
+    case DLLM_ERR_TIMEOUT: return "a device-side wait timed out";
+    case DLLM_ERR_DEVICE: return "device is not an sm_100 GPU";
+    case DLLM_ERR_BOUNDS: return "a device-side bound check failed";
+    default: return "unknown status";
+  }
+}
+
+size_t dllm_workspace_bytes(int32_t B, int32_t L, int32_t d, int32_t V) {
+  if (!shapes_ok(B, L) || V < 1 || d < DLLM_D_MULTIPLE || d % DLLM_D_MULTIPLE != 0) return 0;
+  return ws_layout(B, L, d, V).total;
+}
+
+dllm_status dllm_mask_compact(const uint8_t* M, int32_t B, int32_t L, int32_t* row_idx,
+                              int32_t* seq_off, int32_t* count, void* ws, size_t ws_bytes,
+                              void* stream) {
+  if (!M || !row_idx || !seq_off || !count || !ws) return DLLM_ERR_NULL;
+  if (!shapes_ok(B, L)) return DLLM_ERR_SHAPE;
+  if (!aligned16(M) || !aligned16(row_idx) || !aligned16(seq_off) || !aligned16(count) || !aligned16(ws))
+    return DLLM_ERR_ALIGN;
+  const long long n = static_cast<long long>(B) * L;
+  const size_t need = sizeof(int) * static_cast<size_t>((n + kCompactTile - 1) / kCompactTile);
+  if (ws_bytes < need) return DLLM_ERR_WORKSPACE;
+  DeviceState* ds = nullptr;
+  dllm_status st = device_state(&ds);
+  if (st != DLLM_OK) return st;
+  return launch_compact(M, B, L, row_idx, seq_off, count, static_cast<int*>(ws), ds->status,
+                        static_cast<cudaStream_t>(stream));
+}
+
+dllm_status dllm_masked_logits(const uint16_t* H, const uint8_t* M, const uint16_t* W, int32_t B,
+                               int32_t L, int32_t d, int32_t V, int32_t* tok, float* conf,
+                               float* lse, int32_t* row_idx, int32_t* seq_off, int32_t* count,
+                               void* ws, size_t ws_bytes, void* stream) {
+  LogitsArgs a{H, M, W, B, L, d, V, tok, conf, lse, nullptr, row_idx, seq_off, count,
+               ws, ws_bytes, static_cast<cudaStream_t>(stream)};
+  return run_logits(a, false);
+}
+
+dllm_status dllm_debug_lmhead_logits(const uint16_t* H, const uint8_t* M, const uint16_t* W,
+                                     int32_t B, int32_t L, int32_t d, int32_t V, float* logits_out,
+                                     int32_t* row_idx, int32_t* seq_off, int32_t* count, void* ws,
+                                     size_t ws_bytes, void* stream) {
+  LogitsArgs a{H, M, W, B, L, d, V, nullptr, nullptr, nullptr, logits_out, row_idx, seq_off, count,
+               ws, ws_bytes, static_cast<cudaStream_t>(stream)};
+  return run_logits(a, true);
+}
+
+dllm_status dllm_select_unmask(const float* conf, const int32_t* row_idx, const int32_t* seq_off,
+                               int32_t B, int32_t L, int32_t k, const int32_t* win_lo,
+                               const int32_t* win_hi, const int32_t* tok, int32_t* idx,
+                               int32_t* n_sel, int32_t* tok_sel, float* conf_sel, void* stream) {
+  if (!conf || !row_idx || !seq_off || !idx || !n_sel) return DLLM_ERR_NULL;
+  if ((win_lo == nullptr) != (win_hi == nullptr)) return DLLM_ERR_NULL;
+  if (tok_sel && !tok) return DLLM_ERR_NULL;
+  if (!shapes_ok(B, L) || k < 1 || k > DLLM_MAX_K) return DLLM_ERR_SHAPE;
+  const void* ptrs[] = {conf, row_idx, seq_off, win_lo, win_hi, tok, idx, n_sel, tok_sel, conf_sel};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return DLLM_ERR_ALIGN;
+  DeviceState* ds = nullptr;
+  dllm_status st = device_state(&ds);
+  if (st != DLLM_OK) return st;
+  select_unmask_kernel<<<B, kSelThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      conf, row_idx, seq_off, B * L, L, k, win_lo, win_hi, tok, idx, n_sel, tok_sel, conf_sel);
+  count_launch();
+  return cudaPeekAtLastError() == cudaSuccess ? DLLM_OK : DLLM_ERR_CUDA;
+}
+
+dllm_status dllm_decode_step(const uint16_t* H, const uint8_t* M, const uint16_t* W, int32_t B,
+                             int32_t L, int32_t d, int32_t V, int32_t k, const int32_t* win_lo,
+                             const int32_t* win_hi, int32_t* tok, float* conf, float* lse,
+                             int32_t* row_idx, int32_t* seq_off, int32_t* count, int32_t* idx,
+                             int32_t* n_sel, int32_t* tok_sel, float* conf_sel, void* ws,
+                             size_t ws_bytes, void* stream) {
+  // validate the selection's own arguments first so that nothing is launched on error
+  if (!idx || !n_sel) return DLLM_ERR_NULL;
+  if ((win_lo == nullptr) != (win_hi == nullptr)) return DLLM_ERR_NULL;
+  if (k < 1 || k > DLLM_MAX_K) return DLLM_ERR_SHAPE;
+  const void* ptrs[] = {win_lo, win_hi, idx, n_sel, tok_sel, conf_sel};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return DLLM_ERR_ALIGN;
+  dllm_status st = dllm_masked_logits(H, M, W, B, L, d, V, tok, conf, lse, row_idx, seq_off, count,
+                                      ws, ws_bytes, stream);
+  if (st != DLLM_OK) return st;
+  return dllm_select_unmask(conf, row_idx, seq_off, B, L, k, win_lo, win_hi, tok, idx, n_sel,
+                            tok_sel, conf_sel, stream);
+}
+
+dllm_status dllm_debug_lse_merge(const float* part_m, const float* part_s, const int32_t* part_a,
+                                 int32_t n_rows, int32_t n_split, int32_t* tok, float* conf,
+                                 float* lse, void* stream) {
+  if (!part_m || !part_s || !part_a || !tok || !conf || !lse) return DLLM_ERR_NULL;
+  if (n_rows < 1 || n_split < 1) return DLLM_ERR_SHAPE;
+  const void* ptrs[] = {part_m, part_s, part_a, tok, conf, lse};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return DLLM_ERR_ALIGN;
+  DeviceState* ds = nullptr;
+  dllm_status st = device_state(&ds);
+  if (st != DLLM_OK) return st;
+  int blocks = (n_rows + kMergeThreads - 1) / kMergeThreads;
+  if (blocks > ds->sms * 8) blocks = ds->sms * 8;
+  lse_merge_plain_kernel<<<blocks, kMergeThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      part_m, part_s, part_a, n_rows, n_split, tok, conf, lse);
+  count_launch();
+  return cudaPeekAtLastError() == cudaSuccess ? DLLM_OK : DLLM_ERR_CUDA;
+}
+
+dllm_status dllm_get_status(void* stream) {
+  DeviceState* ds = nullptr;
+  dllm_status st = device_state(&ds);
+  if (st != DLLM_OK) return st;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DLLM_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return DLLM_ERR_CUDA;
+  const int zero = 0;
+  if (v != 0 && cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return DLLM_ERR_CUDA;
+  if (v & kStatusTimeout) return DLLM_ERR_TIMEOUT;
+  if (v & kStatusBounds) return DLLM_ERR_BOUNDS;
+  return DLLM_OK;
+}
+
+dllm_status dllm_prof_begin(void) {
+  g_prof.on = true;
+  g_prof.used = 0;
+  g_prof.gemm_launches = 0;
+  g_prof.kernel_launches = 0;
+  return DLLM_OK;
+}
+
+dllm_status dllm_prof_end(double* gemm_ms, int32_t* gemm_launches, int32_t* kernel_launches) {
+  double total = 0.0;
+  dllm_status st = DLLM_OK;
+  for (size_t i = 0; i + 1 < g_prof.used; i += 2) {
+    if (cudaEventSynchronize(g_prof.ev[i + 1]) != cudaSuccess) { st = DLLM_ERR_CUDA; break; }
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, g_prof.ev[i], g_prof.ev[i + 1]) != cudaSuccess) { st = DLLM_ERR_CUDA; break; }
+    total += ms;
+  }
+  if (gemm_ms) *gemm_ms = total;
+  if (gemm_launches) *gemm_launches = g_prof.gemm_launches;
+  if (kernel_launches) *kernel_launches = g_prof.kernel_launches;
+  g_prof.on = false;
+  g_prof.used = 0;
+  return st;
+}
+
+}  // extern "C"

@@ -1,0 +1,100 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every symbol that
+include/dllm.h declares, and rejects invalid arguments on the host before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mask_only_logits_b200 import _abi, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dllm.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()                       # no-op when libdllm.so is up to date
+    return _abi.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)          # drop comments
+    return sorted(set(re.findall(r"\b(dllm_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_and_bindings_agree():
+    assert declared_functions() == sorted(_abi.PROTOTYPES)
+
+
+def test_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    # and nothing but C symbols: the names are not mangled
+    nm = os.popen(f"nm -D --defined-only {_abi.LIB_PATH}").read()
+    exported = set(re.findall(r"\bT (dllm_\w+)", nm))
+    assert set(declared_functions()) <= exported
+
+
+def test_version_and_status_strings(lib):
+    assert lib.dllm_version() == 10000
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8):
+        assert lib.dllm_status_string(code)
+    assert lib.dllm_status_string(-99) == b"unknown status"
+
+
+def test_workspace_bytes(lib):
+    ws = lib.dllm_workspace_bytes
+    assert ws(1, 256, 256, 4096) > 256 * 256 * 2
+    # grows with B*L*d (the gathered rows dominate), never shrinks with more rows
+    assert ws(1, 4096, 4096, 126464) >= 4096 * 4096 * 2
+    assert ws(1, 131072, 4096, 126464) >= 131072 * 4096 * 2
+    assert ws(8, 8192, 2048, 151936) >= 8 * 8192 * 2048 * 2
+    # invalid shapes -> 0
+    assert ws(0, 10, 64, 10) == 0
+    assert ws(1, 0, 64, 10) == 0
+    assert ws(1, 10, 100, 10) == 0           # d not a multiple of 64
+    assert ws(1, 10, 64, 0) == 0
+    assert ws(1 << 16, 1 << 15, 64, 10) == 0  # B*L >= 2^31
+
+
+def _p(x):
+    return ctypes.c_void_p(x)
+
+
+def test_host_validation_without_gpu(lib):
+    """Every rejection happens before any CUDA call, so it works on a CPU-only machine."""
+    a = 1 << 20                                    # a 16-byte aligned fake address
+    nul = _p(None)
+    # mask_compact
+    assert lib.dllm_mask_compact(nul, 1, 8, _p(a), _p(a), _p(a), _p(a), 1 << 20, nul) == -1
+    assert lib.dllm_mask_compact(_p(a), 0, 8, _p(a), _p(a), _p(a), _p(a), 1 << 20, nul) == -3
+    assert lib.dllm_mask_compact(_p(a + 1), 1, 8, _p(a), _p(a), _p(a), _p(a), 1 << 20, nul) == -2
+    assert lib.dllm_mask_compact(_p(a), 1, 8, _p(a), _p(a), _p(a), _p(a), 0, nul) == -4
+    # masked_logits
+    args = [_p(a), _p(a), _p(a), 1, 256, 256, 4096, _p(a), _p(a), _p(a), _p(a), _p(a), _p(a)]
+    assert lib.dllm_masked_logits(*args, _p(a), 10, nul) == -4             # workspace too small
+    bad_d = list(args)
+    bad_d[5] = 100
+    assert lib.dllm_masked_logits(*bad_d, _p(a), 1 << 30, nul) == -3
+    bad_al = list(args)
+    bad_al[2] = _p(a + 8)
+    assert lib.dllm_masked_logits(*bad_al, _p(a), 1 << 30, nul) == -2
+    null_tok = list(args)
+    null_tok[7] = nul
+    assert lib.dllm_masked_logits(*null_tok, _p(a), 1 << 30, nul) == -1
+    # select_unmask
+    sel = [_p(a), _p(a), _p(a), 1, 16]
+    assert lib.dllm_select_unmask(*sel, 0, nul, nul, nul, _p(a), _p(a), nul, nul, nul) == -3
+    assert lib.dllm_select_unmask(*sel, 1025, nul, nul, nul, _p(a), _p(a), nul, nul, nul) == -3
+    assert lib.dllm_select_unmask(*sel, 4, _p(a), nul, nul, _p(a), _p(a), nul, nul, nul) == -1
+    assert lib.dllm_select_unmask(*sel, 4, nul, nul, nul, _p(a), _p(a), _p(a), nul, nul) == -1
+    assert lib.dllm_select_unmask(*sel, 4, nul, nul, nul, _p(a + 4), _p(a), nul, nul, nul) == -2
+    # decode_step checks the selection arguments before launching anything
+    step = [_p(a), _p(a), _p(a), 1, 256, 256, 4096]
+    assert lib.dllm_decode_step(*step, 0, nul, nul, *[_p(a)] * 6, _p(a), _p(a), nul, nul,
+                                _p(a), 1 << 30, nul) == -3
+    # merge hook
+    assert lib.dllm_debug_lse_merge(nul, _p(a), _p(a), 4, 2, _p(a), _p(a), _p(a), nul) == -1
+    assert lib.dllm_debug_lse_merge(_p(a), _p(a), _p(a), 0, 2, _p(a), _p(a), _p(a), nul) == -3

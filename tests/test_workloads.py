@@ -54,3 +54,19 @@ def test_bf16_bits_roundtrip():
     assert bits.dtype == np.uint16
     back = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
     assert torch.equal(back, t)
+
+
+def test_sweep_matches_individual_draws():
+    names = ["cfg3_r0.1", "cfg3_r0.9"]
+    small = {n: WL.get_config(n, L=512, d=8, V=16) for n in names}
+    WL.CONFIGS.update({f"_t_{n}": c for n, c in small.items()})
+    try:
+        sweep = WL.make_sweep_inputs([f"_t_{n}" for n in names], seed=3)
+        for n in names:
+            one = WL.make_inputs(small[n], seed=3)
+            got = sweep[small[n].name]
+            for key in ("H", "W", "M"):
+                assert torch.equal(one[key], got[key])
+    finally:
+        for n in names:
+            WL.CONFIGS.pop(f"_t_{n}")

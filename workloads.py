@@ -134,6 +134,26 @@ def make_inputs(cfg: Config, seed: int = 0) -> dict:
     return dict(cfg=cfg, H=H, W=W, M=M, k=cfg.k, win_lo=lo, win_hi=hi, seed=seed)
 
 
+def make_sweep_inputs(names: list[str], seed: int = 0) -> dict:
+    """Inputs of several workloads that differ only in their Bernoulli mask ratio (the cfg3
+    sweep): W and H are drawn once, and each mask is drawn from the generator state that
+    follows H, exactly as ``make_inputs`` would for that workload alone."""
+    cfgs = [CONFIGS[n] for n in names]
+    c0 = cfgs[0]
+    for c in cfgs[1:]:
+        assert (c.B, c.L, c.d, c.V) == (c0.B, c0.L, c0.d, c0.V) and c.mask == "bernoulli"
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    W = (torch.randn(c0.V, c0.d, generator=g, dtype=torch.float32) * c0.w_std).to(torch.bfloat16)
+    H = (torch.randn(c0.B * c0.L, c0.d, generator=g, dtype=torch.float32) * c0.h_std).to(torch.bfloat16)
+    state = g.get_state()
+    out = {}
+    for c in cfgs:
+        g.set_state(state)
+        out[c.name] = dict(cfg=c, H=H, W=W, M=make_mask(c, g), k=c.k, win_lo=None, win_hi=None,
+                           seed=seed)
+    return out
+
+
 def sample_rows(count: int, n: int = 512, seed: int = 0) -> np.ndarray:
     """A seeded sample of compacted row numbers in [0, count), ascending."""
     if count <= n:
