@@ -51,6 +51,7 @@ typedef int32_t dllm_status;
 #define DLLM_ERR_TIMEOUT    -6   /* a device-side wait exceeded its limit (kernel returned) */
 #define DLLM_ERR_DEVICE     -7   /* the current device is not an sm_100 GPU                 */
 #define DLLM_ERR_BOUNDS     -8   /* a device-side bound check failed (access skipped)       */
+#define DLLM_ERR_SCRATCH    -9   /* B*L exceeds the fixed scratch of dllm_mask_compact_noalloc */
 
 /* Limits. */
 #define DLLM_MAX_K          1024 /* largest k accepted by dllm_select_unmask                */
@@ -90,6 +91,36 @@ size_t dllm_workspace_bytes(int32_t B, int32_t L, int32_t d, int32_t V);
 dllm_status dllm_mask_compact(const uint8_t* M, int32_t B, int32_t L,
                               int32_t* row_idx, int32_t* seq_off, int32_t* count,
                               void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * dllm_mask_compact_noalloc - dllm_mask_compact without a workspace argument.
+ *
+ * The pages have no counterpart for this call; it exists for callers that cannot allocate
+ * device memory.  Some callers cannot hand the library a workspace: an inference engine
+ * whose memory planner owns every byte of HBM and forbids side allocations, or a plugin
+ * that must not call cudaMalloc (it can synchronise the whole device and stall other
+ * streams).  This variant allocates nothing.  Its scratch (the per-tile mask counts of the
+ * compaction) lives in a fixed array of DLLM_NOALLOC_MAX_TILES ints (64 KiB) in the
+ * library's static device memory, which every GPU that loads the library holds until the
+ * process exits.
+ *
+ * Arguments, outputs and results are exactly those of dllm_mask_compact.
+ * Limits and caveats:
+ *   - B*L must not exceed DLLM_NOALLOC_MAX_POSITIONS (134,217,728 positions); larger inputs
+ *     are rejected with DLLM_ERR_SCRATCH before anything is launched.
+ *   - The first call on a device looks up the scratch array's device address (once per
+ *     device, with that device current); make that first call before any stream capture.
+ *   - All calls on a device share the one scratch array.  Calls whose kernels overlap on the
+ *     GPU (different streams, no ordering between them) race on it and may return wrong
+ *     results; order such calls on one stream or with events.  The array keeps the last
+ *     call's contents; nothing needs clearing, because every slot a call reads is written
+ *     earlier in that same call.
+ */
+#define DLLM_NOALLOC_MAX_TILES      16384
+#define DLLM_NOALLOC_MAX_POSITIONS  (16384LL * 8192LL)
+dllm_status dllm_mask_compact_noalloc(const uint8_t* M, int32_t B, int32_t L,
+                                      int32_t* row_idx, int32_t* seq_off, int32_t* count,
+                                      void* stream);
 
 /*
  * dllm_masked_logits - mask-only LM head with a fused online softmax epilogue (Mosaic page,

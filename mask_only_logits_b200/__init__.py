@@ -20,7 +20,8 @@ import torch
 from . import _abi
 
 __all__ = [
-    "DllmError", "lib", "version", "workspace_bytes", "mask_compact", "masked_logits",
+    "DllmError", "lib", "version", "workspace_bytes", "mask_compact", "mask_compact_noalloc",
+    "masked_logits",
     "select_unmask", "decode_step", "get_status", "debug_lmhead_logits", "debug_lse_merge",
     "prof_begin", "prof_end", "DecodeStep", "MAX_K",
 ]
@@ -29,7 +30,7 @@ MAX_K = 1024
 
 STATUS = {0: "DLLM_OK", -1: "DLLM_ERR_NULL", -2: "DLLM_ERR_ALIGN", -3: "DLLM_ERR_SHAPE",
           -4: "DLLM_ERR_WORKSPACE", -5: "DLLM_ERR_CUDA", -6: "DLLM_ERR_TIMEOUT",
-          -7: "DLLM_ERR_DEVICE", -8: "DLLM_ERR_BOUNDS"}
+          -7: "DLLM_ERR_DEVICE", -8: "DLLM_ERR_BOUNDS", -9: "DLLM_ERR_SCRATCH"}
 
 
 class DllmError(RuntimeError):
@@ -82,6 +83,18 @@ def mask_compact(M, row_idx, seq_off, count, ws, stream=None) -> None:
                                    _ptr(count, torch.int32, "count"), _ptr(ws, None, "ws"),
                                    ws.numel() * ws.element_size(), _stream(stream)),
            "dllm_mask_compact")
+
+
+def mask_compact_noalloc(M, row_idx, seq_off, count, stream=None) -> None:
+    """mask_compact for callers that cannot allocate device memory: no workspace; the
+    library's fixed static scratch is used instead (B*L <= 134,217,728; calls that overlap
+    on the GPU race on that scratch)."""
+    B, L = M.shape
+    _check(lib().dllm_mask_compact_noalloc(_ptr(M, torch.uint8, "M"), B, L,
+                                           _ptr(row_idx, torch.int32, "row_idx"),
+                                           _ptr(seq_off, torch.int32, "seq_off"),
+                                           _ptr(count, torch.int32, "count"), _stream(stream)),
+           "dllm_mask_compact_noalloc")
 
 
 def masked_logits(H, M, W, tok, conf, lse, row_idx, seq_off, count, ws, stream=None) -> None:

@@ -18,6 +18,7 @@ PROTOTYPES = {
     "dllm_status_string": (ctypes.c_char_p, [_st]),
     "dllm_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32]),
     "dllm_mask_compact": (_st, [_p, _i32, _i32, _p, _p, _p, _p, _sz, _p]),
+    "dllm_mask_compact_noalloc": (_st, [_p, _i32, _i32, _p, _p, _p, _p]),
     "dllm_masked_logits": (_st, [_p, _p, _p, _i32, _i32, _i32, _i32, _p, _p, _p, _p, _p, _p,
                                  _p, _sz, _p]),
     "dllm_select_unmask": (_st, [_p, _p, _p, _i32, _i32, _i32, _p, _p, _p, _p, _p, _p, _p, _p]),

@@ -246,9 +246,65 @@ dllm_status run_logits(const LogitsArgs& a, bool debug) {
 }  // namespace
 }  // namespace dllm
 
+// ---------------------------------------------------------------------------------------
+// Allocation-free compaction (dllm_mask_compact_noalloc): the per-tile counts live in this
+// fixed static device array instead of the caller's workspace.  In host code the array's
+// name is only a host-side stand-in; its device address comes from cudaGetSymbolAddress,
+// looked up once per device.
+// ---------------------------------------------------------------------------------------
+static __device__ __align__(256) int g_noalloc_tile_counts[DLLM_NOALLOC_MAX_TILES];
+
+static_assert(static_cast<long long>(DLLM_NOALLOC_MAX_TILES) * dllm::kCompactTile ==
+                  DLLM_NOALLOC_MAX_POSITIONS,
+              "scratch limit and compaction tile size disagree");
+
+namespace {
+struct NoAllocScratch {
+  bool ready = false;
+  dllm_status err = DLLM_OK;
+  int* tiles = nullptr;           // device address of g_noalloc_tile_counts on this device
+};
+std::mutex g_noalloc_mu;
+NoAllocScratch g_noalloc[64];
+
+dllm_status noalloc_scratch(int** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DLLM_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return DLLM_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  NoAllocScratch& st = g_noalloc[dev];
+  if (!st.ready) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_tile_counts);
+    st.err = (e == cudaSuccess && p != nullptr) ? DLLM_OK : DLLM_ERR_CUDA;
+    st.tiles = static_cast<int*>(p);
+    st.ready = true;
+  }
+  if (st.err != DLLM_OK) return st.err;
+  *out = st.tiles;
+  return DLLM_OK;
+}
+}  // namespace
+
 using namespace dllm;
 
 extern "C" {
+
+dllm_status dllm_mask_compact_noalloc(const uint8_t* M, int32_t B, int32_t L, int32_t* row_idx,
+                                      int32_t* seq_off, int32_t* count, void* stream) {
+  if (!M || !row_idx || !seq_off || !count) return DLLM_ERR_NULL;
+  if (!shapes_ok(B, L)) return DLLM_ERR_SHAPE;
+  if (static_cast<long long>(B) * L > DLLM_NOALLOC_MAX_POSITIONS) return DLLM_ERR_SCRATCH;
+  if (!aligned16(M) || !aligned16(row_idx) || !aligned16(seq_off) || !aligned16(count))
+    return DLLM_ERR_ALIGN;
+  DeviceState* ds = nullptr;
+  dllm_status st = device_state(&ds);
+  if (st != DLLM_OK) return st;
+  int* tiles = nullptr;
+  if ((st = noalloc_scratch(&tiles)) != DLLM_OK) return st;
+  return launch_compact(M, B, L, row_idx, seq_off, count, tiles, ds->status,
+                        static_cast<cudaStream_t>(stream));
+}
 
 int32_t dllm_version(void) { return 10000; }
 
@@ -263,6 +319,7 @@ const char* dllm_status_string(dllm_status s) {
     case DLLM_ERR_TIMEOUT: return "a device-side wait timed out";
     case DLLM_ERR_DEVICE: return "device is not an sm_100 GPU";
     case DLLM_ERR_BOUNDS: return "a device-side bound check failed";
+    case DLLM_ERR_SCRATCH: return "B*L exceeds the fixed scratch of the allocation-free entry point";
     default: return "unknown status";
   }
 }
