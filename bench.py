@@ -104,7 +104,7 @@ class ClockSampler:
                 self._t.join(timeout=5)
 
     def summary(self) -> dict:
-        sm, mx, reasons = [], [], set()
+        sm, mx, pw, reasons = [], [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
@@ -113,6 +113,7 @@ class ClockSampler:
             try:
                 sm.append(float(parts[1]))
                 mx.append(float(parts[2]))
+                pw.append(float(parts[3]))
             except ValueError:
                 continue
             for name, flag in zip(names, parts[5:9]):
@@ -121,7 +122,7 @@ class ClockSampler:
         if not sm:
             return dict(sm_mhz=None, sm_max_mhz=None, reasons=[], samples=0)
         return dict(sm_mhz=statistics.median(sm), sm_max_mhz=max(mx), reasons=sorted(reasons),
-                    samples=len(sm))
+                    samples=len(sm), power_w=statistics.median(pw) if pw else None)
 
 
 # ---------------------------------------------------------------------------- oracle leg
@@ -213,6 +214,8 @@ def main() -> None:
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--gemm-variant", type=int, default=0, choices=[0, 1, 2],
+                    help="0 = library default, 1 = single-SM GEMM, 2 = paired-SM GEMM")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     cfg = WL.CONFIGS[args.config]
@@ -249,6 +252,7 @@ def main() -> None:
     win_hi = None if inp["win_hi"] is None else torch.from_numpy(inp["win_hi"]).to(dev)
     torch.cuda.reset_peak_memory_stats(dev)
     base_mem = torch.cuda.memory_allocated(dev)
+    dl.debug_set_gemm_variant(args.gemm_variant)
     step = dl.DecodeStep(cfg.B, cfg.L, cfg.d, cfg.V, cfg.k, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -327,7 +331,10 @@ def main() -> None:
             roofline_ms=roof * 1e3,
             roofline=dict(bound="tensor" if a["flops"] / (peaks["bf16_tflops"] * 1e12) >=
                           a["bytes"] / (peaks["hbm_gbs"] * 1e9) else "hbm",
-                          kernel="masked_lmhead (lmhead_kernel)",
+                          kernel=("masked_lmhead, paired-SM tcgen05 (lmhead_kernel<2>)"
+                                  if args.gemm_variant == 2 or
+                                  (args.gemm_variant == 0 and cfg.B * cfg.L <= 16384) else
+                                  "masked_lmhead, single-SM tcgen05 (lmhead_kernel<1>)"),
                           achieved=tflops_gemm, peak=peaks["bf16_tflops"], unit="TFLOP/s",
                           frac=tflops_gemm / peaks["bf16_tflops"],
                           frac_of_sustained=(tflops_gemm / peaks["bf16_tflops_sustained"]

@@ -22,7 +22,10 @@
  *     caller's workspace, sized by dllm_workspace_bytes().
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  All
  *     work is enqueued asynchronously on it; no call synchronises the host except
- *     dllm_get_status() and dllm_prof_end().
+ *     dllm_get_status() and dllm_prof_end().  Kernels are launched with programmatic
+ *     stream serialization: a kernel may begin its set-up while the previous kernel on the
+ *     stream finishes, but it reads or writes no global memory before every earlier kernel
+ *     on the stream has completed, so stream order is preserved.
  *   - Arguments are validated on the host before anything is launched; an invalid call
  *     returns a negative status and enqueues nothing.
  *   - Errors detected on the device (a wait that gave up, a failed bound check) are
@@ -219,6 +222,15 @@ dllm_status dllm_debug_lmhead_logits(const uint16_t* H, const uint8_t* M, const 
 dllm_status dllm_debug_lse_merge(const float* part_m, const float* part_s,
                                  const int32_t* part_a, int32_t n_rows, int32_t n_split,
                                  int32_t* tok, float* conf, float* lse, void* stream);
+
+/*
+ * Test hook: choose the tensor-core GEMM variant used by later calls in this process:
+ * 2 = CTA pairs (tcgen05 cta_group::2, 256x256 tiles over two SMs), 1 = single CTAs
+ * (cta_group::1, 128x256 tiles), 0 = the default (pairs when B*L <= 16384, single CTAs
+ * above).  Results agree to fp32 rounding; the variants differ in speed.  Returns
+ * DLLM_ERR_SHAPE for other values.
+ */
+dllm_status dllm_debug_set_gemm_variant(int32_t cta_group);
 
 /*
  * Kernel-time accounting for benchmarks.  dllm_prof_begin() starts recording a CUDA event

@@ -23,6 +23,7 @@ __all__ = [
     "DllmError", "lib", "version", "workspace_bytes", "mask_compact", "mask_compact_noalloc",
     "masked_logits",
     "select_unmask", "decode_step", "get_status", "debug_lmhead_logits", "debug_lse_merge",
+    "debug_set_gemm_variant",
     "prof_begin", "prof_end", "DecodeStep", "MAX_K",
 ]
 
@@ -158,6 +159,12 @@ def debug_lse_merge(part_m, part_s, part_a, tok, conf, lse, stream=None) -> None
         _ptr(part_a, torch.int32, "part_a"), n_rows, n_split, _ptr(tok, torch.int32, "tok"),
         _ptr(conf, torch.float32, "conf"), _ptr(lse, torch.float32, "lse"), _stream(stream)),
         "dllm_debug_lse_merge")
+
+
+def debug_set_gemm_variant(cta_group: int) -> None:
+    """Test hook: 2 = paired-SM GEMM, 1 = single-SM GEMM, 0 = default (pairs for
+    B*L <= 16384, single SMs above)."""
+    _check(lib().dllm_debug_set_gemm_variant(cta_group), "dllm_debug_set_gemm_variant")
 
 
 def prof_begin() -> None:

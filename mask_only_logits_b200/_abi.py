@@ -28,6 +28,7 @@ PROTOTYPES = {
     "dllm_debug_lmhead_logits": (_st, [_p, _p, _p, _i32, _i32, _i32, _i32, _p, _p, _p, _p, _p,
                                        _sz, _p]),
     "dllm_debug_lse_merge": (_st, [_p, _p, _p, _i32, _i32, _p, _p, _p, _p]),
+    "dllm_debug_set_gemm_variant": (_st, [_i32]),
     "dllm_prof_begin": (_st, []),
     "dllm_prof_end": (_st, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i32),
                             ctypes.POINTER(_i32)]),

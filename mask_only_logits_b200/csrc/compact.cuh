@@ -67,6 +67,8 @@ __device__ __forceinline__ int block_sum(int v, int* red) {
 __global__ void __launch_bounds__(kCompactThreads)
 compact_count_kernel(const uint8_t* __restrict__ M, long long n, int* __restrict__ tile_count) {
   __shared__ int red[33];
+  pdl_wait();
+  pdl_launch_dependents();
   const long long p0 = (static_cast<long long>(blockIdx.x) * kCompactThreads + threadIdx.x) * kCompactVec;
   const int c = __popc(load_mask16(M, p0, n));
   const int total = block_sum(c, red);
@@ -79,6 +81,8 @@ compact_scatter_kernel(const uint8_t* __restrict__ M, int B, int L, const int* _
                        int* __restrict__ status) {
   __shared__ int red[33];
   __shared__ int warp_excl[kCompactThreads / 32];
+  pdl_wait();
+  pdl_launch_dependents();
   const long long n = static_cast<long long>(B) * L;
   const int t = blockIdx.x;
   // offset of this tile = sum of the counts of tiles 0..t-1
@@ -137,13 +141,18 @@ compact_scatter_kernel(const uint8_t* __restrict__ M, int B, int L, const int* _
 }
 
 // Copy the masked rows H[row_idx[r]] (d bf16 each) into the dense matrix Hm[r] for
-// r < count.  One warp per row, 16-byte vectors.
+// r < count (one warp per row, 16-byte vectors), and zero n_zero ints at `zero`.
 constexpr int kGatherThreads = 256;
 
 __global__ void __launch_bounds__(kGatherThreads)
 gather_rows_kernel(const uint16_t* __restrict__ H, const int* __restrict__ row_idx,
                    const int* __restrict__ count, long long n_pos, int d, uint16_t* __restrict__ Hm,
-                   int* __restrict__ status) {
+                   int* __restrict__ zero, int n_zero, int* __restrict__ status) {
+  pdl_wait();
+  pdl_launch_dependents();
+  // also clear the GEMM's per-m-tile unit counters for this step
+  for (int i = blockIdx.x * kGatherThreads + threadIdx.x; i < n_zero; i += gridDim.x * kGatherThreads)
+    zero[i] = 0;
   int n = *count;
   if (n < 0 || n > n_pos) {                          // cannot happen: bad compaction
     if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(status, kStatusBounds);

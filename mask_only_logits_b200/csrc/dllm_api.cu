@@ -32,8 +32,17 @@ struct DeviceState {
   bool ready = false;
   dllm_status err = DLLM_OK;
   int sms = 0;
+  int pairs = 0;                // co-resident CTA pairs of the cta_group::2 GEMM
   int* status = nullptr;        // device address of g_status on this device
 };
+
+// GEMM variant: 2 = CTA pairs (cta_group::2, 256x256 tiles), 1 = single CTAs
+// (cta_group::1, 128x256 tiles).  0 = default: pairs when B*L <= kPairMaxPositions (few
+// m-tiles: the larger tile does more work per clock), single CTAs above (measured under the
+// 1 kW power cap, the single-CTA kernel does more work per joule and sustains a higher clock
+// on long GEMMs).
+std::atomic<int> g_gemm_variant{0};
+constexpr long long kPairMaxPositions = 16384;
 
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
@@ -60,6 +69,25 @@ inline void count_launch(int n = 1) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Launch with programmatic stream serialization: the kernel may start while the previous
+// kernel on the stream finishes; every kernel of this library waits for its predecessors
+// (griddepcontrol.wait) before it touches global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Per-device setup, once: check the architecture, find g_status, raise the GEMM's shared
@@ -83,11 +111,34 @@ dllm_status device_state(DeviceState** out) {
       if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) st.err = DLLM_ERR_CUDA;
       st.status = static_cast<int*>(p);
       if (st.err == DLLM_OK &&
-          (cudaFuncSetAttribute(lm::lmhead_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                lm::SMEM_BYTES) != cudaSuccess ||
-           cudaFuncSetAttribute(lm::lmhead_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                lm::SMEM_BYTES) != cudaSuccess))
+          (cudaFuncSetAttribute(lm::lmhead_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                lm::Cfg<1>::SMEM_BYTES) != cudaSuccess ||
+           cudaFuncSetAttribute(lm::lmhead_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                lm::Cfg<1>::SMEM_BYTES) != cudaSuccess ||
+           cudaFuncSetAttribute(lm::lmhead_kernel<2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                lm::Cfg<2>::SMEM_BYTES) != cudaSuccess ||
+           cudaFuncSetAttribute(lm::lmhead_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                lm::Cfg<2>::SMEM_BYTES) != cudaSuccess))
         st.err = DLLM_ERR_CUDA;
+      if (st.err == DLLM_OK) {
+        // how many CTA pairs of the paired GEMM can be resident at once (a persistent grid
+        // larger than that would serialise)
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(2 * (st.sms / 2), 1, 1);
+        cfg.blockDim = dim3(lm::kThreads, 1, 1);
+        cfg.dynamicSmemBytes = lm::Cfg<2>::SMEM_BYTES;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, lm::lmhead_kernel<2, false>, &cfg) != cudaSuccess)
+          clusters = 0;
+        st.pairs = clusters < lm::kMaxCtas / 2 ? clusters : lm::kMaxCtas / 2;
+      }
       if (st.err == DLLM_OK && g_encode == nullptr) {
         void* fn = nullptr;
         cudaDriverEntryPointQueryResult q;
@@ -105,24 +156,33 @@ dllm_status device_state(DeviceState** out) {
   return DLLM_OK;
 }
 
-// Workspace layout: [tile counts | gathered rows Hm | part_m | part_s | part_a].
+// Workspace layout: [tile counts | unit counters | gathered rows Hm | part_m | part_s | part_a].
 struct WsLayout {
-  size_t tiles_off, hm_off, pm_off, ps_off, pa_off, total;
+  size_t tiles_off, ctr_off, hm_off, pm_off, ps_off, pa_off, total;
   long long part_cap;
+  int n_ctr;
 };
 
 WsLayout ws_layout(int B, int L, int d, int V) {
   WsLayout w{};
   const long long n = static_cast<long long>(B) * L;
   const long long ntiles = (n + kCompactTile - 1) / kCompactTile;
-  // partial entries: worst case over the masked count (all positions masked) with the
-  // largest CTA count; fewer masked rows never need more.
-  const lm::Plan worst = lm::Plan::make(static_cast<int>(n), V, lm::kMaxCtas, lm::kGroupM);
-  long long cap = worst.ngroups * static_cast<long long>(lm::kMaxCtas) * lm::BM;
+  // partial entries: worst case over the masked count (all positions masked), the largest
+  // number of work holders and either GEMM variant; fewer masked rows never need more.
+  const lm::Plan w1 = lm::Plan::make(static_cast<int>(n), V, lm::kMaxCtas, lm::Cfg<1>::kGroupM,
+                                     lm::Cfg<1>::BM);
+  const lm::Plan w2 = lm::Plan::make(static_cast<int>(n), V, lm::kMaxCtas / 2, lm::Cfg<2>::kGroupM,
+                                     lm::Cfg<2>::BM);
+  const long long cap1 = w1.ngroups * static_cast<long long>(lm::kMaxCtas) * lm::Cfg<1>::BM;
+  const long long cap2 = w2.ngroups * static_cast<long long>(lm::kMaxCtas / 2) * lm::Cfg<2>::BM;
+  long long cap = cap1 > cap2 ? cap1 : cap2;
   if (cap < 1) cap = 1;
   w.part_cap = cap;
+  // one counter per (m-tile, CTA of the pair): ceil(n / 128) + 2 covers both variants
+  w.n_ctr = static_cast<int>((n + 127) / 128 + 2);
   size_t off = 0;
   w.tiles_off = off; off = round_up(off + sizeof(int) * ntiles, 256);
+  w.ctr_off = off;   off = round_up(off + sizeof(int) * static_cast<size_t>(w.n_ctr), 256);
   w.hm_off = off;    off = round_up(off + static_cast<size_t>(n) * d * 2, 256);
   w.pm_off = off;    off = round_up(off + sizeof(float) * cap, 256);
   w.ps_off = off;    off = round_up(off + sizeof(float) * cap, 256);
@@ -139,11 +199,17 @@ dllm_status launch_compact(const uint8_t* M, int B, int L, int* row_idx, int* se
                            int* tiles, int* status, cudaStream_t s) {
   const long long n = static_cast<long long>(B) * L;
   const unsigned ntiles = static_cast<unsigned>((n + kCompactTile - 1) / kCompactTile);
-  compact_count_kernel<<<ntiles, kCompactThreads, 0, s>>>(M, n, tiles);
-  compact_scatter_kernel<<<ntiles, kCompactThreads, 0, s>>>(M, B, L, tiles, row_idx, seq_off, count,
-                                                            status);
-  count_launch(2);
-  return cudaPeekAtLastError() == cudaSuccess ? DLLM_OK : DLLM_ERR_CUDA;
+  // a single tile needs no per-tile counts: its offset is 0
+  if (ntiles > 1) {
+    if (launch_pdl(compact_count_kernel, dim3(ntiles), dim3(kCompactThreads), 0, s, M, n, tiles) != cudaSuccess)
+      return DLLM_ERR_CUDA;
+    count_launch();
+  }
+  if (launch_pdl(compact_scatter_kernel, dim3(ntiles), dim3(kCompactThreads), 0, s, M, B, L,
+                 (const int*)tiles, row_idx, seq_off, count, status) != cudaSuccess)
+    return DLLM_ERR_CUDA;
+  count_launch();
+  return DLLM_OK;
 }
 
 dllm_status make_tmap(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
@@ -191,22 +257,31 @@ dllm_status run_logits(const LogitsArgs& a, bool debug) {
   float* pm = reinterpret_cast<float*>(ws + w.pm_off);
   float* ps = reinterpret_cast<float*>(ws + w.ps_off);
   int* pa = reinterpret_cast<int*>(ws + w.pa_off);
+  int* ctr = reinterpret_cast<int*>(ws + w.ctr_off);
   const long long n = static_cast<long long>(a.B) * a.L;
 
-  const int ctas = ds->sms < lm::kMaxCtas ? ds->sms : lm::kMaxCtas;
-  const lm::Plan worst = lm::Plan::make(static_cast<int>(n), a.V, ctas, lm::kGroupM);
+  // GEMM variant and its work holders (CTAs, or CTA pairs)
+  int cg = g_gemm_variant.load();
+  if (cg == 0) cg = n <= kPairMaxPositions ? 2 : 1;
+  if (cg == 2 && ds->pairs < 1) cg = 1;
+  const int holders = cg == 2 ? ds->pairs : (ds->sms < lm::kMaxCtas ? ds->sms : lm::kMaxCtas);
+  const int bm = cg == 2 ? lm::Cfg<2>::BM : lm::Cfg<1>::BM;
+  const int gmax = cg == 2 ? lm::Cfg<2>::kGroupM : lm::Cfg<1>::kGroupM;
+  const lm::Plan worst = lm::Plan::make(static_cast<int>(n), a.V, holders, gmax, bm);
   if (worst.part_entries() > w.part_cap) return DLLM_ERR_WORKSPACE;   // cannot happen on B200
 
   if ((st = launch_compact(a.M, a.B, a.L, a.row_idx, a.seq_off, a.count, tiles, ds->status, a.s)) != DLLM_OK)
     return st;
 
-  gather_rows_kernel<<<ds->sms * 4, kGatherThreads, 0, a.s>>>(a.H, a.row_idx, a.count, n, a.d, Hm,
-                                                               ds->status);
+  if (launch_pdl(gather_rows_kernel, dim3(ds->sms * 4), dim3(kGatherThreads), 0, a.s, a.H,
+                 (const int*)a.row_idx, (const int*)a.count, n, a.d, Hm, ctr, w.n_ctr,
+                 ds->status) != cudaSuccess)
+    return DLLM_ERR_CUDA;
   count_launch();
 
   CUtensorMap tmA, tmB;
-  if (make_tmap(&tmA, Hm, static_cast<uint64_t>(n), a.d, lm::BM) != DLLM_OK) return DLLM_ERR_CUDA;
-  if (make_tmap(&tmB, a.W, static_cast<uint64_t>(a.V), a.d, lm::BN) != DLLM_OK) return DLLM_ERR_CUDA;
+  if (make_tmap(&tmA, Hm, static_cast<uint64_t>(n), a.d, 128) != DLLM_OK) return DLLM_ERR_CUDA;
+  if (make_tmap(&tmB, a.W, static_cast<uint64_t>(a.V), a.d, lm::BN / cg) != DLLM_OK) return DLLM_ERR_CUDA;
 
   cudaEvent_t e0 = nullptr, e1 = nullptr;
   if (g_prof.on) {
@@ -222,23 +297,50 @@ dllm_status run_logits(const LogitsArgs& a, bool debug) {
     g_prof.used += 2;
     cudaEventRecord(e0, a.s);
   }
-  if (debug)
-    lm::lmhead_kernel<true><<<ctas, lm::kThreads, lm::SMEM_BYTES, a.s>>>(
-        tmA, tmB, a.count, static_cast<int>(n), a.V, a.d, lm::kGroupM, pm, ps, pa, w.part_cap, a.dbg, ds->status);
-  else
-    lm::lmhead_kernel<false><<<ctas, lm::kThreads, lm::SMEM_BYTES, a.s>>>(
-        tmA, tmB, a.count, static_cast<int>(n), a.V, a.d, lm::kGroupM, pm, ps, pa, w.part_cap, nullptr, ds->status);
+  {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[2];
+    cfg.blockDim = dim3(lm::kThreads, 1, 1);
+    cfg.stream = a.s;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cg == 2) {
+      attr[1].id = cudaLaunchAttributeClusterDimension;
+      attr[1].val.clusterDim.x = 2;
+      attr[1].val.clusterDim.y = 1;
+      attr[1].val.clusterDim.z = 1;
+      cfg.numAttrs = 2;
+      cfg.gridDim = dim3(2 * holders, 1, 1);
+      cfg.dynamicSmemBytes = lm::Cfg<2>::SMEM_BYTES;
+    } else {
+      cfg.gridDim = dim3(holders, 1, 1);
+      cfg.dynamicSmemBytes = lm::Cfg<1>::SMEM_BYTES;
+    }
+    const int n_cap = static_cast<int>(n);
+    float* dbg = debug ? a.dbg : nullptr;
+    cudaError_t e;
+    if (cg == 2)
+      e = debug ? cudaLaunchKernelEx(&cfg, lm::lmhead_kernel<2, true>, tmA, tmB, (const int*)a.count, n_cap,
+                                     a.V, a.d, gmax, pm, ps, pa, w.part_cap, ctr, a.tok, a.conf, a.lse,
+                                     dbg, ds->status)
+                : cudaLaunchKernelEx(&cfg, lm::lmhead_kernel<2, false>, tmA, tmB, (const int*)a.count, n_cap,
+                                     a.V, a.d, gmax, pm, ps, pa, w.part_cap, ctr, a.tok, a.conf, a.lse,
+                                     dbg, ds->status);
+    else
+      e = debug ? cudaLaunchKernelEx(&cfg, lm::lmhead_kernel<1, true>, tmA, tmB, (const int*)a.count, n_cap,
+                                     a.V, a.d, gmax, pm, ps, pa, w.part_cap, ctr, a.tok, a.conf, a.lse,
+                                     dbg, ds->status)
+                : cudaLaunchKernelEx(&cfg, lm::lmhead_kernel<1, false>, tmA, tmB, (const int*)a.count, n_cap,
+                                     a.V, a.d, gmax, pm, ps, pa, w.part_cap, ctr, a.tok, a.conf, a.lse,
+                                     dbg, ds->status);
+    if (e != cudaSuccess) return DLLM_ERR_CUDA;
+  }
   count_launch();
   if (g_prof.on) {
     cudaEventRecord(e1, a.s);
     g_prof.gemm_launches++;
-  }
-  if (!debug) {
-    int mblocks = static_cast<int>((n + kMergeThreads - 1) / kMergeThreads);
-    if (mblocks > ds->sms * 8) mblocks = ds->sms * 8;
-    lse_merge_kernel<<<mblocks, kMergeThreads, 0, a.s>>>(a.count, static_cast<int>(n), a.V, ctas, lm::kGroupM, pm, ps, pa,
-                                                        a.tok, a.conf, a.lse);
-    count_launch();
   }
   return cudaPeekAtLastError() == cudaSuccess ? DLLM_OK : DLLM_ERR_CUDA;
 }
@@ -378,10 +480,12 @@ dllm_status dllm_select_unmask(const float* conf, const int32_t* row_idx, const 
   DeviceState* ds = nullptr;
   dllm_status st = device_state(&ds);
   if (st != DLLM_OK) return st;
-  select_unmask_kernel<<<B, kSelThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      conf, row_idx, seq_off, B * L, L, k, win_lo, win_hi, tok, idx, n_sel, tok_sel, conf_sel);
+  if (launch_pdl(select_unmask_kernel, dim3(B), dim3(kSelThreads), 0, static_cast<cudaStream_t>(stream),
+                 conf, row_idx, seq_off, B * L, L, k, win_lo, win_hi, tok, idx, n_sel, tok_sel,
+                 conf_sel) != cudaSuccess)
+    return DLLM_ERR_CUDA;
   count_launch();
-  return cudaPeekAtLastError() == cudaSuccess ? DLLM_OK : DLLM_ERR_CUDA;
+  return DLLM_OK;
 }
 
 dllm_status dllm_decode_step(const uint16_t* H, const uint8_t* M, const uint16_t* W, int32_t B,
@@ -421,6 +525,12 @@ dllm_status dllm_debug_lse_merge(const float* part_m, const float* part_s, const
       part_m, part_s, part_a, n_rows, n_split, tok, conf, lse);
   count_launch();
   return cudaPeekAtLastError() == cudaSuccess ? DLLM_OK : DLLM_ERR_CUDA;
+}
+
+dllm_status dllm_debug_set_gemm_variant(int32_t cta_group) {
+  if (cta_group != 0 && cta_group != 1 && cta_group != 2) return DLLM_ERR_SHAPE;
+  g_gemm_variant.store(cta_group);
+  return DLLM_OK;
 }
 
 dllm_status dllm_get_status(void* stream) {

@@ -1,65 +1,100 @@
 // lmhead.cuh - masked_lmhead: the mask-only LM head on the 5th-generation tensor cores with
 // the softmax statistics fused into the epilogue (Mosaic page, TL;DR and Abstract: the
-// mask-only logits kernel; the logits tensor of the masked rows is never written).
+// mask-only logits kernel; the logits of the masked rows are never written either).
 //
 // C[i, v] = sum_k Hm[i, k] * W[v, k] for the compacted masked rows Hm (bf16, K-major) and
 // the vocabulary projection W (bf16, K-major), fp32 accumulation in tensor memory.
 //
-// Persistent, warp-specialised kernel, one CTA per SM, 192 threads:
-//   warp 0      TMA producer: 128x64 tile of Hm and 256x64 tile of W per stage
+// Persistent, warp-specialised kernel, one CTA per SM, 192 threads, templated on the CTA
+// group size CG:
+//   CG = 1  each CTA owns a 128 x 256 tile (tcgen05.mma.cta_group::1, M=128, N=256)
+//   CG = 2  a cluster of two CTAs on paired SMs owns a 256 x 256 tile
+//           (tcgen05.mma.cta_group::2, M=256, N=256): each CTA stages 128 rows of Hm and
+//           128 rows of W per stage, the leader CTA issues the MMAs for both, and each CTA's
+//           TMEM holds its own 128 rows of the accumulator.  Per SM this halves the W bytes
+//           staged per flop.
+// Roles (per CTA):
+//   warp 0      TMA producer: a 128x64 tile of Hm and a (256/CG)x64 tile of W per stage
 //               (128-byte swizzle) into a kStages-deep shared-memory ring
-//   warp 1      allocates 512 TMEM columns; lane 0 issues tcgen05.mma (M=128, N=256,
-//               K=16, four per stage) into one of two 128x256 fp32 accumulators and
-//               commits stage releases / accumulator-full events to mbarriers
+//   warp 1      allocates 512 TMEM columns; lane 0 of the leader issues the MMAs (four per
+//               stage) into one of two 256-column fp32 accumulators and commits stage
+//               releases / accumulator-full events to mbarriers
 //   warps 2..5  epilogue: warp w reads TMEM lanes 32*(w%4)..+31 (one row per thread) with
 //               tcgen05.ld, keeps a running (max, sum exp(z - max), first argmax) per row
 //               over the vocabulary tiles of its unit, then writes one partial per row
 //
-// Work decomposition.  A "unit" is (m-tile of 128 rows, contiguous range of vocabulary
-// tiles).  m-tiles are taken in groups of up to `gmax`; inside a group of G m-tiles the CTAs
-// are split into P = floor(ctas / G) vocabulary streams, CTA c handling m-tile c % G and
-// stream c / G.  CTAs of one group therefore walk the same W tiles at the same time
-// (each W tile is fetched from HBM about once per group and served to the other G-1 CTAs
-// from L2) while the group's G Hm tiles stay resident in L2.  Per row, the partials of the
-// P streams are merged by lse_merge.
+// Work decomposition.  A "unit" is (m-tile, contiguous range of vocabulary tiles).  m-tiles
+// are taken in groups of up to `gmax`; inside a group of G m-tiles the work holders (CTAs,
+// or CTA pairs for CG = 2) are split into P = floor(holders / G) vocabulary streams, holder
+// c handling m-tile c % G and stream c / G.  Holders of one stream therefore walk the same
+// W tiles at the same time (each W tile is fetched from HBM about once per group and served
+// from L2 to the others) while the group's Hm tiles stay resident in L2.  Per row, the
+// partials of the P streams are merged (lse_merge) by the epilogue of whichever CTA finishes
+// the m-tile's last unit; with P = 1 the unit's statistics are the result.
+//
+// Every wait is bounded (ptx.cuh).  On a timeout the CTA raises its abort flag, every role
+// unwinds, the MMA issuer waits (bounded) for its issued MMAs, the CTA lingers 2 ms so that
+// TMA loads already in flight land, and TMEM is released before the kernel returns.
 #pragma once
 #include "ptx.cuh"
+
+// Compile-time tuning knobs (defaults are the measured best).
+#ifndef DLLM_GROUP_M1
+#define DLLM_GROUP_M1 37          // m-tiles per L2 group, single-CTA variant
+#endif
+#ifndef DLLM_GROUP_M2
+#define DLLM_GROUP_M2 18          // m-tiles per L2 group, CTA-pair variant
+#endif
+#ifndef DLLM_STAGES2
+#define DLLM_STAGES2 6            // shared-memory ring depth, CTA-pair variant
+#endif
+#ifndef DLLM_EPI_BACKOFF_NS
+#define DLLM_EPI_BACKOFF_NS 0     // epilogue: sleep between polls of the accumulator barrier
+#endif
 
 namespace dllm {
 namespace lm {
 
-constexpr int BM = 128;                 // rows per tile (UMMA M)
 constexpr int BN = 256;                 // vocabulary entries per tile (UMMA N)
 constexpr int BK = 64;                  // K per stage: one 128-byte swizzle atom of bf16
 constexpr int UK = 16;                  // K per tcgen05.mma (kind::f16)
-constexpr int kStages = 4;
-constexpr int A_BYTES = BM * BK * 2;    // 16 KiB
-constexpr int B_BYTES = BN * BK * 2;    // 32 KiB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int kThreads = 192;
 constexpr int kEpiWarps = 4;
 constexpr int kTmemCols = 2 * BN;       // two accumulators
 constexpr int kMaxCtas = 160;           // partial-buffer sizing bound (B200: 148 SMs)
-constexpr int kGroupM = 37;             // m-tiles per L2 group (148 = 4 x 37)
-constexpr int SMEM_BYTES = 1024 + kStages * STAGE_BYTES + 256;
-
-// Instruction descriptor, kind::f16: fp32 accumulator (bits 4-5 = 1), A and B bf16
-// (bits 7-9 = 1, bits 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bits 17-22,
-// M >> 4 at bits 24-28.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
-                            (static_cast<uint32_t>(BN >> 3) << 17) |
-                            (static_cast<uint32_t>(BM >> 4) << 24);
-
 constexpr float kLog2e = 1.4426950408889634f;
 
-// The unit schedule, computed identically by the GEMM's three roles and by lse_merge.
-struct Plan {
-  int count, numM, numN, ctas, gmax, ngroups, P_full;
+template <int CG>
+struct Cfg {
+  static_assert(CG == 1 || CG == 2, "CTA group of 1 or 2");
+  static constexpr int BM_CTA = 128;                 // rows per CTA (TMEM lanes)
+  static constexpr int BM = BM_CTA * CG;             // rows per m-tile
+  static constexpr int B_ROWS = BN / CG;             // W rows staged per CTA per stage
+  static constexpr int A_BYTES = BM_CTA * BK * 2;
+  static constexpr int B_BYTES = B_ROWS * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int kStages = CG == 1 ? 4 : DLLM_STAGES2;
+  static constexpr int SMEM_BYTES = 1024 + kStages * STAGE_BYTES + 256;
+  static constexpr int kGroupM = CG == 1 ? DLLM_GROUP_M1 : DLLM_GROUP_M2;  // m-tiles per L2 group
+  // Instruction descriptor, kind::f16: fp32 accumulator (bits 4-5 = 1), A and B bf16
+  // (bits 7-9 = 1, bits 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bits 17-22,
+  // M >> 4 at bits 24-28.
+  static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
+                                     (static_cast<uint32_t>(BN >> 3) << 17) |
+                                     (static_cast<uint32_t>(BM >> 4) << 24);
+};
 
-  __host__ __device__ static Plan make(int count, int V, int ctas, int gmax) {
+// The unit schedule, computed identically by the GEMM's roles and by lse_merge.
+struct Plan {
+  int count, bm, numM, numN, ctas, gmax, ngroups, P_full;
+
+  // ctas = number of work holders (CTAs for CG = 1, CTA pairs for CG = 2);
+  // bm = rows per m-tile.
+  __host__ __device__ static Plan make(int count, int V, int ctas, int gmax, int bm) {
     Plan p;
     p.count = count;
-    p.numM = (count + BM - 1) / BM;
+    p.bm = bm;
+    p.numM = (count + bm - 1) / bm;
     p.numN = (V + BN - 1) / BN;
     p.ctas = ctas;
     p.gmax = gmax < ctas ? gmax : ctas;
@@ -77,33 +112,34 @@ struct Plan {
   }
   // Partial-buffer index of (group g of size G, stream p, row r within the group).
   __host__ __device__ long long part_index(int g, int G, int p, int r) const {
-    return static_cast<long long>(g) * gmax * BM * P_full + static_cast<long long>(p) * G * BM + r;
+    return static_cast<long long>(g) * gmax * bm * P_full + static_cast<long long>(p) * G * bm + r;
   }
-  // Number of partial entries written for this count (upper bound for sizing).
+  // Number of partial entries written for this count.
   __host__ __device__ long long part_entries() const {
     if (ngroups == 0) return 0;
     const int Gl = group_size(ngroups - 1);
     return part_index(ngroups - 1, Gl, 0, 0) +
-           static_cast<long long>(Gl) * BM * streams(Gl, ctas, numN);
+           static_cast<long long>(Gl) * bm * streams(Gl, ctas, numN);
   }
 };
 
-// One unit of a CTA inside group g, or false if the CTA is idle in this group.
+// One unit of a work holder inside group g, or false if it is idle in this group.
 struct Unit {
   int m_tile, m_local, G, p, P, n0, n1;
 };
-__device__ __forceinline__ bool unit_of(const Plan& pl, int g, int cta, Unit& u) {
+__device__ __forceinline__ bool unit_of(const Plan& pl, int g, int holder, Unit& u) {
   u.G = pl.group_size(g);
   u.P = Plan::streams(u.G, pl.ctas, pl.numN);
-  if (cta >= u.G * u.P) return false;
-  u.m_local = cta % u.G;
+  if (holder >= u.G * u.P) return false;
+  u.m_local = holder % u.G;
   u.m_tile = g * pl.gmax + u.m_local;
-  u.p = cta / u.G;
+  u.p = holder / u.G;
   u.n0 = static_cast<int>(static_cast<long long>(u.p) * pl.numN / u.P);
   u.n1 = static_cast<int>(static_cast<long long>(u.p + 1) * pl.numN / u.P);
   return true;
 }
 
+template <int CG>
 struct Smem {
   uint8_t* a;          // kStages x A_BYTES
   uint8_t* b;          // kStages x B_BYTES
@@ -112,25 +148,28 @@ struct Smem {
   uint64_t* tfull;     // 2
   uint64_t* tempty;    // 2
   uint64_t* drain;     // 1: MMA completion on the abort path
+  uint64_t* epi_bar;   // 1: barrier of the four epilogue warps (bounded, unlike bar.sync)
   uint32_t* tmem_slot;
   int* abort_flag;
-};
+  volatile int* last_flag;   // epilogue: this CTA finished the last unit of an m-tile
 
-__device__ __forceinline__ Smem carve(uint8_t* raw) {
-  Smem s;
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
-  s.a = base;
-  s.b = base + kStages * A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(s.b + kStages * B_BYTES);
-  s.full = bars;
-  s.empty = bars + kStages;
-  s.tfull = bars + 2 * kStages;
-  s.tempty = bars + 2 * kStages + 2;
-  s.drain = bars + 2 * kStages + 4;
-  s.tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
-  s.abort_flag = reinterpret_cast<int*>(s.tmem_slot + 1);
-  return s;
-}
+  __device__ __forceinline__ explicit Smem(uint8_t* raw) {
+    using C = Cfg<CG>;
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+    a = base;
+    b = base + C::kStages * C::A_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(b + C::kStages * C::B_BYTES);
+    full = bars;
+    empty = bars + C::kStages;
+    tfull = bars + 2 * C::kStages;
+    tempty = bars + 2 * C::kStages + 2;
+    drain = bars + 2 * C::kStages + 4;
+    epi_bar = bars + 2 * C::kStages + 5;
+    tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::kStages + 6);
+    abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+    last_flag = abort_flag + 1;
+  }
+};
 
 // Online (max, sum of exp(z - max), first argmax) over 32 consecutive logits.
 __device__ __forceinline__ void fold_chunk(float (&v)[32], int col0, int V, float& run_m,
@@ -165,26 +204,92 @@ __device__ __forceinline__ void fold_chunk(float (&v)[32], int col0, int V, floa
   run_s += (s0 + s1) + (s2 + s3);
 }
 
-template <bool kDebugStore>
+// lse_merge of one row: combine n_split partials (m_j, s_j, a_j) found at base + j * stride
+// (j = 0..n_split-1, ascending vocabulary ranges):
+//   m* = max_j m_j, s* = sum_j s_j exp(m_j - m*), tok = a_j of the first j with m_j = m*,
+//   lse = m* + ln s*, conf = exp(m* - lse) = 1 / s*.
+// Partials are read through L2 (they may have been written by other CTAs of the running
+// kernel) in batches of 8 whose loads are all issued before any is used.
+__device__ __forceinline__ void merge_row(const float* __restrict__ pm, const float* __restrict__ ps,
+                                          const int* __restrict__ pa, long long base,
+                                          long long stride, int n_split, int& tok, float& conf,
+                                          float& lse) {
+  constexpr int kBatch = 8;
+  float m = -INFINITY, s = 0.f;
+  int a = 0;
+  for (int j0 = 0; j0 < n_split; j0 += kBatch) {
+    float mb[kBatch], sb[kBatch];
+    int ab[kBatch];
+#pragma unroll
+    for (int t = 0; t < kBatch; ++t) {
+      if (j0 + t < n_split) {
+        const long long e = base + (j0 + t) * stride;
+        mb[t] = __ldcg(pm + e);
+        sb[t] = __ldcg(ps + e);
+        ab[t] = __ldcg(pa + e);
+      } else {
+        mb[t] = -INFINITY;
+        sb[t] = 0.f;
+        ab[t] = 0;
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < kBatch; ++t) {
+      if (j0 + t >= n_split) break;
+      if (mb[t] > m) {               // strict: the earlier split keeps a tie
+        s = s * ex2_approx((m - mb[t]) * kLog2e) + sb[t];
+        m = mb[t];
+        a = ab[t];
+      } else {
+        s += sb[t] * ex2_approx((mb[t] - m) * kLog2e);
+      }
+    }
+  }
+  tok = a;
+  lse = m + logf(s);
+  conf = 1.0f / s;
+}
+
+template <int CG>
+__device__ __forceinline__ void mma_issue(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t acc) {
+  if constexpr (CG == 1) umma_bf16(d_tmem, a_desc, b_desc, idesc, acc);
+  else umma_bf16_pair(d_tmem, a_desc, b_desc, idesc, acc);
+}
+
+// Arrive on barrier `bar` of every CTA of the group once the issued MMAs complete.
+template <int CG>
+__device__ __forceinline__ void mma_commit_all(uint32_t bar) {
+  if constexpr (CG == 1) umma_commit(bar);
+  else umma_commit_pair_both(bar);
+}
+
+template <int CG, bool kDebugStore>
 __global__ void __launch_bounds__(kThreads, 1)
 lmhead_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const int* __restrict__ count_ptr, int n_cap, int V, int d, int gmax,
               float* __restrict__ part_m, float* __restrict__ part_s, int* __restrict__ part_a,
-              long long part_cap, float* __restrict__ dbg_logits, int* __restrict__ status) {
+              long long part_cap, int* __restrict__ unit_ctr, int* __restrict__ out_tok,
+              float* __restrict__ out_conf, float* __restrict__ out_lse,
+              float* __restrict__ dbg_logits, int* __restrict__ status) {
+  using C = Cfg<CG>;
   extern __shared__ uint8_t smem_raw[];
-  Smem sm = carve(smem_raw);
+  Smem<CG> sm(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = CG == 1 ? 0u : cluster_ctarank();   // rank inside the CTA pair
+  const bool leader = rank == 0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < C::kStages; ++s) {
       mbar_init(smem_u32(&sm.full[s]), 1);
       mbar_init(smem_u32(&sm.empty[s]), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&sm.tfull[b]), 1);
-      mbar_init(smem_u32(&sm.tempty[b]), kEpiWarps * 32);
+      mbar_init(smem_u32(&sm.tempty[b]), CG * kEpiWarps * 32);
     }
     mbar_init(smem_u32(sm.drain), 1);
+    mbar_init(smem_u32(sm.epi_bar), kEpiWarps * 32);
     *sm.abort_flag = 0;
     fence_mbar_init();
   }
@@ -193,102 +298,130 @@ lmhead_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(sm.tmem_slot), kTmemCols);
-    tmem_relinquish();
+    if constexpr (CG == 1) {
+      tmem_alloc(smem_u32(sm.tmem_slot), kTmemCols);
+      tmem_relinquish();
+    } else {
+      tmem_alloc_pair(smem_u32(sm.tmem_slot), kTmemCols);
+      tmem_relinquish_pair();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (CG == 1) __syncthreads();
+  else cluster_sync();          // barriers of both CTAs initialised before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *sm.tmem_slot;
   volatile int* abort_flag = sm.abort_flag;
 
+  // everything above touched only this CTA's own resources; from here on the kernel reads
+  // what the compaction and gather kernels wrote
+  pdl_wait();
+  pdl_launch_dependents();
   const int count = *count_ptr;
-  const Plan pl = Plan::make(count < 0 ? 0 : (count > n_cap ? n_cap : count), V, gridDim.x, gmax);
-  const int cta = blockIdx.x;
+  const Plan pl = Plan::make(count < 0 ? 0 : (count > n_cap ? n_cap : count), V,
+                             static_cast<int>(gridDim.x) / CG, gmax, C::BM);
+  const int holder = static_cast<int>(blockIdx.x) / CG;
   const int KB = d / BK;
 
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------ TMA producer ------------------------------
+      // Each CTA stages its own 128 rows of Hm and 256/CG rows of W.  With CG = 2 the
+      // completion is counted on the leader's full barrier (the address with the peer bit
+      // cleared), which the leader arms for the bytes of both CTAs.
       uint32_t it = 0;
       bool ok = true;
       for (int g = 0; g < pl.ngroups && ok; ++g) {
         Unit u;
-        if (!unit_of(pl, g, cta, u)) continue;
+        if (!unit_of(pl, g, holder, u)) continue;
+        const int a_row = u.m_tile * C::BM + static_cast<int>(rank) * C::BM_CTA;
         for (int n = u.n0; n < u.n1 && ok; ++n) {
+          const int b_row = n * BN + static_cast<int>(rank) * C::B_ROWS;
           for (int kb = 0; kb < KB; ++kb, ++it) {
-            const int s = it % kStages;
-            const uint32_t ph = (it / kStages) & 1u;
+            const int s = it % C::kStages;
+            const uint32_t ph = (it / C::kStages) & 1u;
             if (!mbar_wait(smem_u32(&sm.empty[s]), ph ^ 1u, abort_flag, status)) { ok = false; break; }
             const uint32_t fb = smem_u32(&sm.full[s]);
-            mbar_arrive_expect_tx(fb, STAGE_BYTES);
-            tma_load_2d(smem_u32(sm.a + s * A_BYTES), &tmA, fb, kb * BK, u.m_tile * BM);
-            tma_load_2d(smem_u32(sm.b + s * B_BYTES), &tmB, fb, kb * BK, n * BN);
+            if constexpr (CG == 1) {
+              mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+              tma_load_2d(smem_u32(sm.a + s * C::A_BYTES), &tmA, fb, kb * BK, a_row);
+              tma_load_2d(smem_u32(sm.b + s * C::B_BYTES), &tmB, fb, kb * BK, b_row);
+            } else {
+              if (leader) mbar_arrive_expect_tx(fb, CG * C::STAGE_BYTES);
+              const uint32_t fb_leader = fb & kPeerBitMask;
+              tma_load_2d_pair(smem_u32(sm.a + s * C::A_BYTES), &tmA, fb_leader, kb * BK, a_row);
+              tma_load_2d_pair(smem_u32(sm.b + s * C::B_BYTES), &tmB, fb_leader, kb * BK, b_row);
+            }
           }
         }
       }
-      if (!ok) {
-        // Let the loads already issued land before the CTA's shared memory goes away.
-        const uint32_t first = it > static_cast<uint32_t>(kStages) ? it - kStages : 0u;
-        for (uint32_t j = first; j < it; ++j)
-          mbar_wait_drain(smem_u32(&sm.full[j % kStages]), (j / kStages) & 1u, status);
-      }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       // ------------------------------ MMA issuer --------------------------------
       uint32_t it = 0, tile = 0;
       bool ok = true;
       for (int g = 0; g < pl.ngroups && ok; ++g) {
         Unit u;
-        if (!unit_of(pl, g, cta, u)) continue;
+        if (!unit_of(pl, g, holder, u)) continue;
         for (int n = u.n0; n < u.n1 && ok; ++n, ++tile) {
           const uint32_t buf = tile & 1u, tph = (tile >> 1) & 1u;
           if (!mbar_wait(smem_u32(&sm.tempty[buf]), tph ^ 1u, abort_flag, status)) { ok = false; break; }
           tc_fence_after();
           const uint32_t d_tmem = tmem_base + buf * BN;
           for (int kb = 0; kb < KB; ++kb, ++it) {
-            const int s = it % kStages;
-            const uint32_t ph = (it / kStages) & 1u;
+            const int s = it % C::kStages;
+            const uint32_t ph = (it / C::kStages) & 1u;
             if (!mbar_wait(smem_u32(&sm.full[s]), ph, abort_flag, status)) { ok = false; break; }
             tc_fence_after();
-            const uint64_t adesc = sw128_kmajor_desc(smem_u32(sm.a + s * A_BYTES));
-            const uint64_t bdesc = sw128_kmajor_desc(smem_u32(sm.b + s * B_BYTES));
+            const uint64_t adesc = sw128_kmajor_desc(smem_u32(sm.a + s * C::A_BYTES));
+            const uint64_t bdesc = sw128_kmajor_desc(smem_u32(sm.b + s * C::B_BYTES));
 #pragma unroll
             for (int k = 0; k < BK / UK; ++k) {
               // advance 16 bf16 = 32 bytes along K inside the swizzle atom
-              umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, kIdesc, (kb | k) != 0 ? 1u : 0u);
+              mma_issue<CG>(d_tmem, adesc + 2 * k, bdesc + 2 * k, C::kIdesc, (kb | k) != 0 ? 1u : 0u);
             }
-            umma_commit(smem_u32(&sm.empty[s]));     // stage free once these MMAs retire
+            mma_commit_all<CG>(smem_u32(&sm.empty[s]));   // stage free once these MMAs retire
           }
           if (!ok) break;
-          umma_commit(smem_u32(&sm.tfull[buf]));     // accumulator ready for the epilogue
+          mma_commit_all<CG>(smem_u32(&sm.tfull[buf]));   // accumulator ready for the epilogues
         }
       }
       if (!ok) {
         // Make sure no MMA is still writing TMEM before the columns are released.
-        umma_commit(smem_u32(sm.drain));
+        mma_commit_all<CG>(smem_u32(sm.drain));
         mbar_wait_drain(smem_u32(sm.drain), 0u, status);
       }
     }
   } else {
     // -------------------------------- epilogue ---------------------------------
     const int q = warp & 3;                      // TMEM lane quadrant of this warp
-    const int row_in_tile = q * 32 + lane;
+    const int row_in_cta = q * 32 + lane;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-    uint32_t tile = 0;
+    uint32_t tile = 0, epi_phase = 0;
     bool ok = true;
+    // all 128 epilogue threads meet; false (warp-uniform) if the CTA is aborting
+    auto epi_sync = [&]() -> bool {
+      mbar_arrive(smem_u32(sm.epi_bar));
+      const bool got = mbar_wait(smem_u32(sm.epi_bar), epi_phase, abort_flag, status);
+      epi_phase ^= 1u;
+      return __all_sync(0xffffffffu, got);
+    };
     for (int g = 0; g < pl.ngroups && ok; ++g) {
       Unit u;
-      if (!unit_of(pl, g, cta, u)) continue;
-      const int row = u.m_tile * BM + row_in_tile;
+      if (!unit_of(pl, g, holder, u)) continue;
+      const int row_in_tile = static_cast<int>(rank) * C::BM_CTA + row_in_cta;
+      const int row = u.m_tile * C::BM + row_in_tile;
       float run_m = -INFINITY, run_s = 0.f;
       int run_a = 0;
       for (int n = u.n0; n < u.n1; ++n, ++tile) {
         const uint32_t buf = tile & 1u, tph = (tile >> 1) & 1u;
         // every lane waits; the vote reconverges the warp before the .sync.aligned loads and
         // makes the abort decision warp-uniform
-        const bool got = mbar_wait(smem_u32(&sm.tfull[buf]), tph, abort_flag, status);
+        const bool got = DLLM_EPI_BACKOFF_NS > 0
+                             ? mbar_wait_backoff(smem_u32(&sm.tfull[buf]), tph, abort_flag, status,
+                                                 DLLM_EPI_BACKOFF_NS)
+                             : mbar_wait(smem_u32(&sm.tfull[buf]), tph, abort_flag, status);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         tc_fence_after();
         const uint32_t taddr = lane_base + buf * BN;
@@ -308,28 +441,71 @@ lmhead_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
           }
         }
         tc_fence_before();
-        mbar_arrive(smem_u32(&sm.tempty[buf]));
+        // release the accumulator: the leader's MMA waits for the epilogues of both CTAs
+        if constexpr (CG == 1) mbar_arrive(smem_u32(&sm.tempty[buf]));
+        else mbar_arrive_cluster(smem_u32(&sm.tempty[buf]), 0u);
       }
       if (!ok) break;
-      if (!kDebugStore && row < pl.count) {
-        const long long e = pl.part_index(g, u.G, u.p, u.m_local * BM + row_in_tile);
-        if (e < part_cap) {
-          part_m[e] = run_m;
-          part_s[e] = run_s;
-          part_a[e] = run_a;
+      if constexpr (!kDebugStore) {
+        const bool valid = row < pl.count;
+        if (u.P == 1) {
+          // the whole vocabulary in one unit: this is the row's final result
+          if (valid) {
+            out_tok[row] = run_a;
+            out_lse[row] = run_m + logf(run_s);
+            out_conf[row] = 1.0f / run_s;
+          }
         } else {
-          atomicOr(status, kStatusBounds);           // cannot happen: workspace sized for it
+          const long long e = pl.part_index(g, u.G, u.p, u.m_local * C::BM + row_in_tile);
+          if (valid) {
+            if (e < part_cap) {
+              part_m[e] = run_m;
+              part_s[e] = run_s;
+              part_a[e] = run_a;
+            } else {
+              atomicOr(status, kStatusBounds);       // cannot happen: workspace sized for it
+            }
+          }
+          // lse_merge, fused: the last of the P units of this m-tile (half) to finish merges
+          // the P partials of its rows.  Writers fence before the counter increment; the
+          // last arriver fences after it and reads the partials through L2.
+          __threadfence();
+          if (!epi_sync()) { ok = false; break; }
+          if (threadIdx.x == 2 * 32) {
+            const int old = atomicAdd(&unit_ctr[u.m_tile * CG + static_cast<int>(rank)], 1);
+            *sm.last_flag = old == u.P - 1 ? 1 : 0;
+          }
+          if (!epi_sync()) { ok = false; break; }
+          if (*sm.last_flag) {
+            __threadfence();
+            if (valid) {
+              int t;
+              float c, l;
+              merge_row(part_m, part_s, part_a, pl.part_index(g, u.G, 0, u.m_local * C::BM + row_in_tile),
+                        static_cast<long long>(u.G) * C::BM, u.P, t, c, l);
+              out_tok[row] = t;
+              out_conf[row] = c;
+              out_lse[row] = l;
+            }
+          }
         }
       }
     }
   }
 
   tc_fence_before();
-  __syncthreads();
+  if constexpr (CG == 1) __syncthreads();
+  else cluster_sync();          // neither CTA leaves while its peer may still touch its smem
+  if (*abort_flag) {
+    // aborted: give TMA loads already in flight time to land before shared memory is freed
+    const unsigned long long t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 2000000ull) { }
+  }
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    if constexpr (CG == 1) tmem_dealloc(tmem_base, kTmemCols);
+    else tmem_dealloc_pair(tmem_base, kTmemCols);
   }
 }
 

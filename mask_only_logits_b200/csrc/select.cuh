@@ -40,6 +40,8 @@ select_unmask_kernel(const float* __restrict__ conf, const int* __restrict__ row
   __shared__ int sh_lo, sh_hi, sh_n, sh_digit, sh_krem, sh_taken;
   __shared__ int warp_cnt[32];
 
+  pdl_wait();
+  pdl_launch_dependents();
   const int b = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // compacted rows of sequence b (clamped: seq_off comes from the device)
@@ -83,9 +85,17 @@ select_unmask_kernel(const float* __restrict__ conf, const int* __restrict__ row
     for (int shift = 24; shift >= 0; shift -= 8) {
       for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
       __syncthreads();
-      for (int r = c0 + tid; r < c1; r += kSelThreads) {
-        const uint32_t u = __float_as_uint(conf[r]);
-        if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+      // warp-aggregated histogram: confidences crowd into few bins (most share their top
+      // bits), so lanes with the same bin add their count once
+      for (int base = c0; base < c1; base += kSelThreads) {
+        const int r = base + tid;
+        uint32_t bin = 0xFFFFFFFFu;
+        if (r < c1) {
+          const uint32_t u = __float_as_uint(conf[r]);
+          if ((u & pmask) == prefix) bin = (u >> shift) & 255u;
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, bin);
+        if (bin != 0xFFFFFFFFu && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
       }
       __syncthreads();
       if (warp == 0) {

@@ -63,13 +63,22 @@ def _rand_bf16(rng, shape, std):
     return torch.from_numpy((rng.standard_normal(shape) * std).astype(np.float32)).to(torch.bfloat16)
 
 
+@pytest.fixture(params=[2, 1], ids=["pair", "single"])
+def variant(request, dl):
+    """Run a test with the paired-SM GEMM (default) and with the single-SM GEMM."""
+    dl.debug_set_gemm_variant(request.param)
+    yield request.param
+    dl.debug_set_gemm_variant(0)
+
+
 @pytest.mark.parametrize("B,L,d,V,p", [(1, 256, 256, 4096, 0.5),      # cfg0 shapes
                                        (2, 200, 128, 1000, 0.7),       # ragged rows, V tail
                                        (1, 300, 64, 300, 1.0),         # one K block, V tail
                                        (1, 1024, 1024, 2048, 0.6),     # many K blocks
                                        (3, 97, 192, 777, 0.9),         # odd everything
-                                       (1, 5, 64, 1, 1.0)])            # V = 1
-def test_lmhead_raw_logits(dl, B, L, d, V, p):
+                                       (1, 5, 64, 1, 1.0),             # V = 1
+                                       (1, 6000, 128, 700, 0.9)])      # several m-tile groups
+def test_lmhead_raw_logits(dl, variant, B, L, d, V, p):
     rng = np.random.default_rng(d + V)
     H = _rand_bf16(rng, (B * L, d), 1.0)
     W = _rand_bf16(rng, (V, d), 0.02)

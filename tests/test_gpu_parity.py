@@ -154,3 +154,24 @@ def test_run_host_matches_device(dl):
     h_out = step.run_host(inp["H"].pin_memory(), inp["M"].pin_memory(), dev["W"])
     assert torch.equal(h_out["idx"], idx_dev)
     assert step.h2d_bytes() == cfg.B * cfg.L * (cfg.d * 2 + 1)
+
+
+@pytest.mark.parametrize("name", ["cfg0", "cfg1"])
+def test_single_sm_variant(dl, name):
+    """The single-SM (cta_group::1) GEMM variant meets the same bar."""
+    dl.debug_set_gemm_variant(1)
+    try:
+        check_step(dl, WL.make_inputs(WL.CONFIGS[name], seed=0), all_rows=True)
+        cfg = WL.custom_config(3, 777, 192, 1000, 16, r=0.9)
+        check_step(dl, WL.make_inputs(cfg, seed=5), all_rows=True)
+    finally:
+        dl.debug_set_gemm_variant(0)
+
+
+def test_pair_variant_large(dl):
+    """The paired-SM (cta_group::2) GEMM on a large workload (default there: single SMs)."""
+    dl.debug_set_gemm_variant(2)
+    try:
+        check_step(dl, WL.make_inputs(WL.CONFIGS["cfg4"], seed=0), all_rows=False, window_rows=True)
+    finally:
+        dl.debug_set_gemm_variant(0)
