@@ -176,6 +176,14 @@ WsLayout ws_layout(int B, int L, int d, int V) {
   const long long cap1 = w1.ngroups * static_cast<long long>(lm::kMaxCtas) * lm::Cfg<1>::BM;
   const long long cap2 = w2.ngroups * static_cast<long long>(lm::kMaxCtas / 2) * lm::Cfg<2>::BM;
   long long cap = cap1 > cap2 ? cap1 : cap2;
+  // a masked count that fits one group may use remainder holders: (P + R) slots of G m-tiles,
+  // with P * G + R <= holders and R < G <= gmax, so fewer than (holders + gmax^2) m-tile rows
+  const long long r1 = (static_cast<long long>(lm::kMaxCtas) + lm::Cfg<1>::kGroupM * lm::Cfg<1>::kGroupM) *
+                       lm::Cfg<1>::BM;
+  const long long r2 = (static_cast<long long>(lm::kMaxCtas / 2) + lm::Cfg<2>::kGroupM * lm::Cfg<2>::kGroupM) *
+                       lm::Cfg<2>::BM;
+  if (r1 > cap) cap = r1;
+  if (r2 > cap) cap = r2;
   if (cap < 1) cap = 1;
   w.part_cap = cap;
   // one counter per (m-tile, CTA of the pair): ceil(n / 128) + 2 covers both variants
@@ -267,8 +275,18 @@ dllm_status run_logits(const LogitsArgs& a, bool debug) {
   const int holders = cg == 2 ? ds->pairs : (ds->sms < lm::kMaxCtas ? ds->sms : lm::kMaxCtas);
   const int bm = cg == 2 ? lm::Cfg<2>::BM : lm::Cfg<1>::BM;
   const int gmax = cg == 2 ? lm::Cfg<2>::kGroupM : lm::Cfg<1>::kGroupM;
-  const lm::Plan worst = lm::Plan::make(static_cast<int>(n), a.V, holders, gmax, bm);
-  if (worst.part_entries() > w.part_cap) return DLLM_ERR_WORKSPACE;   // cannot happen on B200
+  {
+    // largest partial footprint over every masked count: all positions masked, or any
+    // count that fits one group of m-tiles (remainder holders)
+    long long need = lm::Plan::make(static_cast<int>(n), a.V, holders, gmax, bm).part_entries();
+    const long long mt = (n + bm - 1) / bm;
+    for (long long m = 1; m <= mt && m <= gmax; ++m) {
+      const long long c = m * bm < n ? m * bm : n;
+      const long long e = lm::Plan::make(static_cast<int>(c), a.V, holders, gmax, bm).part_entries();
+      if (e > need) need = e;
+    }
+    if (need > w.part_cap) return DLLM_ERR_WORKSPACE;                  // cannot happen on B200
+  }
 
   if ((st = launch_compact(a.M, a.B, a.L, a.row_idx, a.seq_off, a.count, tiles, ds->status, a.s)) != DLLM_OK)
     return st;

@@ -48,6 +48,9 @@
 #ifndef DLLM_STAGES2
 #define DLLM_STAGES2 6            // shared-memory ring depth, CTA-pair variant
 #endif
+#ifndef DLLM_REMAINDER_HOLDERS
+#define DLLM_REMAINDER_HOLDERS 1  // give the last vocabulary columns to otherwise idle holders
+#endif
 #ifndef DLLM_EPI_BACKOFF_NS
 #define DLLM_EPI_BACKOFF_NS 0     // epilogue: sleep between polls of the accumulator barrier
 #endif
@@ -84,9 +87,22 @@ struct Cfg {
                                      (static_cast<uint32_t>(BM >> 4) << 24);
 };
 
-// The unit schedule, computed identically by the GEMM's roles and by lse_merge.
+// The unit schedule, computed identically by every role of the GEMM.
+//
+// m-tiles are taken in groups of up to gmax.  Inside a group of G m-tiles each holder takes
+// one m-tile and a contiguous range of vocabulary tiles: P = ctas / G "streams" per m-tile,
+// holder h on m-tile h % G and stream h / G, so the holders of one stream walk the same W
+// tiles at the same time and each W tile is fetched from HBM about once per group.
+//
+// Remainder holders (a problem that fits one group, when G does not divide the holders):
+// the streams take exactly rb = numN / P tiles each, and the last rr = numN - P * rb
+// vocabulary columns of every m-tile (G * rr tiles, in m-major order) are split among the
+// R = ctas - G * P holders the streams leave idle.  Every holder then runs at most
+// max(rb, ceil(G * rr / R)) tiles instead of ceil(numN / P).
 struct Plan {
   int count, bm, numM, numN, ctas, gmax, ngroups, P_full;
+  bool rem;        // remainder holders in use (implies ngroups == 1)
+  int R, rb, rr;
 
   // ctas = number of work holders (CTAs for CG = 1, CTA pairs for CG = 2);
   // bm = rows per m-tile.
@@ -100,6 +116,20 @@ struct Plan {
     p.gmax = gmax < ctas ? gmax : ctas;
     p.ngroups = (p.numM + p.gmax - 1) / p.gmax;
     p.P_full = streams(p.gmax, p.ctas, p.numN);
+    p.rem = false;
+    p.R = p.rb = p.rr = 0;
+    if (DLLM_REMAINDER_HOLDERS && p.ngroups == 1) {
+      const int G = p.numM, P = streams(G, ctas, p.numN);
+      const int R = ctas - G * P, rb = p.numN / P, rr = p.numN - P * rb;
+      // only when it shortens the busiest holder: max(rb, ceil(G rr / R)) < ceil(numN / P)
+      const int busiest_rem = R > 0 ? (rb > (G * rr + R - 1) / R ? rb : (G * rr + R - 1) / R) : 0;
+      if (R > 0 && rr > 0 && busiest_rem < rb + 1) {
+        p.rem = true;
+        p.R = R;
+        p.rb = rb;
+        p.rr = rr;
+      }
+    }
     return p;
   }
   __host__ __device__ static int streams(int G, int ctas, int numN) {
@@ -110,32 +140,90 @@ struct Plan {
   __host__ __device__ int group_size(int g) const {
     return g == ngroups - 1 ? numM - g * gmax : gmax;
   }
-  // Partial-buffer index of (group g of size G, stream p, row r within the group).
-  __host__ __device__ long long part_index(int g, int G, int p, int r) const {
-    return static_cast<long long>(g) * gmax * bm * P_full + static_cast<long long>(p) * G * bm + r;
+  // Partial-buffer index of (group g of size G, slot, row r within the group).  Slots:
+  // streams 0..P-1, then remainder holders P..P+R-1.
+  __host__ __device__ long long part_index(int g, int G, int slot, int r) const {
+    return static_cast<long long>(g) * gmax * bm * P_full + static_cast<long long>(slot) * G * bm + r;
   }
   // Number of partial entries written for this count.
   __host__ __device__ long long part_entries() const {
     if (ngroups == 0) return 0;
     const int Gl = group_size(ngroups - 1);
-    return part_index(ngroups - 1, Gl, 0, 0) +
-           static_cast<long long>(Gl) * bm * streams(Gl, ctas, numN);
+    const int slots = streams(Gl, ctas, numN) + (rem ? R : 0);
+    return part_index(ngroups - 1, Gl, 0, 0) + static_cast<long long>(Gl) * bm * slots;
+  }
+  // Remainder holder j: its tiles [i0, i1) of the m-major remainder list, tile i being
+  // vocabulary column P * rb + i % rr of m-tile i / rr.
+  __host__ __device__ void leftover_range(int j, int G, long long& i0, long long& i1) const {
+    const long long T = static_cast<long long>(G) * rr;
+    i0 = T * j / R;
+    i1 = T * (j + 1) / R;
+  }
+  // Remainder holders whose tiles include m-tile m: j_lo..j_hi (none if j_lo > j_hi).
+  __host__ __device__ void leftovers_of(int m, int G, int& j_lo, int& j_hi) const {
+    j_lo = R;
+    j_hi = -1;
+    for (int j = 0; j < R; ++j) {
+      long long i0, i1;
+      leftover_range(j, G, i0, i1);
+      if (i1 > i0 && i0 < static_cast<long long>(m + 1) * rr && i1 > static_cast<long long>(m) * rr) {
+        if (j < j_lo) j_lo = j;
+        j_hi = j;
+      }
+    }
   }
 };
 
-// One unit of a work holder inside group g, or false if it is idle in this group.
+// The unit of a holder inside group g: a stream (one m-tile, vocabulary tiles [n0, n1)) or a
+// remainder holder (remainder tiles [i0, i1)); false if the holder is idle in this group.
 struct Unit {
   int m_tile, m_local, G, p, P, n0, n1;
+  bool leftover;
+  long long i0, i1;
 };
 __device__ __forceinline__ bool unit_of(const Plan& pl, int g, int holder, Unit& u) {
   u.G = pl.group_size(g);
   u.P = Plan::streams(u.G, pl.ctas, pl.numN);
-  if (holder >= u.G * u.P) return false;
-  u.m_local = holder % u.G;
-  u.m_tile = g * pl.gmax + u.m_local;
-  u.p = holder / u.G;
-  u.n0 = static_cast<int>(static_cast<long long>(u.p) * pl.numN / u.P);
-  u.n1 = static_cast<int>(static_cast<long long>(u.p + 1) * pl.numN / u.P);
+  u.leftover = false;
+  if (holder < u.G * u.P) {
+    u.m_local = holder % u.G;
+    u.m_tile = g * pl.gmax + u.m_local;
+    u.p = holder / u.G;
+    if (pl.rem) {
+      u.n0 = u.p * pl.rb;
+      u.n1 = u.n0 + pl.rb;
+    } else {
+      u.n0 = static_cast<int>(static_cast<long long>(u.p) * pl.numN / u.P);
+      u.n1 = static_cast<int>(static_cast<long long>(u.p + 1) * pl.numN / u.P);
+    }
+    return true;
+  }
+  if (pl.rem && holder < u.G * u.P + pl.R) {
+    const int j = holder - u.G * u.P;
+    u.leftover = true;
+    u.p = u.P + j;
+    pl.leftover_range(j, u.G, u.i0, u.i1);
+    return u.i1 > u.i0;
+  }
+  return false;
+}
+
+// Calls f(m_tile, n) for every tile of the holder, in order; stops early when f returns
+// false.  Returns whether all calls returned true.
+template <class F>
+__device__ __forceinline__ bool for_each_tile(const Plan& pl, int holder, F& f) {
+  for (int g = 0; g < pl.ngroups; ++g) {
+    Unit u;
+    if (!unit_of(pl, g, holder, u)) continue;
+    if (u.leftover) {
+      for (long long i = u.i0; i < u.i1; ++i)
+        if (!f(g * pl.gmax + static_cast<int>(i / pl.rr), u.P * pl.rb + static_cast<int>(i % pl.rr)))
+          return false;
+    } else {
+      for (int n = u.n0; n < u.n1; ++n)
+        if (!f(u.m_tile, n)) return false;
+    }
+  }
   return true;
 }
 
@@ -204,26 +292,24 @@ __device__ __forceinline__ void fold_chunk(float (&v)[32], int col0, int V, floa
   run_s += (s0 + s1) + (s2 + s3);
 }
 
-// lse_merge of one row: combine n_split partials (m_j, s_j, a_j) found at base + j * stride
-// (j = 0..n_split-1, ascending vocabulary ranges):
-//   m* = max_j m_j, s* = sum_j s_j exp(m_j - m*), tok = a_j of the first j with m_j = m*,
-//   lse = m* + ln s*, conf = exp(m* - lse) = 1 / s*.
-// Partials are read through L2 (they may have been written by other CTAs of the running
-// kernel) in batches of 8 whose loads are all issued before any is used.
-__device__ __forceinline__ void merge_row(const float* __restrict__ pm, const float* __restrict__ ps,
+// lse_merge of one row, as an accumulation: fold the partials (m_j, s_j, a_j) found at
+// base + j * stride for j = j0..j1-1 (ascending vocabulary ranges) into (m, s, a):
+//   m* = max_j m_j, s* = sum_j s_j exp(m_j - m*), a = a_j of the first j with m_j = m*.
+// Then lse = m* + ln s* and conf = exp(m* - lse) = 1 / s* (merge_finish).  Partials are read
+// through L2 (other CTAs of the running kernel may have written them) in batches of 8 whose
+// loads are all issued before any is used.
+__device__ __forceinline__ void merge_acc(const float* __restrict__ pm, const float* __restrict__ ps,
                                           const int* __restrict__ pa, long long base,
-                                          long long stride, int n_split, int& tok, float& conf,
-                                          float& lse) {
+                                          long long stride, int j0, int j1, float& m, float& s,
+                                          int& a) {
   constexpr int kBatch = 8;
-  float m = -INFINITY, s = 0.f;
-  int a = 0;
-  for (int j0 = 0; j0 < n_split; j0 += kBatch) {
+  for (int jb = j0; jb < j1; jb += kBatch) {
     float mb[kBatch], sb[kBatch];
     int ab[kBatch];
 #pragma unroll
     for (int t = 0; t < kBatch; ++t) {
-      if (j0 + t < n_split) {
-        const long long e = base + (j0 + t) * stride;
+      if (jb + t < j1) {
+        const long long e = base + (jb + t) * stride;
         mb[t] = __ldcg(pm + e);
         sb[t] = __ldcg(ps + e);
         ab[t] = __ldcg(pa + e);
@@ -235,8 +321,8 @@ __device__ __forceinline__ void merge_row(const float* __restrict__ pm, const fl
     }
 #pragma unroll
     for (int t = 0; t < kBatch; ++t) {
-      if (j0 + t >= n_split) break;
-      if (mb[t] > m) {               // strict: the earlier split keeps a tie
+      if (mb[t] == -INFINITY) continue;   // empty partial (or past j1): nothing to add
+      if (mb[t] > m) {                    // strict: the earlier split keeps a tie
         s = s * ex2_approx((m - mb[t]) * kLog2e) + sb[t];
         m = mb[t];
         a = ab[t];
@@ -245,9 +331,23 @@ __device__ __forceinline__ void merge_row(const float* __restrict__ pm, const fl
       }
     }
   }
+}
+
+__device__ __forceinline__ void merge_finish(float m, float s, int a, int& tok, float& conf,
+                                             float& lse) {
   tok = a;
   lse = m + logf(s);
   conf = 1.0f / s;
+}
+
+__device__ __forceinline__ void merge_row(const float* __restrict__ pm, const float* __restrict__ ps,
+                                          const int* __restrict__ pa, long long base,
+                                          long long stride, int n_split, int& tok, float& conf,
+                                          float& lse) {
+  float m = -INFINITY, s = 0.f;
+  int a = 0;
+  merge_acc(pm, ps, pa, base, stride, 0, n_split, m, s, a);
+  merge_finish(m, s, a, tok, conf, lse);
 }
 
 template <int CG>
@@ -330,64 +430,57 @@ lmhead_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
       // completion is counted on the leader's full barrier (the address with the peer bit
       // cleared), which the leader arms for the bytes of both CTAs.
       uint32_t it = 0;
-      bool ok = true;
-      for (int g = 0; g < pl.ngroups && ok; ++g) {
-        Unit u;
-        if (!unit_of(pl, g, holder, u)) continue;
-        const int a_row = u.m_tile * C::BM + static_cast<int>(rank) * C::BM_CTA;
-        for (int n = u.n0; n < u.n1 && ok; ++n) {
-          const int b_row = n * BN + static_cast<int>(rank) * C::B_ROWS;
-          for (int kb = 0; kb < KB; ++kb, ++it) {
-            const int s = it % C::kStages;
-            const uint32_t ph = (it / C::kStages) & 1u;
-            if (!mbar_wait(smem_u32(&sm.empty[s]), ph ^ 1u, abort_flag, status)) { ok = false; break; }
-            const uint32_t fb = smem_u32(&sm.full[s]);
-            if constexpr (CG == 1) {
-              mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
-              tma_load_2d(smem_u32(sm.a + s * C::A_BYTES), &tmA, fb, kb * BK, a_row);
-              tma_load_2d(smem_u32(sm.b + s * C::B_BYTES), &tmB, fb, kb * BK, b_row);
-            } else {
-              if (leader) mbar_arrive_expect_tx(fb, CG * C::STAGE_BYTES);
-              const uint32_t fb_leader = fb & kPeerBitMask;
-              tma_load_2d_pair(smem_u32(sm.a + s * C::A_BYTES), &tmA, fb_leader, kb * BK, a_row);
-              tma_load_2d_pair(smem_u32(sm.b + s * C::B_BYTES), &tmB, fb_leader, kb * BK, b_row);
-            }
+      auto load_tile = [&](int m_tile, int n) -> bool {
+        const int a_row = m_tile * C::BM + static_cast<int>(rank) * C::BM_CTA;
+        const int b_row = n * BN + static_cast<int>(rank) * C::B_ROWS;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % C::kStages;
+          const uint32_t ph = (it / C::kStages) & 1u;
+          if (!mbar_wait(smem_u32(&sm.empty[s]), ph ^ 1u, abort_flag, status)) return false;
+          const uint32_t fb = smem_u32(&sm.full[s]);
+          if constexpr (CG == 1) {
+            mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+            tma_load_2d(smem_u32(sm.a + s * C::A_BYTES), &tmA, fb, kb * BK, a_row);
+            tma_load_2d(smem_u32(sm.b + s * C::B_BYTES), &tmB, fb, kb * BK, b_row);
+          } else {
+            if (leader) mbar_arrive_expect_tx(fb, CG * C::STAGE_BYTES);
+            const uint32_t fb_leader = fb & kPeerBitMask;
+            tma_load_2d_pair(smem_u32(sm.a + s * C::A_BYTES), &tmA, fb_leader, kb * BK, a_row);
+            tma_load_2d_pair(smem_u32(sm.b + s * C::B_BYTES), &tmB, fb_leader, kb * BK, b_row);
           }
         }
-      }
+        return true;
+      };
+      for_each_tile(pl, holder, load_tile);
     }
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       // ------------------------------ MMA issuer --------------------------------
       uint32_t it = 0, tile = 0;
-      bool ok = true;
-      for (int g = 0; g < pl.ngroups && ok; ++g) {
-        Unit u;
-        if (!unit_of(pl, g, holder, u)) continue;
-        for (int n = u.n0; n < u.n1 && ok; ++n, ++tile) {
-          const uint32_t buf = tile & 1u, tph = (tile >> 1) & 1u;
-          if (!mbar_wait(smem_u32(&sm.tempty[buf]), tph ^ 1u, abort_flag, status)) { ok = false; break; }
+      auto mma_tile = [&](int, int) -> bool {
+        const uint32_t buf = tile & 1u, tph = (tile >> 1) & 1u;
+        if (!mbar_wait(smem_u32(&sm.tempty[buf]), tph ^ 1u, abort_flag, status)) return false;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * BN;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % C::kStages;
+          const uint32_t ph = (it / C::kStages) & 1u;
+          if (!mbar_wait(smem_u32(&sm.full[s]), ph, abort_flag, status)) return false;
           tc_fence_after();
-          const uint32_t d_tmem = tmem_base + buf * BN;
-          for (int kb = 0; kb < KB; ++kb, ++it) {
-            const int s = it % C::kStages;
-            const uint32_t ph = (it / C::kStages) & 1u;
-            if (!mbar_wait(smem_u32(&sm.full[s]), ph, abort_flag, status)) { ok = false; break; }
-            tc_fence_after();
-            const uint64_t adesc = sw128_kmajor_desc(smem_u32(sm.a + s * C::A_BYTES));
-            const uint64_t bdesc = sw128_kmajor_desc(smem_u32(sm.b + s * C::B_BYTES));
+          const uint64_t adesc = sw128_kmajor_desc(smem_u32(sm.a + s * C::A_BYTES));
+          const uint64_t bdesc = sw128_kmajor_desc(smem_u32(sm.b + s * C::B_BYTES));
 #pragma unroll
-            for (int k = 0; k < BK / UK; ++k) {
-              // advance 16 bf16 = 32 bytes along K inside the swizzle atom
-              mma_issue<CG>(d_tmem, adesc + 2 * k, bdesc + 2 * k, C::kIdesc, (kb | k) != 0 ? 1u : 0u);
-            }
-            mma_commit_all<CG>(smem_u32(&sm.empty[s]));   // stage free once these MMAs retire
+          for (int k = 0; k < BK / UK; ++k) {
+            // advance 16 bf16 = 32 bytes along K inside the swizzle atom
+            mma_issue<CG>(d_tmem, adesc + 2 * k, bdesc + 2 * k, C::kIdesc, (kb | k) != 0 ? 1u : 0u);
           }
-          if (!ok) break;
-          mma_commit_all<CG>(smem_u32(&sm.tfull[buf]));   // accumulator ready for the epilogues
+          mma_commit_all<CG>(smem_u32(&sm.empty[s]));   // stage free once these MMAs retire
         }
-      }
-      if (!ok) {
+        mma_commit_all<CG>(smem_u32(&sm.tfull[buf]));     // accumulator ready for the epilogues
+        ++tile;
+        return true;
+      };
+      if (!for_each_tile(pl, holder, mma_tile)) {
         // Make sure no MMA is still writing TMEM before the columns are released.
         mma_commit_all<CG>(smem_u32(sm.drain));
         mbar_wait_drain(smem_u32(sm.drain), 0u, status);
@@ -397,6 +490,7 @@ lmhead_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     // -------------------------------- epilogue ---------------------------------
     const int q = warp & 3;                      // TMEM lane quadrant of this warp
     const int row_in_cta = q * 32 + lane;
+    const int row_in_tile = static_cast<int>(rank) * C::BM_CTA + row_in_cta;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     uint32_t tile = 0, epi_phase = 0;
     bool ok = true;
@@ -407,88 +501,126 @@ lmhead_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
       epi_phase ^= 1u;
       return __all_sync(0xffffffffu, got);
     };
+    // fold the next accumulator (vocabulary tile n of m-tile m_tile) into (rm, rs, ra)
+    auto consume = [&](int m_tile, int n, float& rm, float& rs, int& ra) -> bool {
+      const uint32_t buf = tile & 1u, tph = (tile >> 1) & 1u;
+      // every lane waits; the vote reconverges the warp before the .sync.aligned loads and
+      // makes the abort decision warp-uniform
+      const bool got = DLLM_EPI_BACKOFF_NS > 0
+                           ? mbar_wait_backoff(smem_u32(&sm.tfull[buf]), tph, abort_flag, status,
+                                               DLLM_EPI_BACKOFF_NS)
+                           : mbar_wait(smem_u32(&sm.tfull[buf]), tph, abort_flag, status);
+      if (!__all_sync(0xffffffffu, got)) return false;
+      tc_fence_after();
+      const uint32_t taddr = lane_base + buf * BN;
+      const int row = m_tile * C::BM + row_in_tile;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        tmem_ld32(taddr + c * 32, v);
+        tmem_ld_wait();
+        const int col0 = n * BN + c * 32;
+        if constexpr (kDebugStore) {
+          if (row < pl.count) {
+            for (int j = 0; j < 32; ++j)
+              if (col0 + j < V) dbg_logits[static_cast<size_t>(row) * V + col0 + j] = v[j];
+          }
+        } else {
+          fold_chunk(v, col0, V, rm, rs, ra);
+        }
+      }
+      tc_fence_before();
+      // release the accumulator: the leader's MMA waits for the epilogues of both CTAs
+      if constexpr (CG == 1) mbar_arrive(smem_u32(&sm.tempty[buf]));
+      else mbar_arrive_cluster(smem_u32(&sm.tempty[buf]), 0u);
+      ++tile;
+      return true;
+    };
+    auto write_result = [&](int row, float m, float s_, int a) {
+      out_tok[row] = a;
+      out_lse[row] = m + logf(s_);
+      out_conf[row] = 1.0f / s_;
+    };
+    auto write_partial = [&](long long e, float m, float s_, int a) {
+      if (e < part_cap) {
+        part_m[e] = m;
+        part_s[e] = s_;
+        part_a[e] = a;
+      } else {
+        atomicOr(status, kStatusBounds);             // cannot happen: workspace sized for it
+      }
+    };
+
+    // A finished (m-tile, slot) state: the result itself when the m-tile has a single unit,
+    // else a partial; the last of the m-tile's units to finish merges its rows.
+    auto finish = [&](int g, const Unit& u, int m_local, int slot, float rm, float rs, int ra) -> bool {
+      const int m_tile = g * pl.gmax + m_local;
+      const int row = m_tile * C::BM + row_in_tile;
+      const bool valid = row < pl.count;
+      int j_lo = 0, j_hi = -1;
+      if (pl.rem) pl.leftovers_of(m_local, u.G, j_lo, j_hi);
+      const int units = u.P + (j_hi >= j_lo ? j_hi - j_lo + 1 : 0);
+      if (units == 1) {
+        if (valid) write_result(row, rm, rs, ra);
+        return true;
+      }
+      if (valid) write_partial(pl.part_index(g, u.G, slot, m_local * C::BM + row_in_tile), rm, rs, ra);
+      // Writers fence before the counter increment; the last arriver fences after it and
+      // reads the partials through L2.
+      __threadfence();
+      if (!epi_sync()) return false;
+      if (threadIdx.x == 2 * 32) {
+        const int old = atomicAdd(&unit_ctr[m_tile * CG + static_cast<int>(rank)], 1);
+        *sm.last_flag = old == units - 1 ? 1 : 0;
+      }
+      if (!epi_sync()) return false;
+      if (*sm.last_flag) {
+        __threadfence();
+        if (valid) {
+          const long long base = pl.part_index(g, u.G, 0, m_local * C::BM + row_in_tile);
+          const long long stride = static_cast<long long>(u.G) * C::BM;
+          float m = -INFINITY, s_ = 0.f;
+          int a = 0;
+          merge_acc(part_m, part_s, part_a, base, stride, 0, u.P, m, s_, a);
+          if (j_hi >= j_lo) merge_acc(part_m, part_s, part_a, base, stride, u.P + j_lo, u.P + j_hi + 1, m, s_, a);
+          int t;
+          float c, l;
+          merge_finish(m, s_, a, t, c, l);
+          out_tok[row] = t;
+          out_conf[row] = c;
+          out_lse[row] = l;
+        }
+      }
+      return true;
+    };
+
     for (int g = 0; g < pl.ngroups && ok; ++g) {
       Unit u;
       if (!unit_of(pl, g, holder, u)) continue;
-      const int row_in_tile = static_cast<int>(rank) * C::BM_CTA + row_in_cta;
-      const int row = u.m_tile * C::BM + row_in_tile;
-      float run_m = -INFINITY, run_s = 0.f;
-      int run_a = 0;
-      for (int n = u.n0; n < u.n1; ++n, ++tile) {
-        const uint32_t buf = tile & 1u, tph = (tile >> 1) & 1u;
-        // every lane waits; the vote reconverges the warp before the .sync.aligned loads and
-        // makes the abort decision warp-uniform
-        const bool got = DLLM_EPI_BACKOFF_NS > 0
-                             ? mbar_wait_backoff(smem_u32(&sm.tfull[buf]), tph, abort_flag, status,
-                                                 DLLM_EPI_BACKOFF_NS)
-                             : mbar_wait(smem_u32(&sm.tfull[buf]), tph, abort_flag, status);
-        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t taddr = lane_base + buf * BN;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          float v[32];
-          tmem_ld32(taddr + c * 32, v);
-          tmem_ld_wait();
-          const int col0 = n * BN + c * 32;
-          if constexpr (kDebugStore) {
-            if (row < pl.count) {
-              for (int j = 0; j < 32; ++j)
-                if (col0 + j < V) dbg_logits[static_cast<size_t>(row) * V + col0 + j] = v[j];
-            }
-          } else {
-            fold_chunk(v, col0, V, run_m, run_s, run_a);
+      if (u.leftover) {
+        // remainder tiles in m-major order: one running state, finished at each m-tile change
+        int cur = -1;
+        float rm = -INFINITY, rs = 0.f;
+        int ra = 0;
+        for (long long i = u.i0; i < u.i1 && ok; ++i) {
+          const int m_local = static_cast<int>(i / pl.rr);
+          const int n = u.P * pl.rb + static_cast<int>(i % pl.rr);
+          if (m_local != cur) {
+            if (cur >= 0 && !kDebugStore) ok = finish(g, u, cur, u.p, rm, rs, ra);
+            cur = m_local;
+            rm = -INFINITY;
+            rs = 0.f;
+            ra = 0;
           }
+          if (ok && !consume(g * pl.gmax + m_local, n, rm, rs, ra)) ok = false;
         }
-        tc_fence_before();
-        // release the accumulator: the leader's MMA waits for the epilogues of both CTAs
-        if constexpr (CG == 1) mbar_arrive(smem_u32(&sm.tempty[buf]));
-        else mbar_arrive_cluster(smem_u32(&sm.tempty[buf]), 0u);
-      }
-      if (!ok) break;
-      if constexpr (!kDebugStore) {
-        const bool valid = row < pl.count;
-        if (u.P == 1) {
-          // the whole vocabulary in one unit: this is the row's final result
-          if (valid) {
-            out_tok[row] = run_a;
-            out_lse[row] = run_m + logf(run_s);
-            out_conf[row] = 1.0f / run_s;
-          }
-        } else {
-          const long long e = pl.part_index(g, u.G, u.p, u.m_local * C::BM + row_in_tile);
-          if (valid) {
-            if (e < part_cap) {
-              part_m[e] = run_m;
-              part_s[e] = run_s;
-              part_a[e] = run_a;
-            } else {
-              atomicOr(status, kStatusBounds);       // cannot happen: workspace sized for it
-            }
-          }
-          // lse_merge, fused: the last of the P units of this m-tile (half) to finish merges
-          // the P partials of its rows.  Writers fence before the counter increment; the
-          // last arriver fences after it and reads the partials through L2.
-          __threadfence();
-          if (!epi_sync()) { ok = false; break; }
-          if (threadIdx.x == 2 * 32) {
-            const int old = atomicAdd(&unit_ctr[u.m_tile * CG + static_cast<int>(rank)], 1);
-            *sm.last_flag = old == u.P - 1 ? 1 : 0;
-          }
-          if (!epi_sync()) { ok = false; break; }
-          if (*sm.last_flag) {
-            __threadfence();
-            if (valid) {
-              int t;
-              float c, l;
-              merge_row(part_m, part_s, part_a, pl.part_index(g, u.G, 0, u.m_local * C::BM + row_in_tile),
-                        static_cast<long long>(u.G) * C::BM, u.P, t, c, l);
-              out_tok[row] = t;
-              out_conf[row] = c;
-              out_lse[row] = l;
-            }
-          }
-        }
+        if (ok && cur >= 0 && !kDebugStore) ok = finish(g, u, cur, u.p, rm, rs, ra);
+      } else {
+        float rm = -INFINITY, rs = 0.f;
+        int ra = 0;
+        for (int n = u.n0; n < u.n1 && ok; ++n)
+          if (!consume(u.m_tile, n, rm, rs, ra)) ok = false;
+        if (ok && !kDebugStore) ok = finish(g, u, u.m_local, u.p, rm, rs, ra);
       }
     }
   }

@@ -77,7 +77,11 @@ def variant(request, dl):
                                        (1, 1024, 1024, 2048, 0.6),     # many K blocks
                                        (3, 97, 192, 777, 0.9),         # odd everything
                                        (1, 5, 64, 1, 1.0),             # V = 1
-                                       (1, 6000, 128, 700, 0.9)])      # several m-tile groups
+                                       (1, 6000, 128, 700, 0.9),       # several m-tile groups
+                                       (1, 2048, 64, 3000, 1.0),       # 8 m-tiles of 256
+                                       (1, 2300, 64, 2000, 1.0),       # 9 of 256 / 18 of 128: streams
+                                       (1, 1000, 64, 20000, 1.0),      # 8 m-tiles of 128
+                                       (1, 1000, 64, 37800, 1.0)])     # remainder holders
 def test_lmhead_raw_logits(dl, variant, B, L, d, V, p):
     rng = np.random.default_rng(d + V)
     H = _rand_bf16(rng, (B * L, d), 1.0)

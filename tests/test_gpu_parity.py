@@ -115,6 +115,10 @@ def test_cfg1_every_row(dl):
     check_step(dl, WL.make_inputs(WL.CONFIGS["cfg1"], seed=0), all_rows=True)
 
 
+def test_cfg1_m64_every_row(dl):
+    check_step(dl, WL.make_inputs(WL.CONFIGS["cfg1_m64"], seed=0), all_rows=True)
+
+
 def test_cfg2_sampled(dl):
     check_step(dl, WL.make_inputs(WL.CONFIGS["cfg2"], seed=0), all_rows=False)
 
@@ -137,6 +141,9 @@ def test_cfg4_sampled_and_windows(dl):
     (2, 100, 64, 1, 3, "bernoulli", 0.5),        # V = 1: conf = 1, lse = the logit
     (4, 50, 64, 300, 4, "bernoulli", 0.0),       # nothing masked
     (1, 40000, 256, 4096, 1024, "bernoulli", 0.7),   # many m-tiles, largest k
+    (1, 2048, 128, 5000, 16, "bernoulli", 1.0),      # 8 m-tiles of 256 rows
+    (1, 1000, 64, 37800, 32, "bernoulli", 1.0),      # remainder holders (both variants)
+    (1, 12000, 64, 3000, 8, "bernoulli", 0.08),      # sparse mask, few m-tiles of a long L
 ])
 def test_edge_shapes(dl, B, L, d, V, k, mask, r):
     cfg = WL.custom_config(B, L, d, V, k, mask=mask, r=r)

@@ -14,6 +14,8 @@ Taming", Abstract and Fig. 3 (128k context, mask-ratio sweep), and the Sparse-dL
   cfg1   B=1 L=4096   d=4096 V=126464  last 1024 positions masked     k=32
   cfg2   B=1 L=32768  d=4096 V=126464  Bernoulli(0.9) mask            k=64
   cfg3x  B=1 L=131072 d=4096 V=126464  Bernoulli(r), r=0.1/0.5/0.9    k=128
+  cfg1_m64  cfg1's shapes with only the last 64 positions masked (few rows: W streaming
+         from HBM bounds the step, not the tensor cores)
   cfg4   B=8 L=8192   d=2048 V=151936  semi-autoregressive blocks of 32: sequence b's
          current block is block 32*b+16; it and every later position are masked, earlier
          ones are not; unmask candidates are the positions of the current block; k=4
@@ -63,6 +65,9 @@ CONFIGS: dict[str, Config] = {
                         r=0.5, description="B1 L131072 d4096 V126464, Bernoulli(0.5), k=128"),
     "cfg3_r0.9": Config("cfg3_r0.9", B=1, L=131072, d=4096, V=126464, k=128, mask="bernoulli",
                         r=0.9, description="B1 L131072 d4096 V126464, Bernoulli(0.9), k=128"),
+    # supplementary, HBM-bound point: cfg1's shapes with only the last 64 positions masked
+    "cfg1_m64": Config("cfg1_m64", B=1, L=4096, d=4096, V=126464, k=32, mask="suffix",
+                       n_suffix=64, description="B1 L4096 d4096 V126464, last 64 masked, k=32"),
     "cfg4": Config("cfg4", B=8, L=8192, d=2048, V=151936, k=4, mask="semi_ar", block=32,
                    description="B8 L8192 d2048 V151936, 32-token blocks, current block "
                                "32b+16 and later masked, window = current block, k=4"),
