@@ -156,6 +156,26 @@ dllm_status dllm_masked_logits(const uint16_t* H, const uint8_t* M, const uint16
                                void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * dllm_masked_logits_ex - dllm_masked_logits plus alternative certainty scores of each
+ * masked row's softmax p (confidence/entropy-driven unmasking, dLLM inference survey page,
+ * "Main Findings"):
+ *   DLLM_STAT_ENTROPY  entropy[i] = -sum_v p_v ln p_v           (float32, capacity B*L)
+ *   DLLM_STAT_MARGIN   margin[i]  = p_(1) - p_(2), largest minus second-largest probability
+ * `stats` is a bitwise OR of those flags (0 = dllm_masked_logits); each requested output
+ * pointer must be non-NULL and each other one NULL (else DLLM_ERR_NULL); unknown bits give
+ * DLLM_ERR_SHAPE.  The epilogue keeps sum exp(z - max)(z - max) and the second-largest
+ * logit per row next to the max and the sum of exponentials; no logit is stored.
+ * Other arguments, outputs and errors as in dllm_masked_logits.
+ */
+#define DLLM_STAT_ENTROPY 1u
+#define DLLM_STAT_MARGIN  2u
+dllm_status dllm_masked_logits_ex(const uint16_t* H, const uint8_t* M, const uint16_t* W,
+                                  int32_t B, int32_t L, int32_t d, int32_t V, uint32_t stats,
+                                  int32_t* tok, float* conf, float* lse, float* entropy,
+                                  float* margin, int32_t* row_idx, int32_t* seq_off,
+                                  int32_t* count, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * dllm_select_unmask - per-sequence top-k over confidences (confidence-driven unmasking,
  * dLLM inference survey page, "Main Findings").
  *
@@ -181,6 +201,26 @@ dllm_status dllm_select_unmask(const float* conf, const int32_t* row_idx,
                                const int32_t* tok,
                                int32_t* idx, int32_t* n_sel,
                                int32_t* tok_sel, float* conf_sel, void* stream);
+
+/*
+ * dllm_select_unmask_ex - threshold-based parallel unmasking over any per-row score (the
+ * decoding thresholds of the dLLM pages, Dynamic-dLLM abstract).  Per sequence, among the
+ * candidates of dllm_select_unmask, the number taken is
+ *     min(k, max(min(min_sel, n_candidates), #candidates with score >= threshold)),
+ * the best ones by (score descending, position ascending).  With ascending = 1 smaller
+ * scores are better (e.g. the entropy): candidates qualify with score <= threshold and the
+ * order is (score ascending, position ascending).  min_sel >= 1 guarantees that decoding
+ * advances; threshold = -INFINITY (descending) or +INFINITY (ascending) gives plain top-k.
+ * Scores must not be NaN.  score_sel (nullable) receives the scores of the selected
+ * positions (0 padding).  Errors: as dllm_select_unmask, and DLLM_ERR_SHAPE for
+ * min_sel < 0, a NaN threshold or ascending not 0/1.
+ */
+dllm_status dllm_select_unmask_ex(const float* score, const int32_t* row_idx,
+                                  const int32_t* seq_off, int32_t B, int32_t L, int32_t k,
+                                  float threshold, int32_t min_sel, int32_t ascending,
+                                  const int32_t* win_lo, const int32_t* win_hi,
+                                  const int32_t* tok, int32_t* idx, int32_t* n_sel,
+                                  int32_t* tok_sel, float* score_sel, void* stream);
 
 /*
  * dllm_decode_step - the whole hot path in one call: dllm_masked_logits followed by

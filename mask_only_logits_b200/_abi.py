@@ -21,7 +21,11 @@ PROTOTYPES = {
     "dllm_mask_compact_noalloc": (_st, [_p, _i32, _i32, _p, _p, _p, _p]),
     "dllm_masked_logits": (_st, [_p, _p, _p, _i32, _i32, _i32, _i32, _p, _p, _p, _p, _p, _p,
                                  _p, _sz, _p]),
+    "dllm_masked_logits_ex": (_st, [_p, _p, _p, _i32, _i32, _i32, _i32, ctypes.c_uint32, _p, _p,
+                                    _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
     "dllm_select_unmask": (_st, [_p, _p, _p, _i32, _i32, _i32, _p, _p, _p, _p, _p, _p, _p, _p]),
+    "dllm_select_unmask_ex": (_st, [_p, _p, _p, _i32, _i32, _i32, ctypes.c_float, _i32, _i32, _p,
+                                    _p, _p, _p, _p, _p, _p, _p]),
     "dllm_decode_step": (_st, [_p, _p, _p, _i32, _i32, _i32, _i32, _i32, _p, _p, _p, _p, _p,
                                _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
     "dllm_get_status": (_st, [_p]),

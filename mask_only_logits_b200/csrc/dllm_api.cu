@@ -110,15 +110,14 @@ dllm_status device_state(DeviceState** out) {
       void* p = nullptr;
       if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) st.err = DLLM_ERR_CUDA;
       st.status = static_cast<int*>(p);
+      const auto smem_attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
       if (st.err == DLLM_OK &&
-          (cudaFuncSetAttribute(lm::lmhead_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                lm::Cfg<1>::SMEM_BYTES) != cudaSuccess ||
-           cudaFuncSetAttribute(lm::lmhead_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                lm::Cfg<1>::SMEM_BYTES) != cudaSuccess ||
-           cudaFuncSetAttribute(lm::lmhead_kernel<2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                lm::Cfg<2>::SMEM_BYTES) != cudaSuccess ||
-           cudaFuncSetAttribute(lm::lmhead_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                lm::Cfg<2>::SMEM_BYTES) != cudaSuccess))
+          (cudaFuncSetAttribute(lm::lmhead_kernel<1, lm::kModeStats>, smem_attr, lm::Cfg<1>::SMEM_BYTES) ||
+           cudaFuncSetAttribute(lm::lmhead_kernel<1, lm::kModeStatsExt>, smem_attr, lm::Cfg<1>::SMEM_BYTES) ||
+           cudaFuncSetAttribute(lm::lmhead_kernel<1, lm::kModeDebugStore>, smem_attr, lm::Cfg<1>::SMEM_BYTES) ||
+           cudaFuncSetAttribute(lm::lmhead_kernel<2, lm::kModeStats>, smem_attr, lm::Cfg<2>::SMEM_BYTES) ||
+           cudaFuncSetAttribute(lm::lmhead_kernel<2, lm::kModeStatsExt>, smem_attr, lm::Cfg<2>::SMEM_BYTES) ||
+           cudaFuncSetAttribute(lm::lmhead_kernel<2, lm::kModeDebugStore>, smem_attr, lm::Cfg<2>::SMEM_BYTES)))
         st.err = DLLM_ERR_CUDA;
       if (st.err == DLLM_OK) {
         // how many CTA pairs of the paired GEMM can be resident at once (a persistent grid
@@ -135,7 +134,7 @@ dllm_status device_state(DeviceState** out) {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int clusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&clusters, lm::lmhead_kernel<2, false>, &cfg) != cudaSuccess)
+        if (cudaOccupancyMaxActiveClusters(&clusters, lm::lmhead_kernel<2, lm::kModeStats>, &cfg) != cudaSuccess)
           clusters = 0;
         st.pairs = clusters < lm::kMaxCtas / 2 ? clusters : lm::kMaxCtas / 2;
       }
@@ -156,9 +155,10 @@ dllm_status device_state(DeviceState** out) {
   return DLLM_OK;
 }
 
-// Workspace layout: [tile counts | unit counters | gathered rows Hm | part_m | part_s | part_a].
+// Workspace layout:
+// [tile counts | unit counters | gathered rows Hm | part_m | part_s | part_a | part_t | part_m2].
 struct WsLayout {
-  size_t tiles_off, ctr_off, hm_off, pm_off, ps_off, pa_off, total;
+  size_t tiles_off, ctr_off, hm_off, pm_off, ps_off, pa_off, pt_off, pm2_off, total;
   long long part_cap;
   int n_ctr;
 };
@@ -195,6 +195,8 @@ WsLayout ws_layout(int B, int L, int d, int V) {
   w.pm_off = off;    off = round_up(off + sizeof(float) * cap, 256);
   w.ps_off = off;    off = round_up(off + sizeof(float) * cap, 256);
   w.pa_off = off;    off = round_up(off + sizeof(int) * cap, 256);
+  w.pt_off = off;    off = round_up(off + sizeof(float) * cap, 256);
+  w.pm2_off = off;   off = round_up(off + sizeof(float) * cap, 256);
   w.total = off;
   return w;
 }
@@ -235,6 +237,7 @@ dllm_status make_tmap(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t
 struct LogitsArgs {
   const uint16_t* H; const uint8_t* M; const uint16_t* W;
   int B, L, d, V;
+  uint32_t stats; float* entropy; float* margin;
   int* tok; float* conf; float* lse; float* dbg;
   int* row_idx; int* seq_off; int* count;
   void* ws; size_t ws_bytes; cudaStream_t s;
@@ -244,9 +247,13 @@ dllm_status validate_logits(const LogitsArgs& a, bool debug) {
   if (!a.H || !a.M || !a.W || !a.row_idx || !a.seq_off || !a.count || !a.ws) return DLLM_ERR_NULL;
   if (!debug && (!a.tok || !a.conf || !a.lse)) return DLLM_ERR_NULL;
   if (debug && !a.dbg) return DLLM_ERR_NULL;
+  if ((a.stats & ~(DLLM_STAT_ENTROPY | DLLM_STAT_MARGIN)) != 0) return DLLM_ERR_SHAPE;
+  if (((a.stats & DLLM_STAT_ENTROPY) != 0) != (a.entropy != nullptr)) return DLLM_ERR_NULL;
+  if (((a.stats & DLLM_STAT_MARGIN) != 0) != (a.margin != nullptr)) return DLLM_ERR_NULL;
   if (!shapes_ok(a.B, a.L) || a.V < 1 || a.d < DLLM_D_MULTIPLE || a.d % DLLM_D_MULTIPLE != 0)
     return DLLM_ERR_SHAPE;
-  const void* ptrs[] = {a.H, a.M, a.W, a.row_idx, a.seq_off, a.count, a.ws, a.tok, a.conf, a.lse, a.dbg};
+  const void* ptrs[] = {a.H, a.M, a.W, a.row_idx, a.seq_off, a.count, a.ws, a.tok, a.conf, a.lse,
+                        a.dbg, a.entropy, a.margin};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return DLLM_ERR_ALIGN;
   if (a.ws_bytes < ws_layout(a.B, a.L, a.d, a.V).total) return DLLM_ERR_WORKSPACE;
@@ -265,7 +272,11 @@ dllm_status run_logits(const LogitsArgs& a, bool debug) {
   float* pm = reinterpret_cast<float*>(ws + w.pm_off);
   float* ps = reinterpret_cast<float*>(ws + w.ps_off);
   int* pa = reinterpret_cast<int*>(ws + w.pa_off);
+  float* pt = reinterpret_cast<float*>(ws + w.pt_off);
+  float* pm2 = reinterpret_cast<float*>(ws + w.pm2_off);
   int* ctr = reinterpret_cast<int*>(ws + w.ctr_off);
+  const lm::Partials part{pm, ps, pa, pt, pm2};
+  const lm::Outputs outs{a.tok, a.conf, a.lse, a.entropy, a.margin};
   const long long n = static_cast<long long>(a.B) * a.L;
 
   // GEMM variant and its work holders (CTAs, or CTA pairs)
@@ -338,21 +349,21 @@ dllm_status run_logits(const LogitsArgs& a, bool debug) {
     }
     const int n_cap = static_cast<int>(n);
     float* dbg = debug ? a.dbg : nullptr;
+    const int mode = debug ? lm::kModeDebugStore : (a.stats ? lm::kModeStatsExt : lm::kModeStats);
+    const int* cnt = a.count;
     cudaError_t e;
+#define DLLM_LAUNCH_GEMM(CGV, MODE)                                                            \
+  cudaLaunchKernelEx(&cfg, lm::lmhead_kernel<CGV, MODE>, tmA, tmB, cnt, n_cap, a.V, a.d, gmax, \
+                     part, w.part_cap, ctr, outs, dbg, ds->status)
     if (cg == 2)
-      e = debug ? cudaLaunchKernelEx(&cfg, lm::lmhead_kernel<2, true>, tmA, tmB, (const int*)a.count, n_cap,
-                                     a.V, a.d, gmax, pm, ps, pa, w.part_cap, ctr, a.tok, a.conf, a.lse,
-                                     dbg, ds->status)
-                : cudaLaunchKernelEx(&cfg, lm::lmhead_kernel<2, false>, tmA, tmB, (const int*)a.count, n_cap,
-                                     a.V, a.d, gmax, pm, ps, pa, w.part_cap, ctr, a.tok, a.conf, a.lse,
-                                     dbg, ds->status);
+      e = mode == lm::kModeStats ? DLLM_LAUNCH_GEMM(2, lm::kModeStats)
+        : mode == lm::kModeStatsExt ? DLLM_LAUNCH_GEMM(2, lm::kModeStatsExt)
+        : DLLM_LAUNCH_GEMM(2, lm::kModeDebugStore);
     else
-      e = debug ? cudaLaunchKernelEx(&cfg, lm::lmhead_kernel<1, true>, tmA, tmB, (const int*)a.count, n_cap,
-                                     a.V, a.d, gmax, pm, ps, pa, w.part_cap, ctr, a.tok, a.conf, a.lse,
-                                     dbg, ds->status)
-                : cudaLaunchKernelEx(&cfg, lm::lmhead_kernel<1, false>, tmA, tmB, (const int*)a.count, n_cap,
-                                     a.V, a.d, gmax, pm, ps, pa, w.part_cap, ctr, a.tok, a.conf, a.lse,
-                                     dbg, ds->status);
+      e = mode == lm::kModeStats ? DLLM_LAUNCH_GEMM(1, lm::kModeStats)
+        : mode == lm::kModeStatsExt ? DLLM_LAUNCH_GEMM(1, lm::kModeStatsExt)
+        : DLLM_LAUNCH_GEMM(1, lm::kModeDebugStore);
+#undef DLLM_LAUNCH_GEMM
     if (e != cudaSuccess) return DLLM_ERR_CUDA;
   }
   count_launch();
@@ -470,8 +481,18 @@ dllm_status dllm_masked_logits(const uint16_t* H, const uint8_t* M, const uint16
                                int32_t L, int32_t d, int32_t V, int32_t* tok, float* conf,
                                float* lse, int32_t* row_idx, int32_t* seq_off, int32_t* count,
                                void* ws, size_t ws_bytes, void* stream) {
-  LogitsArgs a{H, M, W, B, L, d, V, tok, conf, lse, nullptr, row_idx, seq_off, count,
-               ws, ws_bytes, static_cast<cudaStream_t>(stream)};
+  LogitsArgs a{H, M, W, B, L, d, V, 0u, nullptr, nullptr, tok, conf, lse, nullptr, row_idx, seq_off,
+               count, ws, ws_bytes, static_cast<cudaStream_t>(stream)};
+  return run_logits(a, false);
+}
+
+dllm_status dllm_masked_logits_ex(const uint16_t* H, const uint8_t* M, const uint16_t* W, int32_t B,
+                                  int32_t L, int32_t d, int32_t V, uint32_t stats, int32_t* tok,
+                                  float* conf, float* lse, float* entropy, float* margin,
+                                  int32_t* row_idx, int32_t* seq_off, int32_t* count, void* ws,
+                                  size_t ws_bytes, void* stream) {
+  LogitsArgs a{H, M, W, B, L, d, V, stats, entropy, margin, tok, conf, lse, nullptr, row_idx,
+               seq_off, count, ws, ws_bytes, static_cast<cudaStream_t>(stream)};
   return run_logits(a, false);
 }
 
@@ -479,16 +500,21 @@ dllm_status dllm_debug_lmhead_logits(const uint16_t* H, const uint8_t* M, const 
                                      int32_t B, int32_t L, int32_t d, int32_t V, float* logits_out,
                                      int32_t* row_idx, int32_t* seq_off, int32_t* count, void* ws,
                                      size_t ws_bytes, void* stream) {
-  LogitsArgs a{H, M, W, B, L, d, V, nullptr, nullptr, nullptr, logits_out, row_idx, seq_off, count,
-               ws, ws_bytes, static_cast<cudaStream_t>(stream)};
+  LogitsArgs a{H, M, W, B, L, d, V, 0u, nullptr, nullptr, nullptr, nullptr, nullptr, logits_out,
+               row_idx, seq_off, count, ws, ws_bytes, static_cast<cudaStream_t>(stream)};
   return run_logits(a, true);
 }
 
-dllm_status dllm_select_unmask(const float* conf, const int32_t* row_idx, const int32_t* seq_off,
-                               int32_t B, int32_t L, int32_t k, const int32_t* win_lo,
-                               const int32_t* win_hi, const int32_t* tok, int32_t* idx,
-                               int32_t* n_sel, int32_t* tok_sel, float* conf_sel, void* stream) {
+}  // extern "C"
+
+namespace {
+dllm_status run_select(const float* conf, const int32_t* row_idx, const int32_t* seq_off,
+                       int32_t B, int32_t L, int32_t k, bool use_threshold, float threshold,
+                       int32_t min_sel, bool ascending, const int32_t* win_lo, const int32_t* win_hi,
+                       const int32_t* tok, int32_t* idx, int32_t* n_sel, int32_t* tok_sel,
+                       float* conf_sel, void* stream) {
   if (!conf || !row_idx || !seq_off || !idx || !n_sel) return DLLM_ERR_NULL;
+  if (use_threshold && (min_sel < 0 || threshold != threshold)) return DLLM_ERR_SHAPE;
   if ((win_lo == nullptr) != (win_hi == nullptr)) return DLLM_ERR_NULL;
   if (tok_sel && !tok) return DLLM_ERR_NULL;
   if (!shapes_ok(B, L) || k < 1 || k > DLLM_MAX_K) return DLLM_ERR_SHAPE;
@@ -499,11 +525,32 @@ dllm_status dllm_select_unmask(const float* conf, const int32_t* row_idx, const 
   dllm_status st = device_state(&ds);
   if (st != DLLM_OK) return st;
   if (launch_pdl(select_unmask_kernel, dim3(B), dim3(kSelThreads), 0, static_cast<cudaStream_t>(stream),
-                 conf, row_idx, seq_off, B * L, L, k, win_lo, win_hi, tok, idx, n_sel, tok_sel,
-                 conf_sel) != cudaSuccess)
+                 conf, row_idx, seq_off, B * L, L, k, use_threshold, threshold, min_sel, ascending,
+                 win_lo, win_hi, tok, idx, n_sel, tok_sel, conf_sel) != cudaSuccess)
     return DLLM_ERR_CUDA;
   count_launch();
   return DLLM_OK;
+}
+}  // namespace
+
+extern "C" {
+
+dllm_status dllm_select_unmask(const float* conf, const int32_t* row_idx, const int32_t* seq_off,
+                               int32_t B, int32_t L, int32_t k, const int32_t* win_lo,
+                               const int32_t* win_hi, const int32_t* tok, int32_t* idx,
+                               int32_t* n_sel, int32_t* tok_sel, float* conf_sel, void* stream) {
+  return run_select(conf, row_idx, seq_off, B, L, k, false, 0.f, 0, false, win_lo, win_hi, tok, idx,
+                    n_sel, tok_sel, conf_sel, stream);
+}
+
+dllm_status dllm_select_unmask_ex(const float* score, const int32_t* row_idx, const int32_t* seq_off,
+                                  int32_t B, int32_t L, int32_t k, float threshold, int32_t min_sel,
+                                  int32_t ascending, const int32_t* win_lo, const int32_t* win_hi,
+                                  const int32_t* tok, int32_t* idx, int32_t* n_sel, int32_t* tok_sel,
+                                  float* score_sel, void* stream) {
+  if (ascending != 0 && ascending != 1) return DLLM_ERR_SHAPE;
+  return run_select(score, row_idx, seq_off, B, L, k, true, threshold, min_sel, ascending != 0,
+                    win_lo, win_hi, tok, idx, n_sel, tok_sel, score_sel, stream);
 }
 
 dllm_status dllm_decode_step(const uint16_t* H, const uint8_t* M, const uint16_t* W, int32_t B,

@@ -259,9 +259,31 @@ struct Smem {
   }
 };
 
-// Online (max, sum of exp(z - max), first argmax) over 32 consecutive logits.
-__device__ __forceinline__ void fold_chunk(float (&v)[32], int col0, int V, float& run_m,
-                                           float& run_s, int& run_a) {
+// Epilogue modes: statistics for tok / lse / conf; the same plus the entropy and the
+// top-2 probability margin of each row's softmax; or raw logits stored (test hook).
+constexpr int kModeStats = 0;
+constexpr int kModeStatsExt = 1;
+constexpr int kModeDebugStore = 2;
+
+// Running softmax statistics of one row over the vocabulary seen so far:
+//   m  = max logit, a = its first index, s = sum exp(z - m),
+//   t  = sum exp(z - m) (z - m)  (extended mode; entropy = ln s - t / s),
+//   m2 = second-largest logit    (extended mode; margin p1 - p2 = (1 - exp(m2 - m)) / s).
+struct RowState {
+  float m, s, t, m2;
+  int a;
+  __device__ __forceinline__ void reset() {
+    m = -INFINITY;
+    s = 0.f;
+    t = 0.f;
+    m2 = -INFINITY;
+    a = 0;
+  }
+};
+
+// Fold 32 consecutive logits (vocabulary columns col0..col0+31) into a row's state.
+template <bool kExt>
+__device__ __forceinline__ void fold_chunk(float (&v)[32], int col0, int V, RowState& st) {
   if (col0 + 32 > V) {
 #pragma unroll
     for (int j = 0; j < 32; ++j)
@@ -271,83 +293,147 @@ __device__ __forceinline__ void fold_chunk(float (&v)[32], int col0, int V, floa
 #pragma unroll
   for (int j = 1; j < 32; ++j) mx = fmaxf(mx, v[j]);
   if (mx == -INFINITY) return;                 // the whole chunk is past the vocabulary
-  if (mx > run_m) {                            // strict: earlier (lower) index wins ties
+  float c2 = -INFINITY;                        // chunk's second largest (= mx on a tie)
+  if constexpr (kExt) {
+    int n_at_max = 0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      n_at_max += v[j] == mx ? 1 : 0;
+      c2 = v[j] == mx ? c2 : fmaxf(c2, v[j]);
+    }
+    if (n_at_max > 1) c2 = mx;
+  }
+  if (mx > st.m) {                             // strict: earlier (lower) index wins ties
     int j0 = 31;
 #pragma unroll
     for (int j = 31; j >= 0; --j)
       if (v[j] == mx) j0 = j;
-    run_s *= ex2_approx((run_m - mx) * kLog2e);
-    run_m = mx;
-    run_a = col0 + j0;
+    const float sc = ex2_approx((st.m - mx) * kLog2e);
+    if constexpr (kExt) {
+      // re-centre t on the new max: (z - mx) = (z - m) + (m - mx)
+      if (st.s > 0.f) st.t = sc * (st.t + (st.m - mx) * st.s);
+      st.m2 = fmaxf(st.m, c2);
+    }
+    st.s *= sc;
+    st.m = mx;
+    st.a = col0 + j0;
+  } else if constexpr (kExt) {
+    st.m2 = fmaxf(st.m2, mx);
   }
-  const float mb = run_m * kLog2e;
+  const float mb = st.m * kLog2e;
   float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+  if constexpr (kExt) {
+    float t0 = 0.f, t1 = 0.f;
 #pragma unroll
-  for (int j = 0; j < 32; j += 4) {
-    s0 += ex2_approx(fmaf(v[j + 0], kLog2e, -mb));
-    s1 += ex2_approx(fmaf(v[j + 1], kLog2e, -mb));
-    s2 += ex2_approx(fmaf(v[j + 2], kLog2e, -mb));
-    s3 += ex2_approx(fmaf(v[j + 3], kLog2e, -mb));
+    for (int j = 0; j < 32; j += 2) {
+      const float e0 = ex2_approx(fmaf(v[j + 0], kLog2e, -mb));
+      const float e1 = ex2_approx(fmaf(v[j + 1], kLog2e, -mb));
+      s0 += e0;
+      s1 += e1;
+      // past-the-vocabulary columns are -inf: e = 0, and 0 * (-inf) must not poison t
+      t0 += e0 > 0.f ? e0 * (v[j + 0] - st.m) : 0.f;
+      t1 += e1 > 0.f ? e1 * (v[j + 1] - st.m) : 0.f;
+    }
+    st.t += t0 + t1;
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+      s0 += ex2_approx(fmaf(v[j + 0], kLog2e, -mb));
+      s1 += ex2_approx(fmaf(v[j + 1], kLog2e, -mb));
+      s2 += ex2_approx(fmaf(v[j + 2], kLog2e, -mb));
+      s3 += ex2_approx(fmaf(v[j + 3], kLog2e, -mb));
+    }
   }
-  run_s += (s0 + s1) + (s2 + s3);
+  st.s += (s0 + s1) + (s2 + s3);
 }
 
-// lse_merge of one row, as an accumulation: fold the partials (m_j, s_j, a_j) found at
-// base + j * stride for j = j0..j1-1 (ascending vocabulary ranges) into (m, s, a):
-//   m* = max_j m_j, s* = sum_j s_j exp(m_j - m*), a = a_j of the first j with m_j = m*.
-// Then lse = m* + ln s* and conf = exp(m* - lse) = 1 / s* (merge_finish).  Partials are read
+// Final values of a row state: tok, lse, conf (and entropy, margin).
+__device__ __forceinline__ void state_finish(const RowState& st, int& tok, float& conf, float& lse,
+                                             float& ent, float& margin) {
+  tok = st.a;
+  lse = st.m + logf(st.s);
+  conf = 1.0f / st.s;
+  ent = logf(st.s) - st.t / st.s;
+  margin = (1.0f - ex2_approx((st.m2 - st.m) * kLog2e)) / st.s;
+}
+
+// Partials of one row per vocabulary split (structure of arrays).
+struct Partials {
+  float* m;
+  float* s;
+  int* a;
+  float* t;    // extended mode only
+  float* m2;   // extended mode only
+};
+
+// lse_merge of one row, as an accumulation: fold the partials found at base + j * stride for
+// j = j0..j1-1 (ascending vocabulary ranges) into st:
+//   m* = max_j m_j, s* = sum_j s_j exp(m_j - m*), a = a_j of the first j with m_j = m*,
+//   t* = sum_j exp(m_j - m*) (t_j + (m_j - m*) s_j), m2* = the second largest of all m_j, m2_j.
+// Then lse = m* + ln s* and conf = exp(m* - lse) = 1 / s* (state_finish).  Partials are read
 // through L2 (other CTAs of the running kernel may have written them) in batches of 8 whose
 // loads are all issued before any is used.
-__device__ __forceinline__ void merge_acc(const float* __restrict__ pm, const float* __restrict__ ps,
-                                          const int* __restrict__ pa, long long base,
-                                          long long stride, int j0, int j1, float& m, float& s,
-                                          int& a) {
+template <bool kExt>
+__device__ __forceinline__ void merge_acc(const Partials& P, long long base, long long stride,
+                                          int j0, int j1, RowState& st) {
   constexpr int kBatch = 8;
   for (int jb = j0; jb < j1; jb += kBatch) {
-    float mb[kBatch], sb[kBatch];
+    float mb[kBatch], sb[kBatch], tb[kBatch], m2b[kBatch];
     int ab[kBatch];
 #pragma unroll
-    for (int t = 0; t < kBatch; ++t) {
-      if (jb + t < j1) {
-        const long long e = base + (jb + t) * stride;
-        mb[t] = __ldcg(pm + e);
-        sb[t] = __ldcg(ps + e);
-        ab[t] = __ldcg(pa + e);
+    for (int q = 0; q < kBatch; ++q) {
+      if (jb + q < j1) {
+        const long long e = base + (jb + q) * stride;
+        mb[q] = __ldcg(P.m + e);
+        sb[q] = __ldcg(P.s + e);
+        ab[q] = __ldcg(P.a + e);
+        if constexpr (kExt) {
+          tb[q] = __ldcg(P.t + e);
+          m2b[q] = __ldcg(P.m2 + e);
+        }
       } else {
-        mb[t] = -INFINITY;
-        sb[t] = 0.f;
-        ab[t] = 0;
+        mb[q] = -INFINITY;
+        sb[q] = 0.f;
+        ab[q] = 0;
+        tb[q] = 0.f;
+        m2b[q] = -INFINITY;
       }
     }
 #pragma unroll
-    for (int t = 0; t < kBatch; ++t) {
-      if (mb[t] == -INFINITY) continue;   // empty partial (or past j1): nothing to add
-      if (mb[t] > m) {                    // strict: the earlier split keeps a tie
-        s = s * ex2_approx((m - mb[t]) * kLog2e) + sb[t];
-        m = mb[t];
-        a = ab[t];
+    for (int q = 0; q < kBatch; ++q) {
+      if (mb[q] == -INFINITY) continue;   // empty partial (or past j1): nothing to add
+      if (mb[q] > st.m) {                 // strict: the earlier split keeps a tie
+        const float sc = ex2_approx((st.m - mb[q]) * kLog2e);
+        if constexpr (kExt) {
+          st.t = (st.s > 0.f ? sc * (st.t + (st.m - mb[q]) * st.s) : 0.f) + tb[q];
+          st.m2 = fmaxf(st.m, m2b[q]);
+        }
+        st.s = st.s * sc + sb[q];
+        st.m = mb[q];
+        st.a = ab[q];
       } else {
-        s += sb[t] * ex2_approx((mb[t] - m) * kLog2e);
+        const float sc = ex2_approx((mb[q] - st.m) * kLog2e);
+        if constexpr (kExt) {
+          st.t += sc * (tb[q] + (mb[q] - st.m) * sb[q]);
+          st.m2 = fmaxf(st.m2, mb[q]);
+        }
+        st.s += sb[q] * sc;
       }
     }
   }
 }
 
-__device__ __forceinline__ void merge_finish(float m, float s, int a, int& tok, float& conf,
-                                             float& lse) {
-  tok = a;
-  lse = m + logf(s);
-  conf = 1.0f / s;
-}
-
+// Merge n_split partials at base + j * stride (plain layout; test hook).
 __device__ __forceinline__ void merge_row(const float* __restrict__ pm, const float* __restrict__ ps,
                                           const int* __restrict__ pa, long long base,
                                           long long stride, int n_split, int& tok, float& conf,
                                           float& lse) {
-  float m = -INFINITY, s = 0.f;
-  int a = 0;
-  merge_acc(pm, ps, pa, base, stride, 0, n_split, m, s, a);
-  merge_finish(m, s, a, tok, conf, lse);
+  RowState st;
+  st.reset();
+  Partials P{const_cast<float*>(pm), const_cast<float*>(ps), const_cast<int*>(pa), nullptr, nullptr};
+  merge_acc<false>(P, base, stride, 0, n_split, st);
+  float ent, margin;
+  state_finish(st, tok, conf, lse, ent, margin);
 }
 
 template <int CG>
@@ -364,15 +450,24 @@ __device__ __forceinline__ void mma_commit_all(uint32_t bar) {
   else umma_commit_pair_both(bar);
 }
 
-template <int CG, bool kDebugStore>
+// Results of the kernel (compacted row order).
+struct Outputs {
+  int* tok;
+  float* conf;
+  float* lse;
+  float* entropy;   // extended mode: written when not null
+  float* margin;    // extended mode: written when not null
+};
+
+template <int CG, int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
 lmhead_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const int* __restrict__ count_ptr, int n_cap, int V, int d, int gmax,
-              float* __restrict__ part_m, float* __restrict__ part_s, int* __restrict__ part_a,
-              long long part_cap, int* __restrict__ unit_ctr, int* __restrict__ out_tok,
-              float* __restrict__ out_conf, float* __restrict__ out_lse,
-              float* __restrict__ dbg_logits, int* __restrict__ status) {
+              const Partials part, long long part_cap, int* __restrict__ unit_ctr,
+              const Outputs out, float* __restrict__ dbg_logits, int* __restrict__ status) {
   using C = Cfg<CG>;
+  constexpr bool kDebugStore = kMode == kModeDebugStore;
+  constexpr bool kExt = kMode == kModeStatsExt;
   extern __shared__ uint8_t smem_raw[];
   Smem<CG> sm(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -501,8 +596,8 @@ lmhead_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
       epi_phase ^= 1u;
       return __all_sync(0xffffffffu, got);
     };
-    // fold the next accumulator (vocabulary tile n of m-tile m_tile) into (rm, rs, ra)
-    auto consume = [&](int m_tile, int n, float& rm, float& rs, int& ra) -> bool {
+    // fold the next accumulator (vocabulary tile n of m-tile m_tile) into st
+    auto consume = [&](int m_tile, int n, RowState& st) -> bool {
       const uint32_t buf = tile & 1u, tph = (tile >> 1) & 1u;
       // every lane waits; the vote reconverges the warp before the .sync.aligned loads and
       // makes the abort decision warp-uniform
@@ -526,7 +621,7 @@ lmhead_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
               if (col0 + j < V) dbg_logits[static_cast<size_t>(row) * V + col0 + j] = v[j];
           }
         } else {
-          fold_chunk(v, col0, V, rm, rs, ra);
+          fold_chunk<kExt>(v, col0, V, st);
         }
       }
       tc_fence_before();
@@ -536,16 +631,27 @@ lmhead_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
       ++tile;
       return true;
     };
-    auto write_result = [&](int row, float m, float s_, int a) {
-      out_tok[row] = a;
-      out_lse[row] = m + logf(s_);
-      out_conf[row] = 1.0f / s_;
+    auto write_result = [&](int row, const RowState& st) {
+      int t;
+      float c, l, e, mg;
+      state_finish(st, t, c, l, e, mg);
+      out.tok[row] = t;
+      out.conf[row] = c;
+      out.lse[row] = l;
+      if constexpr (kExt) {
+        if (out.entropy) out.entropy[row] = e;
+        if (out.margin) out.margin[row] = mg;
+      }
     };
-    auto write_partial = [&](long long e, float m, float s_, int a) {
+    auto write_partial = [&](long long e, const RowState& st) {
       if (e < part_cap) {
-        part_m[e] = m;
-        part_s[e] = s_;
-        part_a[e] = a;
+        part.m[e] = st.m;
+        part.s[e] = st.s;
+        part.a[e] = st.a;
+        if constexpr (kExt) {
+          part.t[e] = st.t;
+          part.m2[e] = st.m2;
+        }
       } else {
         atomicOr(status, kStatusBounds);             // cannot happen: workspace sized for it
       }
@@ -553,7 +659,7 @@ lmhead_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
 
     // A finished (m-tile, slot) state: the result itself when the m-tile has a single unit,
     // else a partial; the last of the m-tile's units to finish merges its rows.
-    auto finish = [&](int g, const Unit& u, int m_local, int slot, float rm, float rs, int ra) -> bool {
+    auto finish = [&](int g, const Unit& u, int m_local, int slot, const RowState& st) -> bool {
       const int m_tile = g * pl.gmax + m_local;
       const int row = m_tile * C::BM + row_in_tile;
       const bool valid = row < pl.count;
@@ -561,10 +667,10 @@ lmhead_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
       if (pl.rem) pl.leftovers_of(m_local, u.G, j_lo, j_hi);
       const int units = u.P + (j_hi >= j_lo ? j_hi - j_lo + 1 : 0);
       if (units == 1) {
-        if (valid) write_result(row, rm, rs, ra);
+        if (valid) write_result(row, st);
         return true;
       }
-      if (valid) write_partial(pl.part_index(g, u.G, slot, m_local * C::BM + row_in_tile), rm, rs, ra);
+      if (valid) write_partial(pl.part_index(g, u.G, slot, m_local * C::BM + row_in_tile), st);
       // Writers fence before the counter increment; the last arriver fences after it and
       // reads the partials through L2.
       __threadfence();
@@ -579,16 +685,11 @@ lmhead_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         if (valid) {
           const long long base = pl.part_index(g, u.G, 0, m_local * C::BM + row_in_tile);
           const long long stride = static_cast<long long>(u.G) * C::BM;
-          float m = -INFINITY, s_ = 0.f;
-          int a = 0;
-          merge_acc(part_m, part_s, part_a, base, stride, 0, u.P, m, s_, a);
-          if (j_hi >= j_lo) merge_acc(part_m, part_s, part_a, base, stride, u.P + j_lo, u.P + j_hi + 1, m, s_, a);
-          int t;
-          float c, l;
-          merge_finish(m, s_, a, t, c, l);
-          out_tok[row] = t;
-          out_conf[row] = c;
-          out_lse[row] = l;
+          RowState mst;
+          mst.reset();
+          merge_acc<kExt>(part, base, stride, 0, u.P, mst);
+          if (j_hi >= j_lo) merge_acc<kExt>(part, base, stride, u.P + j_lo, u.P + j_hi + 1, mst);
+          write_result(row, mst);
         }
       }
       return true;
@@ -600,27 +701,25 @@ lmhead_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
       if (u.leftover) {
         // remainder tiles in m-major order: one running state, finished at each m-tile change
         int cur = -1;
-        float rm = -INFINITY, rs = 0.f;
-        int ra = 0;
+        RowState st;
+        st.reset();
         for (long long i = u.i0; i < u.i1 && ok; ++i) {
           const int m_local = static_cast<int>(i / pl.rr);
           const int n = u.P * pl.rb + static_cast<int>(i % pl.rr);
           if (m_local != cur) {
-            if (cur >= 0 && !kDebugStore) ok = finish(g, u, cur, u.p, rm, rs, ra);
+            if (cur >= 0 && !kDebugStore) ok = finish(g, u, cur, u.p, st);
             cur = m_local;
-            rm = -INFINITY;
-            rs = 0.f;
-            ra = 0;
+            st.reset();
           }
-          if (ok && !consume(g * pl.gmax + m_local, n, rm, rs, ra)) ok = false;
+          if (ok && !consume(g * pl.gmax + m_local, n, st)) ok = false;
         }
-        if (ok && cur >= 0 && !kDebugStore) ok = finish(g, u, cur, u.p, rm, rs, ra);
+        if (ok && cur >= 0 && !kDebugStore) ok = finish(g, u, cur, u.p, st);
       } else {
-        float rm = -INFINITY, rs = 0.f;
-        int ra = 0;
+        RowState st;
+        st.reset();
         for (int n = u.n0; n < u.n1 && ok; ++n)
-          if (!consume(u.m_tile, n, rm, rs, ra)) ok = false;
-        if (ok && !kDebugStore) ok = finish(g, u, u.m_local, u.p, rm, rs, ra);
+          if (!consume(u.m_tile, n, st)) ok = false;
+        if (ok && !kDebugStore) ok = finish(g, u, u.m_local, u.p, st);
       }
     }
   }

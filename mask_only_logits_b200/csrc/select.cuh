@@ -3,19 +3,27 @@
 // window [lo, hi) of positions (the current semi-autoregressive block: Sparse-dLLM page,
 // "Experiment", block-wise decoding needs the current block only).
 //
+// Threshold-based parallel unmasking uses the same kernel (decoding thresholds, Dynamic-dLLM
+// abstract on the dLLM pages): with a threshold, the number taken from a sequence is
+// min(k, max(min(min_sel, n), #candidates with score >= threshold)); without one, min(k, n).
+// In ascending order (e.g. entropy: lower is better) every comparison is reversed.
+//
 // One CTA of 1024 threads per sequence.  Key of a candidate in compacted row r:
-//     (float bits of conf[r]) << 32 | ~r
-// Confidences are positive, so their IEEE bits order like the values; within a sequence r
-// ascends with the position, so ~r puts the lower position first among equal confidences.
+//     (order-preserving bits of score[r]) << 32 | ~r
+// Order-preserving bits: a float's IEEE bits with the sign bit flipped, or all bits flipped
+// for negative values, compare as unsigned integers like the floats (scores may be negative,
+// e.g. minus an entropy).  Within a sequence r ascends with the position, so ~r puts the
+// lower position first among equal scores.
 // Steps:
 //   1. candidate range: rows of the sequence whose position lies in the window (one pass:
-//      the window's rows are contiguous because row_idx ascends)
-//   2. if there are more than k candidates, a 4-pass radix select (8 bits per pass) over
-//      the 32 confidence bits finds T, the k-th largest confidence, and how many of the
-//      candidates equal to T are needed
+//      the window's rows are contiguous because row_idx ascends); with a threshold, the
+//      number of candidates at or above it, hence k_eff, the number to take
+//   2. if there are more than k_eff candidates, a 4-pass radix select (8 bits per pass) over
+//      the 32 key bits finds T, the k_eff-th largest key, and how many of the candidates
+//      equal to T are needed
 //   3. one ordered pass collects every candidate above T and the first needed ones equal
 //      to T (block-wide ballot scan keeps them in row order)
-//   4. bitonic sort of the (at most k) keys, descending; write positions, tokens, confs.
+//   4. bitonic sort of the (at most k_eff) keys, descending; write positions, tokens, scores.
 #pragma once
 #include "ptx.cuh"
 
@@ -24,26 +32,36 @@ namespace dllm {
 constexpr int kSelThreads = 1024;
 constexpr int kSelMaxK = 1024;
 
-__device__ __forceinline__ unsigned long long sel_key(float c, int r) {
-  return (static_cast<unsigned long long>(__float_as_uint(c)) << 32) |
+// Float -> unsigned with the same order (for non-NaN values).
+__device__ __forceinline__ uint32_t ordered_bits(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return u ^ (static_cast<uint32_t>(static_cast<int32_t>(u) >> 31) | 0x80000000u);
+}
+
+__device__ __forceinline__ unsigned long long sel_key(uint32_t okey, int r) {
+  return (static_cast<unsigned long long>(okey) << 32) |
          static_cast<unsigned long long>(~static_cast<uint32_t>(r));
 }
 
 __global__ void __launch_bounds__(kSelThreads)
 select_unmask_kernel(const float* __restrict__ conf, const int* __restrict__ row_idx,
                      const int* __restrict__ seq_off, int n_pos, int L, int k,
+                     bool use_threshold, float threshold, int min_sel, bool ascending,
                      const int* __restrict__ win_lo, const int* __restrict__ win_hi,
                      const int* __restrict__ tok, int* __restrict__ idx, int* __restrict__ n_sel,
                      int* __restrict__ tok_sel, float* __restrict__ conf_sel) {
   __shared__ unsigned long long keys[kSelMaxK];
   __shared__ unsigned int hist[256];
-  __shared__ int sh_lo, sh_hi, sh_n, sh_digit, sh_krem, sh_taken;
+  __shared__ int sh_lo, sh_hi, sh_n, sh_digit, sh_krem, sh_taken, sh_q;
   __shared__ int warp_cnt[32];
 
   pdl_wait();
   pdl_launch_dependents();
   const int b = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // key of a score: larger key = better (ascending order: smaller score = better)
+  const uint32_t flip = ascending ? 0xFFFFFFFFu : 0u;
+  auto okey = [&](float f) -> uint32_t { return ordered_bits(f) ^ flip; };
   // compacted rows of sequence b (clamped: seq_off comes from the device)
   const int r0 = max(0, min(seq_off[b], n_pos));
   const int r1 = max(r0, min(seq_off[b + 1], n_pos));
@@ -70,18 +88,32 @@ select_unmask_kernel(const float* __restrict__ conf, const int* __restrict__ row
     c1 = sh_hi > sh_lo ? sh_hi : sh_lo;
   }
   const int n = c1 - c0;
-  const int nsel = n < k ? n : k;
+  int k_eff = n < k ? n : k;
+  if (use_threshold) {
+    if (tid == 0) sh_q = 0;
+    __syncthreads();
+    const uint32_t tq = okey(threshold);
+    int mine = 0;
+    for (int r = c0 + tid; r < c1; r += kSelThreads) mine += okey(conf[r]) >= tq ? 1 : 0;
+    for (int o = 16; o > 0; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
+    if (lane == 0 && mine) atomicAdd(&sh_q, mine);
+    __syncthreads();
+    const int floor_n = min_sel < n ? min_sel : n;
+    const int want = sh_q > floor_n ? sh_q : floor_n;
+    k_eff = want < k ? want : k;
+  }
+  const int nsel = k_eff;
 
   if (tid == 0) sh_n = 0;
   __syncthreads();
 
-  if (n <= k) {
+  if (n <= k_eff) {
     // 2'. every candidate is selected
-    for (int r = c0 + tid; r < c1; r += kSelThreads) keys[r - c0] = sel_key(conf[r], r);
-  } else {
-    // 2. radix select of the k-th largest confidence bits
+    for (int r = c0 + tid; r < c1; r += kSelThreads) keys[r - c0] = sel_key(okey(conf[r]), r);
+  } else if (k_eff > 0) {
+    // 2. radix select of the k_eff-th largest key
     uint32_t prefix = 0, pmask = 0;
-    int krem = k;
+    int krem = k_eff;
     for (int shift = 24; shift >= 0; shift -= 8) {
       for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
       __syncthreads();
@@ -91,7 +123,7 @@ select_unmask_kernel(const float* __restrict__ conf, const int* __restrict__ row
         const int r = base + tid;
         uint32_t bin = 0xFFFFFFFFu;
         if (r < c1) {
-          const uint32_t u = __float_as_uint(conf[r]);
+          const uint32_t u = okey(conf[r]);
           if ((u & pmask) == prefix) bin = (u >> shift) & 255u;
         }
         const unsigned peers = __match_any_sync(0xffffffffu, bin);
@@ -131,17 +163,17 @@ select_unmask_kernel(const float* __restrict__ conf, const int* __restrict__ row
     for (int base = c0; base < c1; base += kSelThreads) {
       const int r = base + tid;
       uint32_t u = 0;
-      if (r < c1) u = __float_as_uint(conf[r]);
+      if (r < c1) u = okey(conf[r]);
       const bool gt = r < c1 && u > T;
       const bool eq = r < c1 && u == T;
-      if (gt) keys[atomicAdd(&sh_n, 1)] = sel_key(__uint_as_float(u), r);
+      if (gt) keys[atomicAdd(&sh_n, 1)] = sel_key(u, r);
       const unsigned bal = __ballot_sync(0xffffffffu, eq);
       if (lane == 0) warp_cnt[warp] = __popc(bal);
       __syncthreads();
       int before = sh_taken;
       for (int w = 0; w < warp; ++w) before += warp_cnt[w];
       before += __popc(bal & ((1u << lane) - 1u));
-      if (eq && before < krem) keys[atomicAdd(&sh_n, 1)] = sel_key(__uint_as_float(u), r);
+      if (eq && before < krem) keys[atomicAdd(&sh_n, 1)] = sel_key(u, r);
       __syncthreads();
       if (tid == 0) {
         int tot = 0;
@@ -180,7 +212,7 @@ select_unmask_kernel(const float* __restrict__ conf, const int* __restrict__ row
       const int r = static_cast<int>(~static_cast<uint32_t>(key & 0xffffffffull));
       idx[o] = static_cast<int>(row_idx[r] - seq_base);
       if (tok_sel) tok_sel[o] = tok[r];
-      if (conf_sel) conf_sel[o] = __uint_as_float(static_cast<uint32_t>(key >> 32));
+      if (conf_sel) conf_sel[o] = conf[r];
     } else {
       idx[o] = -1;
       if (tok_sel) tok_sel[o] = -1;

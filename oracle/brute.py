@@ -47,6 +47,27 @@ def stats(z):
     return tok, m, lse, conf
 
 
+def policy_stats(z):
+    """(entropy, margin) of softmax(z) by definition: -sum p ln p and p_(1) - p_(2)."""
+    m = max(z)
+    e = [math.exp(x - m) for x in z]
+    s = math.fsum(e)
+    p = [x / s for x in e]
+    ent = -math.fsum(q * math.log(q) for q in p if q > 0)
+    ps = sorted(p, reverse=True)
+    margin = ps[0] - ps[1] if len(ps) > 1 else ps[0]
+    return ent, margin
+
+
+def select_threshold(cands, k, threshold, min_sel=1):
+    """cands: list of (score, pos); all with score >= threshold (at most k, at least
+    min(min_sel, len(cands))), best first."""
+    ranked = sorted(cands, key=lambda cp: (-cp[0], cp[1]))
+    n_q = sum(1 for c, _ in cands if c >= threshold)
+    n_take = min(k, max(min(min_sel, len(cands)), n_q))
+    return [p for _, p in ranked[:n_take]]
+
+
 def topk(cands, k):
     """cands: list of (conf, pos); the k best by (conf desc, pos asc)."""
     return [p for _, p in sorted(cands, key=lambda cp: (-cp[0], cp[1]))[:k]]

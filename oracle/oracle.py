@@ -84,7 +84,32 @@ def row_stats(Z: np.ndarray):
     return tok, m, lse, conf
 
 
-def rows_stats_chunked(H_rows_bits: np.ndarray, W_bits: np.ndarray, chunk: int = V_CHUNK):
+def row_policy_stats(Z: np.ndarray):
+    """Per row of Z [n, V]: (entropy, margin) of the softmax p = softmax(Z).
+
+    entropy = -sum_v p_v ln p_v (natural log); margin = p_(1) - p_(2), the gap between the
+    largest and second-largest probability (0 when the maximum is attained twice; p_(1) when
+    V = 1).  These are the alternative certainty scores of entropy- and margin-driven
+    unmasking (dLLM inference survey page, "Main Findings": confidence/entropy-driven
+    unmasking).
+    """
+    Z = np.asarray(Z, dtype=np.float64)
+    m = Z.max(axis=1, keepdims=True)
+    e = np.exp(Z - m)
+    p = e / e.sum(axis=1, keepdims=True)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        plogp = np.where(p > 0, p * np.log(p), 0.0)
+    entropy = -plogp.sum(axis=1)
+    if Z.shape[1] < 2:
+        margin = p[:, 0].copy()
+    else:
+        top2 = np.partition(p, Z.shape[1] - 2, axis=1)[:, -2:]
+        margin = top2[:, 1] - top2[:, 0]
+    return entropy, margin
+
+
+def rows_stats_chunked(H_rows_bits: np.ndarray, W_bits: np.ndarray, chunk: int = V_CHUNK,
+                       with_policy: bool = False):
     """(tok, m, lse, conf, top2_gap) for rows of H given as bf16 bits, W as bf16 bits.
 
     Logits are formed chunk by chunk over the vocabulary and kept whole per row before the
@@ -101,6 +126,9 @@ def rows_stats_chunked(H_rows_bits: np.ndarray, W_bits: np.ndarray, chunk: int =
         Z[:, v0:v1] = logits_rows(H64, bf16_bits_to_f64(W_bits[v0:v1]))
     tok, m, lse, conf = row_stats(Z)
     gap = top2_gap(Z)
+    if with_policy:
+        entropy, margin = row_policy_stats(Z)
+        return tok, m, lse, conf, gap, entropy, margin
     return tok, m, lse, conf, gap
 
 
@@ -179,6 +207,35 @@ def select_unmask(conf, row_idx, seq_off, L: int, k: int, win_lo=None, win_hi=No
 # --------------------------------------------------------------------------------------
 # the whole step
 # --------------------------------------------------------------------------------------
+def select_unmask_threshold(score, row_idx, seq_off, L: int, k: int, threshold: float,
+                            min_sel: int = 1, win_lo=None, win_hi=None):
+    """Threshold-based parallel unmasking (dLLM pages: decoding thresholds): per sequence,
+    every candidate whose score is at least `threshold` is unmasked, at most k of them, and
+    at least min(min_sel, number of candidates) (the best ones) so that decoding always
+    advances.  Order and ties as in ``select_unmask`` (score descending, position
+    ascending).  threshold = -inf gives plain top-k.
+    """
+    score = np.asarray(score)
+    row_idx = np.asarray(row_idx, dtype=np.int64)
+    seq_off = np.asarray(seq_off, dtype=np.int64)
+    B = seq_off.size - 1
+    idx = np.full((B, k), -1, dtype=np.int32)
+    n_sel = np.zeros(B, dtype=np.int32)
+    for b in range(B):
+        r0, r1 = seq_off[b], seq_off[b + 1]
+        pos = row_idx[r0:r1] - b * L
+        c = score[r0:r1]
+        if win_lo is not None:
+            keep = (pos >= win_lo[b]) & (pos < win_hi[b])
+            pos, c = pos[keep], c[keep]
+        n_q = int((c >= threshold).sum())
+        n_take = min(k, max(min(min_sel, c.size), n_q))
+        order = np.lexsort((pos, -c))[:n_take]
+        n_sel[b] = n_take
+        idx[b, :n_take] = pos[order]
+    return idx, n_sel
+
+
 def oracle_rows(H_bits, W_bits, M, rows=None):
     """Mask-only logits statistics for masked rows (all, or the given compacted rows).
 
@@ -190,9 +247,10 @@ def oracle_rows(H_bits, W_bits, M, rows=None):
         rows = np.arange(count, dtype=np.int64)
     rows = np.asarray(rows, dtype=np.int64)
     H_sel = np.asarray(H_bits)[row_idx[rows]]
-    tok, m, lse, conf, gap = rows_stats_chunked(H_sel, np.asarray(W_bits))
+    tok, m, lse, conf, gap, entropy, margin = rows_stats_chunked(H_sel, np.asarray(W_bits),
+                                                                 with_policy=True)
     return dict(row_idx=row_idx, seq_off=seq_off, count=count, rows=rows,
-                tok=tok, m=m, lse=lse, conf=conf, gap=gap)
+                tok=tok, m=m, lse=lse, conf=conf, gap=gap, entropy=entropy, margin=margin)
 
 
 def oracle_step(H_bits, W_bits, M, k, win_lo=None, win_hi=None):

@@ -210,6 +210,83 @@ def check_merge_split_invariance(o):
     assert tok0[3] == 10
 
 
+def check_policy_closed_forms(o):
+    """Entropy / margin of softmax: uniform -> (ln V, 0); one logit c above V-1 zeros ->
+    (ln S - c e^c / S, (e^c - 1) / S) with S = e^c + V - 1; V = 1 -> (0, 1)."""
+    rng = np.random.default_rng(21)
+    d, V = 8, 50
+    w = _rand_bits(rng, (1, d))
+    H = _rand_bits(rng, (3, d))
+    out = o.oracle_rows(H, np.repeat(w, V, axis=0), np.ones((1, 3), np.uint8))
+    np.testing.assert_allclose(out["entropy"], math.log(V), rtol=1e-13)
+    np.testing.assert_allclose(out["margin"], 0.0, atol=1e-15)
+    Wf = np.zeros((V, d), np.float32)
+    Wf[:d, :d] = np.eye(d)
+    for j, c in [(0, 3.0), (4, 0.5), (7, 9.0)]:
+        Hf = np.zeros((1, d), np.float32)
+        Hf[0, j] = c
+        out = o.oracle_rows(_bits(Hf), _bits(Wf), np.ones((1, 1), np.uint8))
+        S = math.exp(c) + V - 1
+        np.testing.assert_allclose(out["entropy"], [math.log(S) - c * math.exp(c) / S], rtol=1e-12)
+        np.testing.assert_allclose(out["margin"], [(math.exp(c) - 1) / S], rtol=1e-12)
+    out = o.oracle_rows(_rand_bits(rng, (2, 8)), _rand_bits(rng, (1, 8)), np.ones((1, 2), np.uint8))
+    np.testing.assert_allclose(out["entropy"], 0.0, atol=0)
+    np.testing.assert_allclose(out["margin"], 1.0, atol=0)
+
+
+def check_policy_library_and_brute(o):
+    """Entropy against scipy.stats.entropy of the softmax, margin against a full sort, both
+    against the pure-Python brute force."""
+    import scipy.stats
+    rng = np.random.default_rng(23)
+    H, W = _rand_bits(rng, (12, 32)), _rand_bits(rng, (200, 32), 0.4)
+    out = o.oracle_rows(H, W, np.ones((1, 12), np.uint8))
+    Z = o.bf16_bits_to_f64(H) @ o.bf16_bits_to_f64(W).T
+    P = scipy.special.softmax(Z, axis=1)
+    np.testing.assert_allclose(out["entropy"], scipy.stats.entropy(P, axis=1), rtol=1e-12)
+    Ps = np.sort(P, axis=1)
+    np.testing.assert_allclose(out["margin"], Ps[:, -1] - Ps[:, -2], rtol=1e-12, atol=1e-15)
+    Hl, Wl = _bf16_list(H), _bf16_list(W)
+    for i in range(4):
+        ent, mar = brute.policy_stats(brute.row_logits(Hl[i], Wl))
+        np.testing.assert_allclose(out["entropy"][i], ent, rtol=1e-12)
+        np.testing.assert_allclose(out["margin"][i], mar, rtol=1e-12, atol=1e-15)
+
+
+def check_threshold_select(o):
+    g = json.load(open(os.path.join(GOLDEN, "threshold_select.json")))
+    M = np.array(g["M"], dtype=np.uint8)
+    row_idx, seq_off, _ = o.mask_compact(M)
+    for dt in (np.float32, np.float64):
+        score = np.array(g["score"], dtype=dt)
+        for c in g["cases"]:
+            lo = np.array([c["lo"]]) if "lo" in c else None
+            hi = np.array([c["hi"]]) if "hi" in c else None
+            idx, n_sel = o.select_unmask_threshold(score, row_idx, seq_off, g["L"], c["k"],
+                                                   c["threshold"], c["min_sel"], lo, hi)
+            assert idx[0].tolist() == c["idx"], (c, idx)
+            assert int(n_sel[0]) == c["n_sel"]
+    # brute force on random inputs; -inf threshold is plain top-k
+    rng = np.random.default_rng(29)
+    for _ in range(20):
+        B, L = int(rng.integers(1, 4)), int(rng.integers(1, 30))
+        M = (rng.random((B, L)) < 0.7).astype(np.uint8)
+        row_idx, seq_off, count = o.mask_compact(M)
+        score = (rng.integers(0, 8, size=count) / 8.0).astype(np.float64)
+        k = int(rng.integers(1, 8))
+        tau = float(rng.choice([-np.inf, 0.25, 0.5, 0.875, 2.0]))
+        ms = int(rng.integers(0, 3))
+        idx, n_sel = o.select_unmask_threshold(score, row_idx, seq_off, L, k, tau, ms)
+        for b in range(B):
+            cands = [(score[r], int(row_idx[r]) - b * L) for r in range(seq_off[b], seq_off[b + 1])]
+            ref = brute.select_threshold(cands, k, tau, ms)
+            assert idx[b, :n_sel[b]].tolist() == ref and int(n_sel[b]) == len(ref)
+        if tau == -np.inf:
+            t_idx, t_n = o.select_unmask(score, row_idx, seq_off, L, k)
+            assert np.array_equal(t_idx, idx) and np.array_equal(t_n, n_sel)
+
+
 ALL_CHECKS = [check_handworked, check_topk_ties, check_compact, check_brute_random,
               check_closed_forms, check_library_routines, check_invariants,
-              check_mask_only_equals_full, check_merge_split_invariance]
+              check_mask_only_equals_full, check_merge_split_invariance,
+              check_policy_closed_forms, check_policy_library_and_brute, check_threshold_select]

@@ -1,0 +1,185 @@
+"""Unmask-policy variants on the GPU against the oracle: softmax entropy and top-2
+probability margin per masked row (dllm_masked_logits_ex), and threshold-based parallel
+unmasking (dllm_select_unmask_ex), descending and ascending.
+
+Tolerances (fp32 accumulation of bf16 products, like lse and conf): entropy within 2e-3
+relative plus 2e-5 absolute; margin within 2e-3 relative plus 1e-4 x conf absolute (the
+margin is (1 - exp(m2 - m)) / s, so an error d in the top-2 logit gap moves it by about
+d x conf).  Selections are bit-exact against the oracle run on the GPU's own scores.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.oracle as O
+import workloads as WL
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dl():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import mask_only_logits_b200 as dl
+    return dl
+
+
+@pytest.fixture(params=[0, 1, 2], ids=["default", "single", "pair"])
+def variant(request, dl):
+    dl.debug_set_gemm_variant(request.param)
+    yield request.param
+    dl.debug_set_gemm_variant(0)
+
+
+def _run_ex(dl, inp, stats):
+    cfg = inp["cfg"]
+    n = cfg.B * cfg.L
+    dev = dict(H=inp["H"].cuda(), M=inp["M"].cuda(), W=inp["W"].cuda())
+    f32 = dict(dtype=torch.float32, device="cuda")
+    i32 = dict(dtype=torch.int32, device="cuda")
+    tok, conf, lse = torch.empty(n, **i32), torch.empty(n, **f32), torch.empty(n, **f32)
+    ent = torch.empty(n, **f32) if stats & dl.STAT_ENTROPY else None
+    mar = torch.empty(n, **f32) if stats & dl.STAT_MARGIN else None
+    row_idx, seq_off, count = torch.empty(n, **i32), torch.empty(cfg.B + 1, **i32), torch.empty(4, **i32)
+    ws = torch.empty(dl.workspace_bytes(cfg.B, cfg.L, cfg.d, cfg.V), dtype=torch.uint8, device="cuda")
+    dl.masked_logits_ex(dev["H"], dev["M"], dev["W"], stats, tok, conf, lse, ent, mar, row_idx,
+                        seq_off, count, ws)
+    assert dl.get_status() == 0
+    c = int(count[0])
+    out = dict(count=c, tok=tok[:c].cpu().numpy(), conf=conf[:c].cpu().numpy(),
+               lse=lse[:c].cpu().numpy(), row_idx=row_idx[:c].cpu().numpy(),
+               seq_off=seq_off.cpu().numpy())
+    if ent is not None:
+        out["entropy"] = ent[:c].cpu().numpy()
+    if mar is not None:
+        out["margin"] = mar[:c].cpu().numpy()
+    return out
+
+
+def _check_policy(g, ref, rows):
+    e_g = g["entropy"][rows].astype(np.float64)
+    m_g = g["margin"][rows].astype(np.float64)
+    assert np.all(np.isfinite(e_g)) and np.all(np.isfinite(m_g))
+    assert np.all(np.abs(e_g - ref["entropy"]) <= 2e-3 * np.abs(ref["entropy"]) + 2e-5), \
+        float(np.max(np.abs(e_g - ref["entropy"])))
+    assert np.all(np.abs(m_g - ref["margin"]) <= 2e-3 * np.abs(ref["margin"]) + 1e-4 * ref["conf"]), \
+        float(np.max(np.abs(m_g - ref["margin"]) / ref["conf"]))
+    # the plain statistics are unchanged by the extended epilogue
+    np.testing.assert_allclose(g["lse"][rows], ref["lse"], rtol=2e-3)
+    np.testing.assert_allclose(g["conf"][rows], ref["conf"], rtol=2e-3)
+
+
+@pytest.mark.parametrize("B,L,d,V,r", [(1, 256, 256, 4096, 0.5),      # cfg0 shapes
+                                       (2, 300, 64, 1000, 0.8),       # V tail, ragged rows
+                                       (1, 6000, 128, 700, 0.9),      # several groups: merged
+                                       (1, 1000, 64, 37800, 1.0),     # remainder holders
+                                       (1, 50, 64, 1, 1.0)])          # V = 1: entropy 0
+def test_entropy_margin(dl, variant, B, L, d, V, r):
+    inp = WL.make_inputs(WL.custom_config(B, L, d, V, 4, r=r), seed=3)
+    g = _run_ex(dl, inp, dl.STAT_ENTROPY | dl.STAT_MARGIN)
+    Hb, Wb, M = WL.bf16_bits(inp["H"]), WL.bf16_bits(inp["W"]), inp["M"].numpy()
+    rows = np.arange(g["count"])
+    ref = O.oracle_rows(Hb, Wb, M, rows)
+    _check_policy(g, ref, rows)
+    ok_tok = (g["tok"] == ref["tok"]) | (ref["gap"] < 1e-3)
+    assert ok_tok.all()
+
+
+def test_entropy_margin_cfg1_every_row(dl):
+    inp = WL.make_inputs(WL.CONFIGS["cfg1"], seed=0)
+    g = _run_ex(dl, inp, dl.STAT_ENTROPY | dl.STAT_MARGIN)
+    Hb, Wb, M = WL.bf16_bits(inp["H"]), WL.bf16_bits(inp["W"]), inp["M"].numpy()
+    rows = np.arange(g["count"])
+    _check_policy(g, O.oracle_rows(Hb, Wb, M, rows), rows)
+
+
+def test_margin_exact_ties_and_single_flags(dl):
+    # duplicated vocabulary rows -> the top logit is attained twice: margin exactly 0
+    rng = np.random.default_rng(4)
+    W = torch.from_numpy((rng.standard_normal((300, 64)) * 0.3).astype(np.float32)).to(torch.bfloat16)
+    W[200] = W[7]
+    inp = WL.make_inputs(WL.custom_config(1, 128, 64, 300, 4, r=1.0), seed=1)
+    inp["W"] = W
+    g = _run_ex(dl, inp, dl.STAT_MARGIN)
+    ref = O.oracle_rows(WL.bf16_bits(inp["H"]), WL.bf16_bits(W), inp["M"].numpy())
+    tie_rows = np.flatnonzero(ref["margin"] == 0.0)
+    assert np.all(g["margin"][tie_rows] == 0.0)
+    assert "entropy" not in g
+    g2 = _run_ex(dl, inp, dl.STAT_ENTROPY)
+    assert "margin" not in g2 and np.all(np.isfinite(g2["entropy"]))
+
+
+def _select_ex(dl, score_np, M_np, k, tau, min_sel, ascending, win=None):
+    B, L = M_np.shape
+    row_idx, seq_off, count = O.mask_compact(M_np)
+    score = torch.from_numpy(score_np.astype(np.float32)).cuda()
+    idx = torch.full((B, k), -9, dtype=torch.int32, device="cuda")
+    n_sel = torch.full((B,), -9, dtype=torch.int32, device="cuda")
+    sc_sel = torch.empty((B, k), dtype=torch.float32, device="cuda")
+    lo = hi = None
+    if win is not None:
+        lo = torch.from_numpy(win[0].astype(np.int32)).cuda()
+        hi = torch.from_numpy(win[1].astype(np.int32)).cuda()
+    dl.select_unmask_ex(score, torch.from_numpy(row_idx).cuda(), torch.from_numpy(seq_off).cuda(),
+                        B, L, k, tau, min_sel, idx, n_sel, ascending, lo, hi, score_sel=sc_sel)
+    s32 = score_np.astype(np.float32).astype(np.float64)
+    # ascending order == descending order of the negated scores (negation is exact)
+    ref_idx, ref_n = O.select_unmask_threshold(-s32 if ascending else s32, row_idx, seq_off, L,
+                                               k, -tau if ascending else tau, min_sel,
+                                               None if win is None else win[0],
+                                               None if win is None else win[1])
+    np.testing.assert_array_equal(n_sel.cpu().numpy(), ref_n)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
+    return idx.cpu().numpy(), n_sel.cpu().numpy()
+
+
+@pytest.mark.parametrize("ascending", [False, True])
+@pytest.mark.parametrize("tau,min_sel,k", [(0.5, 1, 64), (0.9, 1, 16), (0.99, 0, 16),
+                                           (0.99, 3, 16), (-1.0, 1, 32), (0.25, 1, 1024)])
+def test_threshold_select_bit_exact(dl, ascending, tau, min_sel, k):
+    rng = np.random.default_rng(abs(int(tau * 100)) + k)
+    B, L = 3, 5000
+    M = (rng.random((B, L)) < 0.6).astype(np.uint8)
+    n = int(M.sum())
+    score = (rng.integers(0, 64, size=n) / 64.0).astype(np.float32)     # many exact ties
+    if ascending:
+        score = -score + 0.5                                               # negative values too
+    _select_ex(dl, score, M, k, tau, min_sel, ascending)
+
+
+def test_threshold_select_plain_topk_and_windows(dl):
+    rng = np.random.default_rng(9)
+    M = WL.make_mask(WL.CONFIGS["cfg4"]).numpy()
+    n = int(M.sum())
+    score = rng.standard_normal(n).astype(np.float32)
+    lo, hi = WL.make_windows(WL.CONFIGS["cfg4"])
+    idx, n_sel = _select_ex(dl, score, M, 4, float("-inf"), 1, False, (lo, hi))
+    row_idx, seq_off, _ = O.mask_compact(M)
+    t_idx, t_n = O.select_unmask(score, row_idx, seq_off, M.shape[1], 4, lo, hi)
+    assert np.array_equal(idx, t_idx) and np.array_equal(n_sel, t_n)
+    _select_ex(dl, score, M, 8, 0.0, 2, False, (lo, hi))
+    _select_ex(dl, score, M, 8, 0.0, 2, True, (lo, hi))
+    _select_ex(dl, score, M, 32, float("inf"), 1, True)
+
+
+def test_entropy_driven_step(dl):
+    """Entropy-driven unmasking end to end: entropies from the GEMM epilogue, then the k
+    lowest-entropy positions (ascending) with a threshold, against the oracle's selection
+    on the same (GPU) entropies."""
+    inp = WL.make_inputs(WL.CONFIGS["cfg0"], seed=2)
+    g = _run_ex(dl, inp, dl.STAT_ENTROPY)
+    M = inp["M"].numpy()
+    ent = g["entropy"]
+    tau = float(np.quantile(ent, 0.1))
+    ent_dev = torch.from_numpy(ent).cuda()
+    B, L = M.shape
+    idx = torch.empty((B, 8), dtype=torch.int32, device="cuda")
+    n_sel = torch.empty((B,), dtype=torch.int32, device="cuda")
+    dl.select_unmask_ex(ent_dev, torch.from_numpy(g["row_idx"]).cuda(),
+                        torch.from_numpy(g["seq_off"]).cuda(), B, L, 8, tau, 1, idx, n_sel,
+                        ascending=True)
+    e64 = ent.astype(np.float64)
+    ref_idx, ref_n = O.select_unmask_threshold(-e64, g["row_idx"], g["seq_off"], L, 8, -tau, 1)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
+    np.testing.assert_array_equal(n_sel.cpu().numpy(), ref_n)

@@ -116,7 +116,51 @@ def _make_select(variant):
     return select_unmask
 
 
+def _policy_entropy_log2(Z):
+    Z = np.asarray(Z, dtype=np.float64)
+    m = Z.max(axis=1, keepdims=True)
+    p = np.exp(Z - m)
+    p = p / p.sum(axis=1, keepdims=True)
+    ent = -(p * np.log2(np.where(p > 0, p, 1.0))).sum(axis=1)      # wrong log base
+    s = np.sort(p, axis=1)
+    return ent, s[:, -1] - (s[:, -2] if p.shape[1] > 1 else 0)
+
+
+def _policy_margin_of_logits(Z):
+    Z = np.asarray(Z, dtype=np.float64)
+    m = Z.max(axis=1, keepdims=True)
+    p = np.exp(Z - m)
+    p = p / p.sum(axis=1, keepdims=True)
+    ent = -(p * np.log(np.where(p > 0, p, 1.0))).sum(axis=1)
+    s = np.sort(Z, axis=1)                                           # logits, not probabilities
+    return ent, s[:, -1] - (s[:, -2] if Z.shape[1] > 1 else 0)
+
+
+def _threshold_strict(score, row_idx, seq_off, L, k, threshold, min_sel=1, win_lo=None, win_hi=None):
+    score = np.asarray(score)
+    row_idx = np.asarray(row_idx, dtype=np.int64)
+    seq_off = np.asarray(seq_off, dtype=np.int64)
+    B = seq_off.size - 1
+    idx = np.full((B, k), -1, dtype=np.int32)
+    n_sel = np.zeros(B, dtype=np.int32)
+    for b in range(B):
+        pos = row_idx[seq_off[b]:seq_off[b + 1]] - b * L
+        c = score[seq_off[b]:seq_off[b + 1]]
+        if win_lo is not None:
+            keep = (pos >= win_lo[b]) & (pos < win_hi[b])
+            pos, c = pos[keep], c[keep]
+        n_q = int((c > threshold).sum())                              # strict: drops equality
+        n_take = min(k, max(min(min_sel, c.size), n_q))
+        order = np.lexsort((pos, -c))[:n_take]
+        n_sel[b] = n_take
+        idx[b, :n_take] = pos[order]
+    return idx, n_sel
+
+
 MUTATIONS = {
+    "entropy_log2": ("row_policy_stats", _policy_entropy_log2),
+    "margin_of_logits": ("row_policy_stats", _policy_margin_of_logits),
+    "threshold_strict": ("select_unmask_threshold", _threshold_strict),
     "argmin_for_argmax": ("row_stats", _row_stats_argmin),
     "lse_drops_max": ("row_stats", _row_stats_drop_m),
     "conf_wrong_sign": ("row_stats", _row_stats_sign),
