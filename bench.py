@@ -46,6 +46,31 @@ def load_peaks() -> dict:
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
 
 
+GEMM_SOURCES = ["mask_only_logits_b200/csrc/lmhead.cuh", "mask_only_logits_b200/csrc/ptx.cuh"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "lmhead_traffic.json")
+
+
+def gemm_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in GEMM_SOURCES:
+        h.update(open(os.path.join(ROOT, rel), "rb").read())
+    return h.hexdigest()
+
+
+def measured_traffic(workload: str, kernel: str):
+    """DRAM bytes (read + write) per GEMM launch from the committed ncu capture, if it was
+    taken on this workload and kernel and the GEMM's sources have not changed since."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    rec = json.load(open(TRAFFIC_FILE))
+    for c in rec.get("captures", []):
+        if (c["workload"] == workload and c["kernel"] == kernel
+                and c["source_sha256"] == gemm_source_hash()):
+            return c["dram_read_bytes"] + c["dram_write_bytes"]
+    return None
+
+
 def algorithmic(cfg, M: int) -> dict:
     """Work of one step: flops of the dense contraction and bytes that must move once."""
     flops = 2.0 * M * cfg.V * cfg.d
@@ -298,13 +323,19 @@ def main() -> None:
     for _ in range(3):
         step.run_host(H_host, M_host, W, win_lo, win_hi, stream)
     barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        step.run_host(H_host, M_host, W, win_lo, win_hi, stream)
-    e1.record(stream)
+    # the decode loop a serving process runs: each step's inputs copied in from pinned host
+    # memory (overlapping the previous step) and its selection copied back
+    for _ in step.run_host_pipeline([(H_host, M_host)] * 3, W, win_lo, win_hi, stream):
+        pass
     torch.cuda.synchronize(dev)
-    e2e_ms = D.max_over_ranks([e0.elapsed_time(e1)], dev)[0]
+    barrier()
+    t0 = time.perf_counter()
+    n_out = 0
+    for _ in step.run_host_pipeline([(H_host, M_host)] * e2e_steps, W, win_lo, win_hi, stream):
+        n_out += 1
+    torch.cuda.synchronize(dev)
+    e2e_ms = D.max_over_ranks([(time.perf_counter() - t0) * 1e3], dev)[0]
+    assert n_out == e2e_steps
     barrier()
 
     if rank == 0:
@@ -318,6 +349,8 @@ def main() -> None:
         step_tflops = a["flops"] / (ms_step / 1e3) / 1e12
         step_gbs = a["bytes"] / (ms_step / 1e3) / 1e9
         full_logits = cfg.B * cfg.L * cfg.V * 4
+        paired = args.gemm_variant == 2 or (args.gemm_variant == 0 and cfg.B * cfg.L <= 16384)
+        gemm_kernel_name = "lmhead_kernel<2, 0>" if paired else "lmhead_kernel<1, 0>"
         line = dict(
             metric=METRIC, value=rows_s, unit=UNIT, n_gpus=world, steps=args.steps,
             warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True, scaling="weak",
@@ -328,16 +361,17 @@ def main() -> None:
             roofline_ms=roof * 1e3,
             roofline=dict(bound="tensor" if a["flops"] / (peaks["bf16_tflops"] * 1e12) >=
                           a["bytes"] / (peaks["hbm_gbs"] * 1e9) else "hbm",
-                          kernel=("masked_lmhead, paired-SM tcgen05 (lmhead_kernel<2>)"
-                                  if args.gemm_variant == 2 or
-                                  (args.gemm_variant == 0 and cfg.B * cfg.L <= 16384) else
-                                  "masked_lmhead, single-SM tcgen05 (lmhead_kernel<1>)"),
+                          kernel=("masked_lmhead, paired-SM tcgen05 (lmhead_kernel<2, 0>)"
+                                  if paired else
+                                  "masked_lmhead, single-SM tcgen05 (lmhead_kernel<1, 0>)"),
                           achieved=tflops_gemm, peak=peaks["bf16_tflops"], unit="TFLOP/s",
                           frac=tflops_gemm / peaks["bf16_tflops"],
                           frac_of_sustained=(tflops_gemm / peaks["bf16_tflops_sustained"]
                                              if peaks.get("bf16_tflops_sustained") else None),
                           peak_source=peaks["source"] + " (burst bf16 GEMM)",
-                          gemm_ms_avg=gemm_avg_s * 1e3, traffic=None),
+                          gemm_ms_avg=gemm_avg_s * 1e3,
+                          algorithmic_bytes=2.0 * cfg.V * cfg.d + 2.0 * count * cfg.d,
+                          traffic=measured_traffic(cfg.name, gemm_kernel_name)),
             gpu_launches=launches,
             memory=dict(peak_step_bytes=int(step_peak),
                         full_logits_fp32_bytes=int(full_logits),
@@ -346,7 +380,10 @@ def main() -> None:
                              "analytic"),
             e2e=dict(value=count * world * e2e_steps / (e2e_ms / 1e3), unit=UNIT,
                      h2d_bytes_per_step=step.h2d_bytes(), d2h_bytes_per_step=step.d2h_bytes(),
-                     ms_per_step=e2e_ms / e2e_steps),
+                     ms_per_step=e2e_ms / e2e_steps,
+                     note="DecodeStep.run_host_pipeline: per step H and the mask copied from "
+                          "pinned host memory (overlapping the previous step's compute) and the "
+                          "selection copied back; wall clock, device synchronised at both ends"),
             clocks=clk.summary(),
         )
         if cpu is not None:

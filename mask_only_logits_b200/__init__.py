@@ -21,13 +21,15 @@ from . import _abi
 
 __all__ = [
     "DllmError", "lib", "version", "workspace_bytes", "mask_compact", "mask_compact_noalloc",
-    "masked_logits",
+    "masked_logits", "masked_logits_ex", "select_unmask_ex", "STAT_ENTROPY", "STAT_MARGIN",
     "select_unmask", "decode_step", "get_status", "debug_lmhead_logits", "debug_lse_merge",
     "debug_set_gemm_variant",
     "prof_begin", "prof_end", "DecodeStep", "MAX_K",
 ]
 
 MAX_K = 1024
+STAT_ENTROPY = 1
+STAT_MARGIN = 2
 
 STATUS = {0: "DLLM_OK", -1: "DLLM_ERR_NULL", -2: "DLLM_ERR_ALIGN", -3: "DLLM_ERR_SHAPE",
           -4: "DLLM_ERR_WORKSPACE", -5: "DLLM_ERR_CUDA", -6: "DLLM_ERR_TIMEOUT",
@@ -108,6 +110,37 @@ def masked_logits(H, M, W, tok, conf, lse, row_idx, seq_off, count, ws, stream=N
         _ptr(seq_off, torch.int32, "seq_off"), _ptr(count, torch.int32, "count"),
         _ptr(ws, None, "ws"), ws.numel() * ws.element_size(), _stream(stream)),
         "dllm_masked_logits")
+
+
+def masked_logits_ex(H, M, W, stats, tok, conf, lse, entropy, margin, row_idx, seq_off, count,
+                     ws, stream=None) -> None:
+    """masked_logits plus the softmax entropy and/or top-2 probability margin per masked row
+    (stats: bitwise OR of STAT_ENTROPY and STAT_MARGIN; pass None for outputs not asked for)."""
+    B, L = M.shape
+    V, d = W.shape
+    _check(lib().dllm_masked_logits_ex(
+        _ptr(H, torch.bfloat16, "H"), _ptr(M, torch.uint8, "M"), _ptr(W, torch.bfloat16, "W"),
+        B, L, d, V, stats, _ptr(tok, torch.int32, "tok"), _ptr(conf, torch.float32, "conf"),
+        _ptr(lse, torch.float32, "lse"), _ptr(entropy, torch.float32, "entropy"),
+        _ptr(margin, torch.float32, "margin"), _ptr(row_idx, torch.int32, "row_idx"),
+        _ptr(seq_off, torch.int32, "seq_off"), _ptr(count, torch.int32, "count"),
+        _ptr(ws, None, "ws"), ws.numel() * ws.element_size(), _stream(stream)),
+        "dllm_masked_logits_ex")
+
+
+def select_unmask_ex(score, row_idx, seq_off, B, L, k, threshold, min_sel, idx, n_sel,
+                     ascending=False, win_lo=None, win_hi=None, tok=None, tok_sel=None,
+                     score_sel=None, stream=None) -> None:
+    """Threshold-based selection: per sequence min(k, max(min(min_sel, n), #qualifying))
+    best candidates; qualifying = score >= threshold (<= with ascending=True)."""
+    _check(lib().dllm_select_unmask_ex(
+        _ptr(score, torch.float32, "score"), _ptr(row_idx, torch.int32, "row_idx"),
+        _ptr(seq_off, torch.int32, "seq_off"), B, L, k, float(threshold), min_sel,
+        1 if ascending else 0, _ptr(win_lo, torch.int32, "win_lo"),
+        _ptr(win_hi, torch.int32, "win_hi"), _ptr(tok, torch.int32, "tok"),
+        _ptr(idx, torch.int32, "idx"), _ptr(n_sel, torch.int32, "n_sel"),
+        _ptr(tok_sel, torch.int32, "tok_sel"), _ptr(score_sel, torch.float32, "score_sel"),
+        _stream(stream)), "dllm_select_unmask_ex")
 
 
 def select_unmask(conf, row_idx, seq_off, B, L, k, idx, n_sel, win_lo=None, win_hi=None,
@@ -250,6 +283,74 @@ class DecodeStep:
             hb["conf_sel"].copy_(self.conf_sel, non_blocking=True)
         s.synchronize()
         return dict(idx=hb["idx"], n_sel=hb["n_sel"], tok_sel=hb["tok_sel"], conf_sel=hb["conf_sel"])
+
+    def run_host_pipeline(self, batches, W, win_lo=None, win_hi=None, stream=None,
+                          copy_stream=None):
+        """Decode steps over host batches [(H_host, M_host), ...] (pinned), with the copy of
+        batch i+1 into the device overlapping the step of batch i.
+
+        Two device input buffers alternate; a copy stream loads batch i+1 while the compute
+        stream runs step i and copies its selection back to pinned host memory.  Yields, per
+        step, host tensors idx, n_sel, tok_sel, conf_sel (valid until the next iteration).
+        """
+        B, L, d, k = self.B, self.L, self.d, self.k
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        cs = copy_stream if copy_stream is not None else torch.cuda.Stream(self.device)
+        if getattr(self, "_pipe", None) is None:
+            pin = dict(pin_memory=True)
+            self._pipe = dict(
+                H=[torch.empty(B * L, d, dtype=torch.bfloat16, device=self.device) for _ in range(2)],
+                M=[torch.empty(B, L, dtype=torch.uint8, device=self.device) for _ in range(2)],
+                out=[dict(idx=torch.empty(B, k, dtype=torch.int32, **pin),
+                          n_sel=torch.empty(B, dtype=torch.int32, **pin),
+                          tok_sel=torch.empty(B, k, dtype=torch.int32, **pin),
+                          conf_sel=torch.empty(B, k, dtype=torch.float32, **pin)) for _ in range(2)])
+        pb = self._pipe
+        loaded = [torch.cuda.Event() for _ in range(2)]
+        freed = [torch.cuda.Event() for _ in range(2)]
+        done = [torch.cuda.Event() for _ in range(2)]
+
+        def load(i, Hh, Mh):
+            b = i & 1
+            with torch.cuda.stream(cs):
+                if i >= 2:
+                    cs.wait_event(freed[b])          # step i-2 no longer reads this buffer
+                pb["H"][b].copy_(Hh, non_blocking=True)
+                pb["M"][b].copy_(Mh, non_blocking=True)
+                loaded[b].record(cs)
+
+        it = iter(batches)
+        first = next(it, None)
+        if first is None:
+            return
+        load(0, *first)
+        i = 0
+        pending = None
+        nxt = next(it, None)
+        while True:
+            b = i & 1
+            if nxt is not None:
+                load(i + 1, *nxt)                    # overlaps step i below
+            with torch.cuda.stream(s):
+                s.wait_event(loaded[b])
+                self.run(pb["H"][b], pb["M"][b], W, win_lo, win_hi, s)
+                freed[b].record(s)
+                o = pb["out"][b]
+                o["idx"].copy_(self.idx, non_blocking=True)
+                o["n_sel"].copy_(self.n_sel, non_blocking=True)
+                o["tok_sel"].copy_(self.tok_sel, non_blocking=True)
+                o["conf_sel"].copy_(self.conf_sel, non_blocking=True)
+                done[b].record(s)
+            if pending is not None:
+                done[pending].synchronize()
+                yield pb["out"][pending]
+            pending = b
+            if nxt is None:
+                break
+            nxt = next(it, None)
+            i += 1
+        done[pending].synchronize()
+        yield pb["out"][pending]
 
     def h2d_bytes(self) -> int:
         return self.B * self.L * self.d * 2 + self.B * self.L

@@ -31,6 +31,7 @@ namespace dllm {
 
 constexpr int kSelThreads = 1024;
 constexpr int kSelMaxK = 1024;
+constexpr int kSelStage = 4096;     // up to this many candidates: keys staged in shared memory
 
 // Float -> unsigned with the same order (for non-NaN values).
 __device__ __forceinline__ uint32_t ordered_bits(float f) {
@@ -51,6 +52,7 @@ select_unmask_kernel(const float* __restrict__ conf, const int* __restrict__ row
                      const int* __restrict__ tok, int* __restrict__ idx, int* __restrict__ n_sel,
                      int* __restrict__ tok_sel, float* __restrict__ conf_sel) {
   __shared__ unsigned long long keys[kSelMaxK];
+  __shared__ uint32_t skey[kSelStage];
   __shared__ unsigned int hist[256];
   __shared__ int sh_lo, sh_hi, sh_n, sh_digit, sh_krem, sh_taken, sh_q;
   __shared__ int warp_cnt[32];
@@ -88,13 +90,20 @@ select_unmask_kernel(const float* __restrict__ conf, const int* __restrict__ row
     c1 = sh_hi > sh_lo ? sh_hi : sh_lo;
   }
   const int n = c1 - c0;
+  // small candidate sets: read the scores once and keep their keys in shared memory
+  const bool staged = n <= kSelStage;
+  if (staged) {
+    for (int r = c0 + tid; r < c1; r += kSelThreads) skey[r - c0] = okey(conf[r]);
+    __syncthreads();
+  }
+  auto key_of = [&](int r) -> uint32_t { return staged ? skey[r - c0] : okey(conf[r]); };
   int k_eff = n < k ? n : k;
   if (use_threshold) {
     if (tid == 0) sh_q = 0;
     __syncthreads();
     const uint32_t tq = okey(threshold);
     int mine = 0;
-    for (int r = c0 + tid; r < c1; r += kSelThreads) mine += okey(conf[r]) >= tq ? 1 : 0;
+    for (int r = c0 + tid; r < c1; r += kSelThreads) mine += key_of(r) >= tq ? 1 : 0;
     for (int o = 16; o > 0; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
     if (lane == 0 && mine) atomicAdd(&sh_q, mine);
     __syncthreads();
@@ -109,7 +118,7 @@ select_unmask_kernel(const float* __restrict__ conf, const int* __restrict__ row
 
   if (n <= k_eff) {
     // 2'. every candidate is selected
-    for (int r = c0 + tid; r < c1; r += kSelThreads) keys[r - c0] = sel_key(okey(conf[r]), r);
+    for (int r = c0 + tid; r < c1; r += kSelThreads) keys[r - c0] = sel_key(key_of(r), r);
   } else if (k_eff > 0) {
     // 2. radix select of the k_eff-th largest key
     uint32_t prefix = 0, pmask = 0;
@@ -123,7 +132,7 @@ select_unmask_kernel(const float* __restrict__ conf, const int* __restrict__ row
         const int r = base + tid;
         uint32_t bin = 0xFFFFFFFFu;
         if (r < c1) {
-          const uint32_t u = okey(conf[r]);
+          const uint32_t u = key_of(r);
           if ((u & pmask) == prefix) bin = (u >> shift) & 255u;
         }
         const unsigned peers = __match_any_sync(0xffffffffu, bin);
@@ -163,7 +172,7 @@ select_unmask_kernel(const float* __restrict__ conf, const int* __restrict__ row
     for (int base = c0; base < c1; base += kSelThreads) {
       const int r = base + tid;
       uint32_t u = 0;
-      if (r < c1) u = okey(conf[r]);
+      if (r < c1) u = key_of(r);
       const bool gt = r < c1 && u > T;
       const bool eq = r < c1 && u == T;
       if (gt) keys[atomicAdd(&sh_n, 1)] = sel_key(u, r);

@@ -182,3 +182,24 @@ def test_pair_variant_large(dl):
         check_step(dl, WL.make_inputs(WL.CONFIGS["cfg4"], seed=0), all_rows=False, window_rows=True)
     finally:
         dl.debug_set_gemm_variant(0)
+
+
+def test_run_host_pipeline_matches_device_steps(dl):
+    """Overlapped copies must not mix batches: each yielded selection equals that batch's
+    device-resident step."""
+    cfg = WL.CONFIGS["cfg0"]
+    inps = [WL.make_inputs(cfg, seed=s) for s in (0, 1, 2, 3, 4)]
+    W = inps[0]["W"].cuda()                      # one resident W for every batch
+    step = dl.DecodeStep(cfg.B, cfg.L, cfg.d, cfg.V, cfg.k)
+    expected = []
+    for inp in inps:
+        out = step.run(inp["H"].cuda(), inp["M"].cuda(), W)
+        expected.append((out["idx"].cpu().clone(), out["n_sel"].cpu().clone(),
+                         out["tok_sel"].cpu().clone()))
+    batches = [(inp["H"].pin_memory(), inp["M"].pin_memory()) for inp in inps]
+    got = [(o["idx"].clone(), o["n_sel"].clone(), o["tok_sel"].clone())
+           for o in step.run_host_pipeline(batches, W)]
+    assert len(got) == len(expected)
+    for (gi, gn, gt), (ei, en, et) in zip(got, expected):
+        assert torch.equal(gi, ei) and torch.equal(gn, en) and torch.equal(gt, et)
+    assert not all(torch.equal(got[0][0], g[0]) for g in got[1:])   # batches really differ
