@@ -87,6 +87,34 @@ def roofline_s(cfg, M: int, peaks: dict) -> float:
     return max(a["flops"] / (peaks["bf16_tflops"] * 1e12), a["bytes"] / (peaks["hbm_gbs"] * 1e9))
 
 
+def gemm_roofline(cfg, count: int, peaks: dict, gemm_s: float, paired: bool, kernel: str) -> dict:
+    """Roofline of the dominant kernel (the masked LM-head GEMM with its fused epilogue):
+    the tensor pipe when its flops take longer than its bytes at the measured peaks, else
+    HBM.  Algorithmic work per launch: 2 * count * V * d flops; bytes = W once (2 V d) plus
+    the gathered masked rows once (2 count d)."""
+    flops = 2.0 * count * cfg.V * cfg.d
+    gemm_bytes = 2.0 * cfg.V * cfg.d + 2.0 * count * cfg.d
+    tensor_bound = flops / (peaks["bf16_tflops"] * 1e12) >= gemm_bytes / (peaks["hbm_gbs"] * 1e9)
+    out = dict(bound="tensor" if tensor_bound else "hbm",
+               kernel=("masked_lmhead, paired-SM tcgen05 (lmhead_kernel<2, 0>)" if paired else
+                       "masked_lmhead, single-SM tcgen05 (lmhead_kernel<1, 0>)"))
+    tflops = flops / gemm_s / 1e12
+    gbs = gemm_bytes / gemm_s / 1e9
+    if tensor_bound:
+        out.update(achieved=tflops, peak=peaks["bf16_tflops"], unit="TFLOP/s",
+                   frac=tflops / peaks["bf16_tflops"],
+                   frac_of_sustained=(tflops / peaks["bf16_tflops_sustained"]
+                                      if peaks.get("bf16_tflops_sustained") else None),
+                   peak_source=peaks["source"] + " (burst bf16 GEMM)",
+                   achieved_gbs=gbs)
+    else:
+        out.update(achieved=gbs, peak=peaks["hbm_gbs"], unit="GB/s", frac=gbs / peaks["hbm_gbs"],
+                   peak_source=peaks["source"] + " (HBM copy)", achieved_tflops=tflops)
+    out.update(gemm_ms_avg=gemm_s * 1e3, algorithmic_bytes=gemm_bytes, algorithmic_flops=flops,
+               traffic=measured_traffic(cfg.name, kernel))
+    return out
+
+
 # ------------------------------------------------------------------------------ clocks
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples while the timed region runs."""
@@ -156,6 +184,8 @@ def oracle_rate(inp: dict, rows: np.ndarray) -> tuple[float, float]:
     the unmask selection over them; returns (seconds, rows)."""
     import oracle.oracle as O
     Hb, Wb, M = WL.bf16_bits(inp["H"]), WL.bf16_bits(inp["W"]), inp["M"].numpy()
+    if inp["cfg"].block_only:
+        M = O.window_mask(M, inp["win_lo"], inp["win_hi"])
     row_idx, seq_off, count = O.mask_compact(M)
     t0 = time.perf_counter()
     ref = O.rows_stats_chunked(Hb[row_idx[rows]], Wb)
@@ -176,7 +206,7 @@ def cpu_baseline(inp: dict, budget_s: float = 10.0) -> dict:
     """The oracle on a bounded sample of the workload's masked rows: the sample doubles until
     one run takes about budget_s (or covers every masked row); the last run is reported."""
     cfg = inp["cfg"]
-    count = int(inp["M"].sum())
+    count = rows_of_step(inp)
     rng = np.random.default_rng(0)
     n_rows = min(count, 32)
     while True:
@@ -196,7 +226,7 @@ def run_reference(args, cfg) -> None:
     if rank != 0:
         return
     inp = WL.make_inputs(cfg, seed=0)
-    count = int(inp["M"].sum())
+    count = rows_of_step(inp)
     rng = np.random.default_rng(0)
     t, n = oracle_rate(inp, np.sort(rng.choice(count, size=min(count, 8), replace=False)))
     per_row = t / n
@@ -219,6 +249,17 @@ def run_reference(args, cfg) -> None:
                                   sample=f"{rows_per_step} random masked rows per step of {cfg.name}"),
                 e2e=dict(value=value, unit=UNIT, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
     print(json.dumps(line), flush=True)
+
+
+def rows_of_step(inp: dict) -> int:
+    """Masked rows whose logits one step computes: all masked positions, or with
+    current-block-only logits those inside each sequence's window."""
+    M = inp["M"].numpy() != 0
+    if not inp["cfg"].block_only:
+        return int(M.sum())
+    pos = np.arange(M.shape[1])[None, :]
+    inside = (pos >= inp["win_lo"][:, None]) & (pos < inp["win_hi"][:, None])
+    return int((M & inside).sum())
 
 
 def workload_config(cfg, count: int) -> dict:
@@ -259,7 +300,8 @@ def main() -> None:
 
     # inputs (each rank its own seeded batch), and the oracle baseline before any GPU work
     inp = WL.make_inputs(cfg, seed=D.replica_seed(0, rank))
-    count = int(inp["M"].sum())
+    count = rows_of_step(inp)
+    blk = cfg.block_only
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(inp)
@@ -279,11 +321,13 @@ def main() -> None:
     stream = torch.cuda.current_stream(dev)
 
     for _ in range(args.warmup):
-        step.run(H, M, W, win_lo, win_hi, stream)
+        step.run(H, M, W, win_lo, win_hi, stream, blk)
     torch.cuda.synchronize(dev)
     status = dl.get_status(stream)
     if status != 0:
         raise RuntimeError(f"device status {status} after warm-up")
+    if int(step.count[0]) != count:
+        raise RuntimeError(f"the step computed {int(step.count[0])} rows, expected {count}")
     step_peak = torch.cuda.max_memory_allocated(dev) - base_mem
 
     def barrier():
@@ -297,7 +341,7 @@ def main() -> None:
         barrier()
         ev0.record(stream)
         for _ in range(args.steps):
-            step.run(H, M, W, win_lo, win_hi, stream)
+            step.run(H, M, W, win_lo, win_hi, stream, blk)
         ev1.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
@@ -308,7 +352,7 @@ def main() -> None:
     barrier()
     dl.prof_begin()
     for _ in range(args.steps):
-        step.run(H, M, W, win_lo, win_hi, stream)
+        step.run(H, M, W, win_lo, win_hi, stream, blk)
     torch.cuda.synchronize(dev)
     gemm_ms, gemm_launches, launches = dl.prof_end()
     status = dl.get_status(stream)
@@ -321,17 +365,19 @@ def main() -> None:
     H_host = inp["H"].pin_memory()
     M_host = inp["M"].pin_memory()
     for _ in range(3):
-        step.run_host(H_host, M_host, W, win_lo, win_hi, stream)
+        step.run_host(H_host, M_host, W, win_lo, win_hi, stream, blk)
     barrier()
     # the decode loop a serving process runs: each step's inputs copied in from pinned host
     # memory (overlapping the previous step) and its selection copied back
-    for _ in step.run_host_pipeline([(H_host, M_host)] * 3, W, win_lo, win_hi, stream):
+    for _ in step.run_host_pipeline([(H_host, M_host)] * 3, W, win_lo, win_hi, stream,
+                                    block_only=blk):
         pass
     torch.cuda.synchronize(dev)
     barrier()
     t0 = time.perf_counter()
     n_out = 0
-    for _ in step.run_host_pipeline([(H_host, M_host)] * e2e_steps, W, win_lo, win_hi, stream):
+    for _ in step.run_host_pipeline([(H_host, M_host)] * e2e_steps, W, win_lo, win_hi, stream,
+                                    block_only=blk):
         n_out += 1
     torch.cuda.synchronize(dev)
     e2e_ms = D.max_over_ranks([(time.perf_counter() - t0) * 1e3], dev)[0]
@@ -344,7 +390,6 @@ def main() -> None:
         ms_step = t_ms / args.steps
         rows_s = count * world * args.steps / (t_ms / 1e3)
         gemm_avg_s = gemm_ms / max(1, gemm_launches) / 1e3
-        tflops_gemm = a["flops"] / gemm_avg_s / 1e12
         roof = roofline_s(cfg, count, peaks)
         step_tflops = a["flops"] / (ms_step / 1e3) / 1e12
         step_gbs = a["bytes"] / (ms_step / 1e3) / 1e9
@@ -359,19 +404,7 @@ def main() -> None:
             tflops=step_tflops, gbs=step_gbs,
             roofline_frac_step=roof / (ms_step / 1e3),
             roofline_ms=roof * 1e3,
-            roofline=dict(bound="tensor" if a["flops"] / (peaks["bf16_tflops"] * 1e12) >=
-                          a["bytes"] / (peaks["hbm_gbs"] * 1e9) else "hbm",
-                          kernel=("masked_lmhead, paired-SM tcgen05 (lmhead_kernel<2, 0>)"
-                                  if paired else
-                                  "masked_lmhead, single-SM tcgen05 (lmhead_kernel<1, 0>)"),
-                          achieved=tflops_gemm, peak=peaks["bf16_tflops"], unit="TFLOP/s",
-                          frac=tflops_gemm / peaks["bf16_tflops"],
-                          frac_of_sustained=(tflops_gemm / peaks["bf16_tflops_sustained"]
-                                             if peaks.get("bf16_tflops_sustained") else None),
-                          peak_source=peaks["source"] + " (burst bf16 GEMM)",
-                          gemm_ms_avg=gemm_avg_s * 1e3,
-                          algorithmic_bytes=2.0 * cfg.V * cfg.d + 2.0 * count * cfg.d,
-                          traffic=measured_traffic(cfg.name, gemm_kernel_name)),
+            roofline=gemm_roofline(cfg, count, peaks, gemm_avg_s, paired, gemm_kernel_name),
             gpu_launches=launches,
             memory=dict(peak_step_bytes=int(step_peak),
                         full_logits_fp32_bytes=int(full_logits),

@@ -96,6 +96,22 @@ dllm_status dllm_mask_compact(const uint8_t* M, int32_t B, int32_t L,
                               void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * dllm_mask_compact_window - dllm_mask_compact restricted to one window per sequence: the
+ * compacted rows are the masked positions l of sequence b with win_lo[b] <= l < win_hi[b]
+ * (semi-autoregressive decoding works on the current block of each sequence only,
+ * Sparse-dLLM page, "Experiment").  row_idx, seq_off and count then describe those rows
+ * only.  Any window values are accepted (win_lo[b] >= win_hi[b] is an empty window).
+ *
+ *   win_lo, win_hi  device int32 [B], both non-NULL, or both NULL (= dllm_mask_compact).
+ * Other arguments, outputs and errors as in dllm_mask_compact; DLLM_ERR_NULL if exactly
+ * one window pointer is NULL.
+ */
+dllm_status dllm_mask_compact_window(const uint8_t* M, int32_t B, int32_t L,
+                                     const int32_t* win_lo, const int32_t* win_hi,
+                                     int32_t* row_idx, int32_t* seq_off, int32_t* count,
+                                     void* ws, size_t ws_bytes, void* stream);
+
+/*
  * dllm_mask_compact_noalloc - dllm_mask_compact without a workspace argument.
  *
  * The pages have no counterpart for this call; it exists for callers that cannot allocate
@@ -176,6 +192,24 @@ dllm_status dllm_masked_logits_ex(const uint16_t* H, const uint8_t* M, const uin
                                   int32_t* count, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * dllm_masked_logits_window - current-block-only logits: dllm_masked_logits_ex on the
+ * masked positions inside each sequence's window [win_lo[b], win_hi[b]) only (the rows of
+ * dllm_mask_compact_window).  Masked positions outside the window get no logits and no
+ * output row; they are decoded when their own block becomes current (Sparse-dLLM page,
+ * "Experiment": block-wise semi-autoregressive decoding).
+ *
+ *   win_lo, win_hi  device int32 [B], both required (DLLM_ERR_NULL otherwise).
+ * Other arguments, outputs and errors as in dllm_masked_logits_ex.
+ */
+dllm_status dllm_masked_logits_window(const uint16_t* H, const uint8_t* M, const uint16_t* W,
+                                      int32_t B, int32_t L, int32_t d, int32_t V,
+                                      const int32_t* win_lo, const int32_t* win_hi,
+                                      uint32_t stats, int32_t* tok, float* conf, float* lse,
+                                      float* entropy, float* margin, int32_t* row_idx,
+                                      int32_t* seq_off, int32_t* count, void* ws,
+                                      size_t ws_bytes, void* stream);
+
+/*
  * dllm_select_unmask - per-sequence top-k over confidences (confidence-driven unmasking,
  * dLLM inference survey page, "Main Findings").
  *
@@ -233,6 +267,22 @@ dllm_status dllm_decode_step(const uint16_t* H, const uint8_t* M, const uint16_t
                              int32_t* row_idx, int32_t* seq_off, int32_t* count,
                              int32_t* idx, int32_t* n_sel, int32_t* tok_sel, float* conf_sel,
                              void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * dllm_decode_block_step - one semi-autoregressive decode step over the current blocks:
+ * dllm_masked_logits_window followed by dllm_select_unmask, so logits are computed only
+ * for the masked positions inside each sequence's window.  The selection (idx, n_sel,
+ * tok_sel, conf_sel) equals that of dllm_decode_step with the same windows; tok, conf, lse,
+ * row_idx, seq_off and count cover the in-window rows only.  win_lo and win_hi are
+ * required.  Other arguments and errors as in dllm_decode_step.
+ */
+dllm_status dllm_decode_block_step(const uint16_t* H, const uint8_t* M, const uint16_t* W,
+                                   int32_t B, int32_t L, int32_t d, int32_t V, int32_t k,
+                                   const int32_t* win_lo, const int32_t* win_hi,
+                                   int32_t* tok, float* conf, float* lse,
+                                   int32_t* row_idx, int32_t* seq_off, int32_t* count,
+                                   int32_t* idx, int32_t* n_sel, int32_t* tok_sel,
+                                   float* conf_sel, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * dllm_get_status - synchronise `stream`, then return (and clear) the device-side status

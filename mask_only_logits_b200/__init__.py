@@ -78,14 +78,26 @@ def workspace_bytes(B: int, L: int, d: int, V: int) -> int:
     return int(lib().dllm_workspace_bytes(B, L, d, V))
 
 
-def mask_compact(M, row_idx, seq_off, count, ws, stream=None) -> None:
+def mask_compact(M, row_idx, seq_off, count, ws, stream=None, win_lo=None, win_hi=None) -> None:
+    """Compaction of the masked positions of M; with windows (device int32 [B] each), of
+    the masked positions l of sequence b with win_lo[b] <= l < win_hi[b] only."""
     B, L = M.shape
-    _check(lib().dllm_mask_compact(_ptr(M, torch.uint8, "M"), B, L,
-                                   _ptr(row_idx, torch.int32, "row_idx"),
-                                   _ptr(seq_off, torch.int32, "seq_off"),
-                                   _ptr(count, torch.int32, "count"), _ptr(ws, None, "ws"),
-                                   ws.numel() * ws.element_size(), _stream(stream)),
-           "dllm_mask_compact")
+    if win_lo is None and win_hi is None:
+        _check(lib().dllm_mask_compact(_ptr(M, torch.uint8, "M"), B, L,
+                                       _ptr(row_idx, torch.int32, "row_idx"),
+                                       _ptr(seq_off, torch.int32, "seq_off"),
+                                       _ptr(count, torch.int32, "count"), _ptr(ws, None, "ws"),
+                                       ws.numel() * ws.element_size(), _stream(stream)),
+               "dllm_mask_compact")
+        return
+    _check(lib().dllm_mask_compact_window(_ptr(M, torch.uint8, "M"), B, L,
+                                          _ptr(win_lo, torch.int32, "win_lo"),
+                                          _ptr(win_hi, torch.int32, "win_hi"),
+                                          _ptr(row_idx, torch.int32, "row_idx"),
+                                          _ptr(seq_off, torch.int32, "seq_off"),
+                                          _ptr(count, torch.int32, "count"), _ptr(ws, None, "ws"),
+                                          ws.numel() * ws.element_size(), _stream(stream)),
+           "dllm_mask_compact_window")
 
 
 def mask_compact_noalloc(M, row_idx, seq_off, count, stream=None) -> None:
@@ -113,19 +125,26 @@ def masked_logits(H, M, W, tok, conf, lse, row_idx, seq_off, count, ws, stream=N
 
 
 def masked_logits_ex(H, M, W, stats, tok, conf, lse, entropy, margin, row_idx, seq_off, count,
-                     ws, stream=None) -> None:
+                     ws, stream=None, win_lo=None, win_hi=None) -> None:
     """masked_logits plus the softmax entropy and/or top-2 probability margin per masked row
-    (stats: bitwise OR of STAT_ENTROPY and STAT_MARGIN; pass None for outputs not asked for)."""
+    (stats: bitwise OR of STAT_ENTROPY and STAT_MARGIN; pass None for outputs not asked for).
+    With windows (device int32 [B] each), only the masked rows inside each sequence's window
+    [win_lo[b], win_hi[b]) get logits (current-block-only decoding)."""
     B, L = M.shape
     V, d = W.shape
-    _check(lib().dllm_masked_logits_ex(
-        _ptr(H, torch.bfloat16, "H"), _ptr(M, torch.uint8, "M"), _ptr(W, torch.bfloat16, "W"),
-        B, L, d, V, stats, _ptr(tok, torch.int32, "tok"), _ptr(conf, torch.float32, "conf"),
-        _ptr(lse, torch.float32, "lse"), _ptr(entropy, torch.float32, "entropy"),
-        _ptr(margin, torch.float32, "margin"), _ptr(row_idx, torch.int32, "row_idx"),
-        _ptr(seq_off, torch.int32, "seq_off"), _ptr(count, torch.int32, "count"),
-        _ptr(ws, None, "ws"), ws.numel() * ws.element_size(), _stream(stream)),
-        "dllm_masked_logits_ex")
+    common = (_ptr(tok, torch.int32, "tok"), _ptr(conf, torch.float32, "conf"),
+              _ptr(lse, torch.float32, "lse"), _ptr(entropy, torch.float32, "entropy"),
+              _ptr(margin, torch.float32, "margin"), _ptr(row_idx, torch.int32, "row_idx"),
+              _ptr(seq_off, torch.int32, "seq_off"), _ptr(count, torch.int32, "count"),
+              _ptr(ws, None, "ws"), ws.numel() * ws.element_size(), _stream(stream))
+    ins = (_ptr(H, torch.bfloat16, "H"), _ptr(M, torch.uint8, "M"), _ptr(W, torch.bfloat16, "W"),
+           B, L, d, V)
+    if win_lo is None and win_hi is None:
+        _check(lib().dllm_masked_logits_ex(*ins, stats, *common), "dllm_masked_logits_ex")
+    else:
+        _check(lib().dllm_masked_logits_window(*ins, _ptr(win_lo, torch.int32, "win_lo"),
+                                               _ptr(win_hi, torch.int32, "win_hi"), stats,
+                                               *common), "dllm_masked_logits_window")
 
 
 def select_unmask_ex(score, row_idx, seq_off, B, L, k, threshold, min_sel, idx, n_sel,
@@ -155,10 +174,15 @@ def select_unmask(conf, row_idx, seq_off, B, L, k, idx, n_sel, win_lo=None, win_
 
 
 def decode_step(H, M, W, k, tok, conf, lse, row_idx, seq_off, count, idx, n_sel, ws,
-                win_lo=None, win_hi=None, tok_sel=None, conf_sel=None, stream=None) -> None:
+                win_lo=None, win_hi=None, tok_sel=None, conf_sel=None, stream=None,
+                block_only=False) -> None:
+    """The whole step.  With block_only=True (windows required) logits are computed for the
+    masked rows inside the windows only (dllm_decode_block_step); the selection is the same."""
     B, L = M.shape
     V, d = W.shape
-    _check(lib().dllm_decode_step(
+    fn, name = ((lib().dllm_decode_block_step, "dllm_decode_block_step") if block_only
+                else (lib().dllm_decode_step, "dllm_decode_step"))
+    _check(fn(
         _ptr(H, torch.bfloat16, "H"), _ptr(M, torch.uint8, "M"), _ptr(W, torch.bfloat16, "W"),
         B, L, d, V, k, _ptr(win_lo, torch.int32, "win_lo"), _ptr(win_hi, torch.int32, "win_hi"),
         _ptr(tok, torch.int32, "tok"), _ptr(conf, torch.float32, "conf"),
@@ -166,8 +190,7 @@ def decode_step(H, M, W, k, tok, conf, lse, row_idx, seq_off, count, idx, n_sel,
         _ptr(seq_off, torch.int32, "seq_off"), _ptr(count, torch.int32, "count"),
         _ptr(idx, torch.int32, "idx"), _ptr(n_sel, torch.int32, "n_sel"),
         _ptr(tok_sel, torch.int32, "tok_sel"), _ptr(conf_sel, torch.float32, "conf_sel"),
-        _ptr(ws, None, "ws"), ws.numel() * ws.element_size(), _stream(stream)),
-        "dllm_decode_step")
+        _ptr(ws, None, "ws"), ws.numel() * ws.element_size(), _stream(stream)), name)
 
 
 def get_status(stream=None) -> int:
@@ -243,10 +266,12 @@ class DecodeStep:
         self.ws = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
         self._host = None
 
-    def run(self, H, M, W, win_lo=None, win_hi=None, stream=None) -> dict:
+    def run(self, H, M, W, win_lo=None, win_hi=None, stream=None, block_only=False) -> dict:
+        """One step on device tensors.  block_only=True (windows required): logits for the
+        masked rows inside the windows only; tok/conf/lse/row_idx then cover those rows."""
         decode_step(H, M, W, self.k, self.tok, self.conf, self.lse, self.row_idx, self.seq_off,
                     self.count, self.idx, self.n_sel, self.ws, win_lo, win_hi, self.tok_sel,
-                    self.conf_sel, stream)
+                    self.conf_sel, stream, block_only)
         return dict(tok=self.tok, conf=self.conf, lse=self.lse, row_idx=self.row_idx,
                     seq_off=self.seq_off, count=self.count[:1], idx=self.idx, n_sel=self.n_sel,
                     tok_sel=self.tok_sel, conf_sel=self.conf_sel)
@@ -265,7 +290,8 @@ class DecodeStep:
                 conf_sel=torch.empty(B, k, dtype=torch.float32, **pin))
         return self._host
 
-    def run_host(self, H_host, M_host, W, win_lo=None, win_hi=None, stream=None) -> dict:
+    def run_host(self, H_host, M_host, W, win_lo=None, win_hi=None, stream=None,
+                 block_only=False) -> dict:
         """One step from pinned host H and M: copy them in, run, copy the selection back.
 
         W (the resident vocabulary projection) and the windows are device tensors.  Returns
@@ -276,7 +302,7 @@ class DecodeStep:
         with torch.cuda.stream(s):
             hb["H"].copy_(H_host, non_blocking=True)
             hb["M"].copy_(M_host, non_blocking=True)
-            self.run(hb["H"], hb["M"], W, win_lo, win_hi, s)
+            self.run(hb["H"], hb["M"], W, win_lo, win_hi, s, block_only)
             hb["idx"].copy_(self.idx, non_blocking=True)
             hb["n_sel"].copy_(self.n_sel, non_blocking=True)
             hb["tok_sel"].copy_(self.tok_sel, non_blocking=True)
@@ -285,7 +311,7 @@ class DecodeStep:
         return dict(idx=hb["idx"], n_sel=hb["n_sel"], tok_sel=hb["tok_sel"], conf_sel=hb["conf_sel"])
 
     def run_host_pipeline(self, batches, W, win_lo=None, win_hi=None, stream=None,
-                          copy_stream=None):
+                          copy_stream=None, block_only=False):
         """Decode steps over host batches [(H_host, M_host), ...] (pinned), with the copy of
         batch i+1 into the device overlapping the step of batch i.
 
@@ -333,7 +359,7 @@ class DecodeStep:
                 load(i + 1, *nxt)                    # overlaps step i below
             with torch.cuda.stream(s):
                 s.wait_event(loaded[b])
-                self.run(pb["H"][b], pb["M"][b], W, win_lo, win_hi, s)
+                self.run(pb["H"][b], pb["M"][b], W, win_lo, win_hi, s, block_only)
                 freed[b].record(s)
                 o = pb["out"][b]
                 o["idx"].copy_(self.idx, non_blocking=True)

@@ -18,16 +18,22 @@ PROTOTYPES = {
     "dllm_status_string": (ctypes.c_char_p, [_st]),
     "dllm_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32]),
     "dllm_mask_compact": (_st, [_p, _i32, _i32, _p, _p, _p, _p, _sz, _p]),
+    "dllm_mask_compact_window": (_st, [_p, _i32, _i32, _p, _p, _p, _p, _p, _p, _sz, _p]),
     "dllm_mask_compact_noalloc": (_st, [_p, _i32, _i32, _p, _p, _p, _p]),
     "dllm_masked_logits": (_st, [_p, _p, _p, _i32, _i32, _i32, _i32, _p, _p, _p, _p, _p, _p,
                                  _p, _sz, _p]),
     "dllm_masked_logits_ex": (_st, [_p, _p, _p, _i32, _i32, _i32, _i32, ctypes.c_uint32, _p, _p,
                                     _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
+    "dllm_masked_logits_window": (_st, [_p, _p, _p, _i32, _i32, _i32, _i32, _p, _p,
+                                        ctypes.c_uint32, _p, _p, _p, _p, _p, _p, _p, _p, _p, _sz,
+                                        _p]),
     "dllm_select_unmask": (_st, [_p, _p, _p, _i32, _i32, _i32, _p, _p, _p, _p, _p, _p, _p, _p]),
     "dllm_select_unmask_ex": (_st, [_p, _p, _p, _i32, _i32, _i32, ctypes.c_float, _i32, _i32, _p,
                                     _p, _p, _p, _p, _p, _p, _p]),
     "dllm_decode_step": (_st, [_p, _p, _p, _i32, _i32, _i32, _i32, _i32, _p, _p, _p, _p, _p,
                                _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
+    "dllm_decode_block_step": (_st, [_p, _p, _p, _i32, _i32, _i32, _i32, _i32, _p, _p, _p, _p,
+                                     _p, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
     "dllm_get_status": (_st, [_p]),
     "dllm_debug_lmhead_logits": (_st, [_p, _p, _p, _i32, _i32, _i32, _i32, _p, _p, _p, _p, _p,
                                        _sz, _p]),

@@ -4,6 +4,9 @@
 // The Mosaic page (TL;DR, Abstract) computes logits at masked positions only; compaction
 // turns the mask into the list of rows the LM head must see.
 //
+// Optional per-sequence windows [lo_b, hi_b) restrict the compaction to the masked positions
+// of each sequence's current block.
+//
 // Two launches, both over tiles of kCompactTile positions (one 16-byte vector per thread):
 //   compact_count_kernel    tile t -> number of nonzero mask bytes in the tile
 //   compact_scatter_kernel  tile t -> its offset (sum of earlier tiles' counts, reduced by
@@ -47,6 +50,31 @@ __device__ __forceinline__ uint32_t load_mask16(const uint8_t* __restrict__ M, l
   return bits;
 }
 
+// Keeps the bits of `bits` (positions p0 + j, all < n) whose position lies inside its
+// sequence's window: lo[b] <= l < hi[b] for position b * L + l.  Without windows (lo NULL)
+// every bit is kept.  Semi-autoregressive decoding works on one block of each sequence at
+// a time (Sparse-dLLM page, "Experiment"), so only the block's masked rows need logits.
+__device__ __forceinline__ uint32_t window_filter(uint32_t bits, long long p0, int L,
+                                                  const int* __restrict__ lo,
+                                                  const int* __restrict__ hi) {
+  if (lo == nullptr || bits == 0u) return bits;
+  long long b = p0 / L;
+  int l = static_cast<int>(p0 - b * L);
+  int wl = __ldg(lo + b), wh = __ldg(hi + b);
+  uint32_t keep = 0u;
+  const int last = 31 - __clz(static_cast<int>(bits));            // highest set bit
+  for (int j = 0; j <= last; ++j) {
+    if (l >= wl && l < wh) keep |= 1u << j;
+    if (++l == L && j < last) {          // position p0 + j + 1 <= p0 + last < n: b + 1 < B
+      l = 0;
+      ++b;
+      wl = __ldg(lo + b);
+      wh = __ldg(hi + b);
+    }
+  }
+  return bits & keep;
+}
+
 // Block-wide sum of one int per thread (blockDim.x == kCompactThreads).
 __device__ __forceinline__ int block_sum(int v, int* red) {
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -65,18 +93,20 @@ __device__ __forceinline__ int block_sum(int v, int* red) {
 }
 
 __global__ void __launch_bounds__(kCompactThreads)
-compact_count_kernel(const uint8_t* __restrict__ M, long long n, int* __restrict__ tile_count) {
+compact_count_kernel(const uint8_t* __restrict__ M, long long n, int L, const int* __restrict__ win_lo,
+                     const int* __restrict__ win_hi, int* __restrict__ tile_count) {
   __shared__ int red[33];
   pdl_wait();
   pdl_launch_dependents();
   const long long p0 = (static_cast<long long>(blockIdx.x) * kCompactThreads + threadIdx.x) * kCompactVec;
-  const int c = __popc(load_mask16(M, p0, n));
+  const int c = __popc(window_filter(load_mask16(M, p0, n), p0, L, win_lo, win_hi));
   const int total = block_sum(c, red);
   if (threadIdx.x == 0) tile_count[blockIdx.x] = total;
 }
 
 __global__ void __launch_bounds__(kCompactThreads)
-compact_scatter_kernel(const uint8_t* __restrict__ M, int B, int L, const int* __restrict__ tile_count,
+compact_scatter_kernel(const uint8_t* __restrict__ M, int B, int L, const int* __restrict__ win_lo,
+                       const int* __restrict__ win_hi, const int* __restrict__ tile_count,
                        int* __restrict__ row_idx, int* __restrict__ seq_off, int* __restrict__ count,
                        int* __restrict__ status) {
   __shared__ int red[33];
@@ -91,7 +121,7 @@ compact_scatter_kernel(const uint8_t* __restrict__ M, int B, int L, const int* _
   const int tile_base = block_sum(part, red);
 
   const long long p0 = (static_cast<long long>(t) * kCompactThreads + threadIdx.x) * kCompactVec;
-  const uint32_t bits = load_mask16(M, p0, n);
+  const uint32_t bits = window_filter(load_mask16(M, p0, n), p0, L, win_lo, win_hi);
   const int c = __popc(bits);
   // block-wide exclusive scan of c
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;

@@ -205,18 +205,20 @@ bool shapes_ok(int B, int L) {
   return B >= 1 && L >= 1 && static_cast<long long>(B) * L < (1ll << 31);
 }
 
-dllm_status launch_compact(const uint8_t* M, int B, int L, int* row_idx, int* seq_off, int* count,
-                           int* tiles, int* status, cudaStream_t s) {
+dllm_status launch_compact(const uint8_t* M, int B, int L, const int* win_lo, const int* win_hi,
+                           int* row_idx, int* seq_off, int* count, int* tiles, int* status,
+                           cudaStream_t s) {
   const long long n = static_cast<long long>(B) * L;
   const unsigned ntiles = static_cast<unsigned>((n + kCompactTile - 1) / kCompactTile);
   // a single tile needs no per-tile counts: its offset is 0
   if (ntiles > 1) {
-    if (launch_pdl(compact_count_kernel, dim3(ntiles), dim3(kCompactThreads), 0, s, M, n, tiles) != cudaSuccess)
+    if (launch_pdl(compact_count_kernel, dim3(ntiles), dim3(kCompactThreads), 0, s, M, n, L, win_lo,
+                   win_hi, tiles) != cudaSuccess)
       return DLLM_ERR_CUDA;
     count_launch();
   }
-  if (launch_pdl(compact_scatter_kernel, dim3(ntiles), dim3(kCompactThreads), 0, s, M, B, L,
-                 (const int*)tiles, row_idx, seq_off, count, status) != cudaSuccess)
+  if (launch_pdl(compact_scatter_kernel, dim3(ntiles), dim3(kCompactThreads), 0, s, M, B, L, win_lo,
+                 win_hi, (const int*)tiles, row_idx, seq_off, count, status) != cudaSuccess)
     return DLLM_ERR_CUDA;
   count_launch();
   return DLLM_OK;
@@ -237,6 +239,7 @@ dllm_status make_tmap(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t
 struct LogitsArgs {
   const uint16_t* H; const uint8_t* M; const uint16_t* W;
   int B, L, d, V;
+  const int* win_lo; const int* win_hi;          // rows restricted to windows, or both NULL
   uint32_t stats; float* entropy; float* margin;
   int* tok; float* conf; float* lse; float* dbg;
   int* row_idx; int* seq_off; int* count;
@@ -247,13 +250,14 @@ dllm_status validate_logits(const LogitsArgs& a, bool debug) {
   if (!a.H || !a.M || !a.W || !a.row_idx || !a.seq_off || !a.count || !a.ws) return DLLM_ERR_NULL;
   if (!debug && (!a.tok || !a.conf || !a.lse)) return DLLM_ERR_NULL;
   if (debug && !a.dbg) return DLLM_ERR_NULL;
+  if ((a.win_lo == nullptr) != (a.win_hi == nullptr)) return DLLM_ERR_NULL;
   if ((a.stats & ~(DLLM_STAT_ENTROPY | DLLM_STAT_MARGIN)) != 0) return DLLM_ERR_SHAPE;
   if (((a.stats & DLLM_STAT_ENTROPY) != 0) != (a.entropy != nullptr)) return DLLM_ERR_NULL;
   if (((a.stats & DLLM_STAT_MARGIN) != 0) != (a.margin != nullptr)) return DLLM_ERR_NULL;
   if (!shapes_ok(a.B, a.L) || a.V < 1 || a.d < DLLM_D_MULTIPLE || a.d % DLLM_D_MULTIPLE != 0)
     return DLLM_ERR_SHAPE;
   const void* ptrs[] = {a.H, a.M, a.W, a.row_idx, a.seq_off, a.count, a.ws, a.tok, a.conf, a.lse,
-                        a.dbg, a.entropy, a.margin};
+                        a.dbg, a.entropy, a.margin, a.win_lo, a.win_hi};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return DLLM_ERR_ALIGN;
   if (a.ws_bytes < ws_layout(a.B, a.L, a.d, a.V).total) return DLLM_ERR_WORKSPACE;
@@ -299,7 +303,8 @@ dllm_status run_logits(const LogitsArgs& a, bool debug) {
     if (need > w.part_cap) return DLLM_ERR_WORKSPACE;                  // cannot happen on B200
   }
 
-  if ((st = launch_compact(a.M, a.B, a.L, a.row_idx, a.seq_off, a.count, tiles, ds->status, a.s)) != DLLM_OK)
+  if ((st = launch_compact(a.M, a.B, a.L, a.win_lo, a.win_hi, a.row_idx, a.seq_off, a.count, tiles,
+                           ds->status, a.s)) != DLLM_OK)
     return st;
 
   if (launch_pdl(gather_rows_kernel, dim3(ds->sms * 4), dim3(kGatherThreads), 0, a.s, a.H,
@@ -433,11 +438,11 @@ dllm_status dllm_mask_compact_noalloc(const uint8_t* M, int32_t B, int32_t L, in
   if (st != DLLM_OK) return st;
   int* tiles = nullptr;
   if ((st = noalloc_scratch(&tiles)) != DLLM_OK) return st;
-  return launch_compact(M, B, L, row_idx, seq_off, count, tiles, ds->status,
+  return launch_compact(M, B, L, nullptr, nullptr, row_idx, seq_off, count, tiles, ds->status,
                         static_cast<cudaStream_t>(stream));
 }
 
-int32_t dllm_version(void) { return 10000; }
+int32_t dllm_version(void) { return 10100; }
 
 const char* dllm_status_string(dllm_status s) {
   switch (s) {
@@ -460,29 +465,38 @@ size_t dllm_workspace_bytes(int32_t B, int32_t L, int32_t d, int32_t V) {
   return ws_layout(B, L, d, V).total;
 }
 
-dllm_status dllm_mask_compact(const uint8_t* M, int32_t B, int32_t L, int32_t* row_idx,
-                              int32_t* seq_off, int32_t* count, void* ws, size_t ws_bytes,
-                              void* stream) {
+dllm_status dllm_mask_compact_window(const uint8_t* M, int32_t B, int32_t L, const int32_t* win_lo,
+                                     const int32_t* win_hi, int32_t* row_idx, int32_t* seq_off,
+                                     int32_t* count, void* ws, size_t ws_bytes, void* stream) {
   if (!M || !row_idx || !seq_off || !count || !ws) return DLLM_ERR_NULL;
+  if ((win_lo == nullptr) != (win_hi == nullptr)) return DLLM_ERR_NULL;
   if (!shapes_ok(B, L)) return DLLM_ERR_SHAPE;
   if (!aligned16(M) || !aligned16(row_idx) || !aligned16(seq_off) || !aligned16(count) || !aligned16(ws))
     return DLLM_ERR_ALIGN;
+  if ((win_lo && !aligned16(win_lo)) || (win_hi && !aligned16(win_hi))) return DLLM_ERR_ALIGN;
   const long long n = static_cast<long long>(B) * L;
   const size_t need = sizeof(int) * static_cast<size_t>((n + kCompactTile - 1) / kCompactTile);
   if (ws_bytes < need) return DLLM_ERR_WORKSPACE;
   DeviceState* ds = nullptr;
   dllm_status st = device_state(&ds);
   if (st != DLLM_OK) return st;
-  return launch_compact(M, B, L, row_idx, seq_off, count, static_cast<int*>(ws), ds->status,
-                        static_cast<cudaStream_t>(stream));
+  return launch_compact(M, B, L, win_lo, win_hi, row_idx, seq_off, count, static_cast<int*>(ws),
+                        ds->status, static_cast<cudaStream_t>(stream));
+}
+
+dllm_status dllm_mask_compact(const uint8_t* M, int32_t B, int32_t L, int32_t* row_idx,
+                              int32_t* seq_off, int32_t* count, void* ws, size_t ws_bytes,
+                              void* stream) {
+  return dllm_mask_compact_window(M, B, L, nullptr, nullptr, row_idx, seq_off, count, ws, ws_bytes,
+                                  stream);
 }
 
 dllm_status dllm_masked_logits(const uint16_t* H, const uint8_t* M, const uint16_t* W, int32_t B,
                                int32_t L, int32_t d, int32_t V, int32_t* tok, float* conf,
                                float* lse, int32_t* row_idx, int32_t* seq_off, int32_t* count,
                                void* ws, size_t ws_bytes, void* stream) {
-  LogitsArgs a{H, M, W, B, L, d, V, 0u, nullptr, nullptr, tok, conf, lse, nullptr, row_idx, seq_off,
-               count, ws, ws_bytes, static_cast<cudaStream_t>(stream)};
+  LogitsArgs a{H, M, W, B, L, d, V, nullptr, nullptr, 0u, nullptr, nullptr, tok, conf, lse, nullptr,
+               row_idx, seq_off, count, ws, ws_bytes, static_cast<cudaStream_t>(stream)};
   return run_logits(a, false);
 }
 
@@ -491,8 +505,20 @@ dllm_status dllm_masked_logits_ex(const uint16_t* H, const uint8_t* M, const uin
                                   float* conf, float* lse, float* entropy, float* margin,
                                   int32_t* row_idx, int32_t* seq_off, int32_t* count, void* ws,
                                   size_t ws_bytes, void* stream) {
-  LogitsArgs a{H, M, W, B, L, d, V, stats, entropy, margin, tok, conf, lse, nullptr, row_idx,
-               seq_off, count, ws, ws_bytes, static_cast<cudaStream_t>(stream)};
+  LogitsArgs a{H, M, W, B, L, d, V, nullptr, nullptr, stats, entropy, margin, tok, conf, lse, nullptr,
+               row_idx, seq_off, count, ws, ws_bytes, static_cast<cudaStream_t>(stream)};
+  return run_logits(a, false);
+}
+
+dllm_status dllm_masked_logits_window(const uint16_t* H, const uint8_t* M, const uint16_t* W,
+                                      int32_t B, int32_t L, int32_t d, int32_t V,
+                                      const int32_t* win_lo, const int32_t* win_hi, uint32_t stats,
+                                      int32_t* tok, float* conf, float* lse, float* entropy,
+                                      float* margin, int32_t* row_idx, int32_t* seq_off,
+                                      int32_t* count, void* ws, size_t ws_bytes, void* stream) {
+  if (!win_lo || !win_hi) return DLLM_ERR_NULL;
+  LogitsArgs a{H, M, W, B, L, d, V, win_lo, win_hi, stats, entropy, margin, tok, conf, lse, nullptr,
+               row_idx, seq_off, count, ws, ws_bytes, static_cast<cudaStream_t>(stream)};
   return run_logits(a, false);
 }
 
@@ -500,8 +526,8 @@ dllm_status dllm_debug_lmhead_logits(const uint16_t* H, const uint8_t* M, const 
                                      int32_t B, int32_t L, int32_t d, int32_t V, float* logits_out,
                                      int32_t* row_idx, int32_t* seq_off, int32_t* count, void* ws,
                                      size_t ws_bytes, void* stream) {
-  LogitsArgs a{H, M, W, B, L, d, V, 0u, nullptr, nullptr, nullptr, nullptr, nullptr, logits_out,
-               row_idx, seq_off, count, ws, ws_bytes, static_cast<cudaStream_t>(stream)};
+  LogitsArgs a{H, M, W, B, L, d, V, nullptr, nullptr, 0u, nullptr, nullptr, nullptr, nullptr, nullptr,
+               logits_out, row_idx, seq_off, count, ws, ws_bytes, static_cast<cudaStream_t>(stream)};
   return run_logits(a, true);
 }
 
@@ -570,6 +596,26 @@ dllm_status dllm_decode_step(const uint16_t* H, const uint8_t* M, const uint16_t
                                       ws, ws_bytes, stream);
   if (st != DLLM_OK) return st;
   return dllm_select_unmask(conf, row_idx, seq_off, B, L, k, win_lo, win_hi, tok, idx, n_sel,
+                            tok_sel, conf_sel, stream);
+}
+
+dllm_status dllm_decode_block_step(const uint16_t* H, const uint8_t* M, const uint16_t* W, int32_t B,
+                                   int32_t L, int32_t d, int32_t V, int32_t k, const int32_t* win_lo,
+                                   const int32_t* win_hi, int32_t* tok, float* conf, float* lse,
+                                   int32_t* row_idx, int32_t* seq_off, int32_t* count, int32_t* idx,
+                                   int32_t* n_sel, int32_t* tok_sel, float* conf_sel, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  if (!idx || !n_sel || !win_lo || !win_hi) return DLLM_ERR_NULL;
+  if (k < 1 || k > DLLM_MAX_K) return DLLM_ERR_SHAPE;
+  const void* ptrs[] = {idx, n_sel, tok_sel, conf_sel};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return DLLM_ERR_ALIGN;
+  dllm_status st = dllm_masked_logits_window(H, M, W, B, L, d, V, win_lo, win_hi, 0u, tok, conf, lse,
+                                             nullptr, nullptr, row_idx, seq_off, count, ws, ws_bytes,
+                                             stream);
+  if (st != DLLM_OK) return st;
+  // every compacted row already lies in its window: no window test is needed in the selection
+  return dllm_select_unmask(conf, row_idx, seq_off, B, L, k, nullptr, nullptr, tok, idx, n_sel,
                             tok_sel, conf_sel, stream);
 }
 

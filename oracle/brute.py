@@ -28,6 +28,18 @@ def compact(mask_rows):
     return row_idx, seq_off
 
 
+def compact_window(mask_rows, win_lo, win_hi):
+    """Like ``compact`` but only positions l of sequence b with win_lo[b] <= l < win_hi[b]."""
+    row_idx, seq_off = [], [0]
+    L = len(mask_rows[0]) if mask_rows else 0
+    for b, row in enumerate(mask_rows):
+        for l, v in enumerate(row):
+            if v and win_lo[b] <= l < win_hi[b]:
+                row_idx.append(b * L + l)
+        seq_off.append(len(row_idx))
+    return row_idx, seq_off
+
+
 def dot(h, w):
     """Correctly rounded dot product of two float lists (math.fsum of exact products)."""
     return math.fsum(a * b for a, b in zip(h, w))

@@ -61,6 +61,18 @@ def mask_compact(M: np.ndarray):
     return row_idx, seq_off, int(row_idx.size)
 
 
+def window_mask(M: np.ndarray, win_lo, win_hi) -> np.ndarray:
+    """M restricted to the current block of each sequence: position l of sequence b stays
+    masked only if win_lo[b] <= l < win_hi[b].  Block-wise (semi-autoregressive) decoding
+    only ever unmasks positions of the current block (Sparse-dLLM page, "Experiment"), so
+    these are the only rows whose logits a block step needs."""
+    M = np.asarray(M)
+    l = np.arange(M.shape[1], dtype=np.int64)[None, :]
+    lo = np.asarray(win_lo, dtype=np.int64)[:, None]
+    hi = np.asarray(win_hi, dtype=np.int64)[:, None]
+    return ((M != 0) & (l >= lo) & (l < hi)).astype(np.uint8)
+
+
 # --------------------------------------------------------------------------------------
 # logits and per-row statistics
 # --------------------------------------------------------------------------------------
@@ -262,6 +274,12 @@ def oracle_step(H_bits, W_bits, M, k, win_lo=None, win_hi=None):
                                win_lo, win_hi)
     out.update(idx=idx, n_sel=n_sel)
     return out
+
+
+def oracle_block_step(H_bits, W_bits, M, k, win_lo, win_hi):
+    """A decode step with current-block-only logits: statistics for the masked rows inside
+    the windows only, then the same windowed selection as ``oracle_step``."""
+    return oracle_step(H_bits, W_bits, window_mask(M, win_lo, win_hi), k, win_lo, win_hi)
 
 
 def full_then_gather(H_bits, W_bits, M):

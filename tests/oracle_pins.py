@@ -286,7 +286,38 @@ def check_threshold_select(o):
             assert np.array_equal(t_idx, idx) and np.array_equal(t_n, n_sel)
 
 
+def check_block_step(o):
+    """Current-block-only logits: the windowed mask equals brute-force windowed compaction
+    (including empty, inverted and out-of-range windows), and the block step selects exactly
+    what the full step selects with the same windows, with per-row statistics equal to the
+    full step's rows at the same positions."""
+    rng = np.random.default_rng(21)
+    for case in range(10):
+        B, L = int(rng.integers(1, 4)), int(rng.integers(1, 40))
+        M = (rng.random((B, L)) < 0.6).astype(np.uint8)
+        lo = rng.integers(-3, L + 2, size=B)
+        hi = lo + rng.integers(-2, L + 3, size=B)
+        if case == 0:                                          # window edges on masked cells
+            M[:] = 1
+            lo[:] = 1
+            hi[:] = max(2, L - 1)
+        Mw = o.window_mask(M, lo, hi)
+        r1, s1, c1 = o.mask_compact(Mw)
+        r2, s2 = brute.compact_window(M.tolist(), lo.tolist(), hi.tolist())
+        assert r1.tolist() == r2 and s1.tolist() == s2 and c1 == len(r2), (M, lo, hi)
+        d, V, k = int(rng.integers(1, 6)), int(rng.integers(1, 20)), int(rng.integers(1, 5))
+        H, W = _rand_bits(rng, (B * L, d)), _rand_bits(rng, (V, d), 0.5)
+        blk = o.oracle_block_step(H, W, M, k, lo, hi)
+        full = o.oracle_step(H, W, M, k, lo, hi)
+        assert np.array_equal(blk["idx"], full["idx"]) and np.array_equal(blk["n_sel"], full["n_sel"])
+        where = {int(p): i for i, p in enumerate(full["row_idx"])}
+        sel = [where[int(p)] for p in blk["row_idx"]]
+        for key in ("tok", "m", "lse", "conf"):
+            assert np.array_equal(blk[key], np.asarray(full[key])[sel]), key
+
+
 ALL_CHECKS = [check_handworked, check_topk_ties, check_compact, check_brute_random,
               check_closed_forms, check_library_routines, check_invariants,
               check_mask_only_equals_full, check_merge_split_invariance,
-              check_policy_closed_forms, check_policy_library_and_brute, check_threshold_select]
+              check_policy_closed_forms, check_policy_library_and_brute, check_threshold_select,
+              check_block_step]

@@ -38,7 +38,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.dllm_version() == 10000
+    assert lib.dllm_version() == 10100
     for code in (0, -1, -2, -3, -4, -5, -6, -7, -8):
         assert lib.dllm_status_string(code)
     assert lib.dllm_status_string(-99) == b"unknown status"
@@ -98,3 +98,28 @@ def test_host_validation_without_gpu(lib):
     # merge hook
     assert lib.dllm_debug_lse_merge(nul, _p(a), _p(a), 4, 2, _p(a), _p(a), _p(a), nul) == -1
     assert lib.dllm_debug_lse_merge(_p(a), _p(a), _p(a), 0, 2, _p(a), _p(a), _p(a), nul) == -3
+
+
+def test_window_entry_points_validate_on_host(lib):
+    a = 1 << 20
+    nul = _p(None)
+    # compaction: exactly one window pointer given, or a misaligned one
+    assert lib.dllm_mask_compact_window(_p(a), 1, 8, _p(a), nul, _p(a), _p(a), _p(a), _p(a),
+                                        1 << 20, nul) == -1
+    assert lib.dllm_mask_compact_window(_p(a), 1, 8, _p(a), _p(a + 4), _p(a), _p(a), _p(a), _p(a),
+                                        1 << 20, nul) == -2
+    assert lib.dllm_mask_compact_window(_p(a), 0, 8, _p(a), _p(a), _p(a), _p(a), _p(a), _p(a),
+                                        1 << 20, nul) == -3
+    # current-block-only logits: windows are required
+    ins = [_p(a), _p(a), _p(a), 1, 256, 256, 4096]
+    outs = [_p(a), _p(a), _p(a), nul, nul, _p(a), _p(a), _p(a), _p(a), 1 << 30, nul]
+    assert lib.dllm_masked_logits_window(*ins, nul, nul, 0, *outs) == -1
+    assert lib.dllm_masked_logits_window(*ins, _p(a), nul, 0, *outs) == -1
+    assert lib.dllm_masked_logits_window(*ins, _p(a), _p(a), 4, *outs) == -3      # unknown stat
+    small_ws = outs[:-2] + [10, nul]
+    assert lib.dllm_masked_logits_window(*ins, _p(a), _p(a), 0, *small_ws) == -4
+    # block step: windows required, k checked before any launch
+    assert lib.dllm_decode_block_step(*ins, 4, nul, nul, *[_p(a)] * 6, _p(a), _p(a), nul, nul,
+                                      _p(a), 1 << 30, nul) == -1
+    assert lib.dllm_decode_block_step(*ins, 0, _p(a), _p(a), *[_p(a)] * 6, _p(a), _p(a), nul, nul,
+                                      _p(a), 1 << 30, nul) == -3

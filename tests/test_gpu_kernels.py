@@ -58,6 +58,49 @@ def test_compact_nonbinary_and_workload_masks(dl):
         _compact_case(dl, WL.make_mask(cfg, g).numpy())
 
 
+def _compact_window_case(dl, M_np, lo, hi):
+    B, L = M_np.shape
+    n = B * L
+    row_idx = torch.full((n,), -7, dtype=torch.int32, device="cuda")
+    seq_off = torch.full((B + 1,), -7, dtype=torch.int32, device="cuda")
+    count = torch.full((4,), -7, dtype=torch.int32, device="cuda")
+    ws = torch.empty(dl.workspace_bytes(B, L, 64, 1), dtype=torch.uint8, device="cuda")
+    dl.mask_compact(torch.from_numpy(M_np).cuda(), row_idx, seq_off, count, ws,
+                    win_lo=torch.from_numpy(lo.astype(np.int32)).cuda(),
+                    win_hi=torch.from_numpy(hi.astype(np.int32)).cuda())
+    assert dl.get_status() == 0
+    r_ref, s_ref, c_ref = O.mask_compact(O.window_mask(M_np, lo, hi))
+    c = int(count[0])
+    assert c == c_ref
+    np.testing.assert_array_equal(row_idx[:c].cpu().numpy(), r_ref)
+    np.testing.assert_array_equal(seq_off.cpu().numpy(), s_ref)
+    assert bool((row_idx[c:] == -7).all())
+
+
+@pytest.mark.parametrize("B,L,p", [(1, 256, 0.5), (8, 8192, 1.0), (3, 1000, 0.5), (7, 3, 0.6),
+                                   (5, 1, 1.0), (2, 8191, 0.3), (37, 1111, 0.5), (1, 131072, 0.9),
+                                   (64, 17, 0.8)])
+def test_compact_windows_bit_exact(dl, B, L, p):
+    """Current-block-only compaction: windows of random placement and width, including
+    empty, inverted, negative and past-the-end ones, and sequences shorter than a vector."""
+    rng = np.random.default_rng(B * 31 + L)
+    M = (rng.random((B, L)) < p).astype(np.uint8)
+    lo = rng.integers(-5, L + 3, size=B)
+    hi = lo + rng.integers(-3, max(2, L // 3), size=B)
+    _compact_window_case(dl, M, lo, hi)
+    # every window the whole sequence / no window at all / one position
+    _compact_window_case(dl, M, np.zeros(B, np.int64), np.full(B, L))
+    _compact_window_case(dl, M, np.full(B, L), np.full(B, L + 5))
+    _compact_window_case(dl, M, np.full(B, L - 1), np.full(B, L))
+
+
+def test_compact_windows_semi_ar(dl):
+    cfg = WL.CONFIGS["cfg4"]
+    M = WL.make_mask(cfg).numpy()
+    lo, hi = WL.make_windows(cfg)
+    _compact_window_case(dl, M, lo, hi)
+
+
 # ------------------------------------------------------------------- tensor-core GEMM logits
 def _rand_bf16(rng, shape, std):
     return torch.from_numpy((rng.standard_normal(shape) * std).astype(np.float32)).to(torch.bfloat16)

@@ -30,7 +30,8 @@ def run_gpu(dl, inp):
     cfg = inp["cfg"]
     dev = GU.to_device(inp)
     step = dl.DecodeStep(cfg.B, cfg.L, cfg.d, cfg.V, inp["k"])
-    out = step.run(dev["H"], dev["M"], dev["W"], dev["win_lo"], dev["win_hi"])
+    out = step.run(dev["H"], dev["M"], dev["W"], dev["win_lo"], dev["win_hi"],
+                   block_only=cfg.block_only)
     assert dl.get_status() == 0
     c = int(out["count"][0])
     res = {key: out[key].cpu().numpy() for key in ("tok", "conf", "lse", "row_idx", "seq_off",
@@ -46,6 +47,8 @@ def run_gpu(dl, inp):
 def check_step(dl, inp, all_rows: bool, window_rows: bool = False):
     cfg = inp["cfg"]
     Hb, Wb, M = GU.inputs_bits(inp)
+    if cfg.block_only:             # current-block-only logits: the rows inside the windows
+        M = O.window_mask(M, inp["win_lo"], inp["win_hi"])
     g = run_gpu(dl, inp)
     # compaction: bit-exact
     row_idx, seq_off, count = O.mask_compact(M)
@@ -132,6 +135,28 @@ def test_cfg3_sweep_sampled(dl):
 
 def test_cfg4_sampled_and_windows(dl):
     check_step(dl, WL.make_inputs(WL.CONFIGS["cfg4"], seed=0), all_rows=False, window_rows=True)
+
+
+def test_cfg4_block_every_row(dl):
+    """Current-block-only logits (dllm_decode_block_step) on cfg4: every in-window row
+    against the oracle, and the same selection as the oracle's full windowed step."""
+    inp = WL.make_inputs(WL.CONFIGS["cfg4_block"], seed=0)
+    g, _ = check_step(dl, inp, all_rows=True)
+    assert g["count"] == 8 * 32
+
+
+@pytest.mark.parametrize("B,L,d,V,k,r", [(3, 1000, 128, 777, 5, 0.7), (5, 64, 64, 300, 40, 1.0),
+                                         (2, 20000, 256, 4096, 16, 0.5)])
+def test_block_only_random_windows(dl, B, L, d, V, k, r):
+    """Block-only steps with windows of random placement and width (empty, inverted and
+    out-of-range ones included) over Bernoulli masks."""
+    inp = WL.make_inputs(WL.custom_config(B, L, d, V, k, r=r, block_only=True), seed=7)
+    rng = np.random.default_rng(B + L)
+    lo = rng.integers(-4, L, size=B)
+    hi = lo + rng.integers(-2, max(3, L // 2), size=B)
+    hi[0] = lo[0]                                           # one empty window
+    inp["win_lo"], inp["win_hi"] = lo.astype(np.int32), hi.astype(np.int32)
+    check_step(dl, inp, all_rows=True)
 
 
 @pytest.mark.parametrize("B,L,d,V,k,mask,r", [

@@ -32,7 +32,7 @@ def variant(request, dl):
     dl.debug_set_gemm_variant(0)
 
 
-def _run_ex(dl, inp, stats):
+def _run_ex(dl, inp, stats, win=None):
     cfg = inp["cfg"]
     n = cfg.B * cfg.L
     dev = dict(H=inp["H"].cuda(), M=inp["M"].cuda(), W=inp["W"].cuda())
@@ -43,8 +43,12 @@ def _run_ex(dl, inp, stats):
     mar = torch.empty(n, **f32) if stats & dl.STAT_MARGIN else None
     row_idx, seq_off, count = torch.empty(n, **i32), torch.empty(cfg.B + 1, **i32), torch.empty(4, **i32)
     ws = torch.empty(dl.workspace_bytes(cfg.B, cfg.L, cfg.d, cfg.V), dtype=torch.uint8, device="cuda")
+    lo = hi = None
+    if win is not None:
+        lo = torch.from_numpy(np.asarray(win[0], dtype=np.int32)).cuda()
+        hi = torch.from_numpy(np.asarray(win[1], dtype=np.int32)).cuda()
     dl.masked_logits_ex(dev["H"], dev["M"], dev["W"], stats, tok, conf, lse, ent, mar, row_idx,
-                        seq_off, count, ws)
+                        seq_off, count, ws, win_lo=lo, win_hi=hi)
     assert dl.get_status() == 0
     c = int(count[0])
     out = dict(count=c, tok=tok[:c].cpu().numpy(), conf=conf[:c].cpu().numpy(),
@@ -92,6 +96,20 @@ def test_entropy_margin_cfg1_every_row(dl):
     Hb, Wb, M = WL.bf16_bits(inp["H"]), WL.bf16_bits(inp["W"]), inp["M"].numpy()
     rows = np.arange(g["count"])
     _check_policy(g, O.oracle_rows(Hb, Wb, M, rows), rows)
+
+
+def test_entropy_margin_current_block_only(dl, variant):
+    """dllm_masked_logits_window: statistics for the masked rows inside the windows only."""
+    inp = WL.make_inputs(WL.custom_config(4, 3000, 128, 5000, 4, r=0.8), seed=6)
+    lo = np.array([0, 100, 2990, 1500])
+    hi = np.array([32, 164, 3100, 1200])                       # the last window is empty
+    g = _run_ex(dl, inp, dl.STAT_ENTROPY | dl.STAT_MARGIN, (lo, hi))
+    Mw = O.window_mask(inp["M"].numpy(), lo, hi)
+    ref = O.oracle_rows(WL.bf16_bits(inp["H"]), WL.bf16_bits(inp["W"]), Mw)
+    assert g["count"] == ref["count"]
+    np.testing.assert_array_equal(g["row_idx"], ref["row_idx"])
+    np.testing.assert_array_equal(g["seq_off"], ref["seq_off"])
+    _check_policy(g, ref, np.arange(g["count"]))
 
 
 def test_margin_exact_ties_and_single_flags(dl):

@@ -157,7 +157,23 @@ def _threshold_strict(score, row_idx, seq_off, L, k, threshold, min_sel=1, win_l
     return idx, n_sel
 
 
+def _window_mask_closed(M, win_lo, win_hi):
+    M = np.asarray(M)
+    l = np.arange(M.shape[1])[None, :]
+    inside = (l >= np.asarray(win_lo)[:, None]) & (l <= np.asarray(win_hi)[:, None])   # closed
+    return ((M != 0) & inside).astype(np.uint8)
+
+
+def _window_mask_ignores_seq(M, win_lo, win_hi):
+    M = np.asarray(M)
+    l = np.arange(M.shape[1])[None, :]
+    inside = (l >= int(np.asarray(win_lo)[0])) & (l < int(np.asarray(win_hi)[0]))  # seq 0's window
+    return ((M != 0) & inside).astype(np.uint8)
+
+
 MUTATIONS = {
+    "block_window_closed": ("window_mask", _window_mask_closed),
+    "block_window_first_seq_only": ("window_mask", _window_mask_ignores_seq),
     "entropy_log2": ("row_policy_stats", _policy_entropy_log2),
     "margin_of_logits": ("row_policy_stats", _policy_margin_of_logits),
     "threshold_strict": ("select_unmask_threshold", _threshold_strict),

@@ -19,6 +19,8 @@ Taming", Abstract and Fig. 3 (128k context, mask-ratio sweep), and the Sparse-dL
   cfg4   B=8 L=8192   d=2048 V=151936  semi-autoregressive blocks of 32: sequence b's
          current block is block 32*b+16; it and every later position are masked, earlier
          ones are not; unmask candidates are the positions of the current block; k=4
+  cfg4_block  cfg4 with logits for the current block's masked rows only (Sparse-dLLM
+         page, "Experiment": block-wise decoding needs the current block only)
 
 Random draws, in this order, from one ``torch.Generator`` (CPU) seeded with ``seed``:
 W ~ N(0, 0.02^2) [V, d] in fp32, then H ~ N(0, 1) [B*L, d] in fp32, then for Bernoulli
@@ -47,6 +49,7 @@ class Config:
     r: float = 0.0       # Bernoulli mask ratio
     n_suffix: int = 0    # masked suffix length ("suffix")
     block: int = 32      # semi-autoregressive block length ("semi_ar")
+    block_only: bool = False   # logits for the masked rows of the current block only
     w_std: float = 0.02
     h_std: float = 1.0
     description: str = ""
@@ -71,6 +74,12 @@ CONFIGS: dict[str, Config] = {
     "cfg4": Config("cfg4", B=8, L=8192, d=2048, V=151936, k=4, mask="semi_ar", block=32,
                    description="B8 L8192 d2048 V151936, 32-token blocks, current block "
                                "32b+16 and later masked, window = current block, k=4"),
+    # cfg4 decoded block-wise with current-block-only logits: 8 x 32 rows (few rows, so
+    # streaming W from HBM and the tensor cores bound the step about equally)
+    "cfg4_block": Config("cfg4_block", B=8, L=8192, d=2048, V=151936, k=4, mask="semi_ar",
+                         block=32, block_only=True,
+                         description="B8 L8192 d2048 V151936, cfg4's mask and windows, logits "
+                                     "for the current 32-token block only (256 rows), k=4"),
 }
 
 
@@ -83,9 +92,9 @@ def get_config(name: str, **overrides) -> Config:
 
 
 def custom_config(B, L, d, V, k, mask="bernoulli", r=0.5, n_suffix=0, block=32,
-                  name="custom") -> Config:
+                  name="custom", block_only=False) -> Config:
     return Config(name, B=B, L=L, d=d, V=V, k=k, mask=mask, r=r, n_suffix=n_suffix,
-                  block=block)
+                  block=block, block_only=block_only)
 
 
 def _bernoulli_mask(g: torch.Generator, B: int, L: int, r: float) -> torch.Tensor:
