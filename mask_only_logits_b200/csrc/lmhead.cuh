@@ -87,7 +87,7 @@ struct Cfg {
                                      (static_cast<uint32_t>(BM >> 4) << 24);
 };
 
-// The unit schedule, computed identically by every role of the GEMM.
+// The unit schedule, computed identically by every role of the GEMM (and by host code).
 //
 // m-tiles are taken in groups of up to gmax.  Inside a group of G m-tiles each holder takes
 // one m-tile and a contiguous range of vocabulary tiles: P = ctas / G "streams" per m-tile,
@@ -181,7 +181,7 @@ struct Unit {
   bool leftover;
   long long i0, i1;
 };
-__device__ __forceinline__ bool unit_of(const Plan& pl, int g, int holder, Unit& u) {
+__host__ __device__ __forceinline__ bool unit_of(const Plan& pl, int g, int holder, Unit& u) {
   u.G = pl.group_size(g);
   u.P = Plan::streams(u.G, pl.ctas, pl.numN);
   u.leftover = false;
@@ -211,7 +211,7 @@ __device__ __forceinline__ bool unit_of(const Plan& pl, int g, int holder, Unit&
 // Calls f(m_tile, n) for every tile of the holder, in order; stops early when f returns
 // false.  Returns whether all calls returned true.
 template <class F>
-__device__ __forceinline__ bool for_each_tile(const Plan& pl, int holder, F& f) {
+__host__ __device__ __forceinline__ bool for_each_tile(const Plan& pl, int holder, F& f) {
   for (int g = 0; g < pl.ngroups; ++g) {
     Unit u;
     if (!unit_of(pl, g, holder, u)) continue;
