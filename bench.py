@@ -271,6 +271,104 @@ def workload_config(cfg, count: int) -> dict:
 
 
 # ------------------------------------------------------------------------------ our arm
+def run_vocab_sharded(args, cfg) -> None:
+    """One decode step with the vocabulary projection split by rows over the ranks
+    (``sharded.VocabShardedStep``): every rank holds the same H and mask and its shard of W;
+    the step's only exchange is an all-gather of the per-row partials.  Strong scaling: the
+    job processes one step's masked rows per step whatever the number of ranks."""
+    from mask_only_logits_b200 import dist as D
+    info = D.rank_info()
+    world, rank, local = info.world, info.rank, info.local_rank
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    dist = D.init_process_group("nccl", timeout_s=120, device=dev) if world > 1 else None
+    inp = WL.make_inputs(cfg, seed=0)                 # the same problem on every rank
+    count = rows_of_step(inp)
+    cpu = cpu_baseline(inp) if rank == 0 and world == 1 and not args.no_cpu_baseline else None
+    import mask_only_logits_b200 as dl
+    from mask_only_logits_b200.sharded import VocabShardedStep
+    dl.debug_set_gemm_variant(args.gemm_variant)
+    step = VocabShardedStep(cfg.B, cfg.L, cfg.d, cfg.V, cfg.k, rank=rank, world=world, device=dev)
+    H, M = inp["H"].to(dev), inp["M"].to(dev)
+    W_shard = inp["W"][step.v0:step.v1].contiguous().to(dev)
+    win_lo = None if inp["win_lo"] is None else torch.from_numpy(inp["win_lo"]).to(dev)
+    win_hi = None if inp["win_hi"] is None else torch.from_numpy(inp["win_hi"]).to(dev)
+    stream = torch.cuda.current_stream(dev)
+    blk = cfg.block_only
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        step.run(H, M, W_shard, win_lo, win_hi, stream, blk)
+    torch.cuda.synchronize(dev)
+    if dl.get_status(stream) != 0 or int(step.count[0]) != count:
+        raise RuntimeError("warm-up failed")
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        barrier()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step.run(H, M, W_shard, win_lo, win_hi, stream, blk)
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+    t_ms = ev0.elapsed_time(ev1)
+    barrier()
+    dl.prof_begin()
+    for _ in range(args.steps):
+        step.run(H, M, W_shard, win_lo, win_hi, stream, blk)
+    torch.cuda.synchronize(dev)
+    gemm_ms, gemm_launches, launches = dl.prof_end()
+    if dl.get_status(stream) != 0:
+        raise RuntimeError("device status after the timed region")
+    t_ms, gemm_ms = D.max_over_ranks([t_ms, gemm_ms], dev)
+    # end to end: H and the mask from pinned host memory, the selection back, every step
+    e2e_steps = args.e2e_steps or max(10, min(args.steps, 200))
+    H_host, M_host = inp["H"].pin_memory(), inp["M"].pin_memory()
+    H_dev, M_dev = torch.empty_like(H), torch.empty_like(M)
+    idx_host = torch.empty(cfg.B, cfg.k, dtype=torch.int32).pin_memory()
+    barrier()
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        H_dev.copy_(H_host, non_blocking=True)
+        M_dev.copy_(M_host, non_blocking=True)
+        step.run(H_dev, M_dev, W_shard, win_lo, win_hi, stream, blk)
+        idx_host.copy_(step.idx, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    e2e_ms = D.max_over_ranks([(time.perf_counter() - t0) * 1e3], dev)[0]
+    barrier()
+    if rank == 0:
+        peaks = load_peaks()
+        shard_cfg = WL.get_config(cfg.name, V=step.v1 - step.v0)
+        ms_step = t_ms / args.steps
+        roof = gemm_roofline(shard_cfg, count, peaks, gemm_ms / max(1, gemm_launches) / 1e3,
+                             args.gemm_variant == 2 or (args.gemm_variant == 0 and cfg.B * cfg.L <= 16384),
+                             "vocabulary shard")
+        roof["traffic"] = None
+        roof["shard"] = f"rows [{step.v0}, {step.v1}) of W on rank 0"
+        line = dict(
+            metric=METRIC, value=count * args.steps / (t_ms / 1e3), unit=UNIT, n_gpus=world,
+            steps=args.steps, warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True,
+            scaling="strong", vs_baseline=None, dtype="bf16", data="synthetic",
+            config=dict(workload_config(cfg, count), parallelism=f"vocabulary-parallel over {world} GPU(s)"),
+            roofline=roof, gpu_launches=launches,
+            e2e=dict(value=count * e2e_steps / (e2e_ms / 1e3), unit=UNIT,
+                     h2d_bytes_per_step=cfg.B * cfg.L * (2 * cfg.d + 1),
+                     d2h_bytes_per_step=cfg.B * cfg.k * 4, ms_per_step=e2e_ms / e2e_steps,
+                     note="every rank copies H and the mask in from pinned host memory and "
+                          "its selection back each step; wall clock, max over ranks"),
+            clocks=clk.summary())
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main() -> None:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -280,6 +378,9 @@ def main() -> None:
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--shard", default="replica", choices=["replica", "vocab"],
+                    help="replica: one independent step per rank (weak scaling); vocab: one "
+                         "step with W split by rows over the ranks (strong scaling)")
     ap.add_argument("--gemm-variant", type=int, default=0, choices=[0, 1, 2],
                     help="0 = library default, 1 = single-SM GEMM, 2 = paired-SM GEMM")
     args = ap.parse_args()
@@ -290,6 +391,9 @@ def main() -> None:
         run_reference(args, cfg)
         return
 
+    if args.shard == "vocab":
+        run_vocab_sharded(args, cfg)
+        return
     from mask_only_logits_b200 import dist as D
     info = D.rank_info()
     world, rank, local = info.world, info.rank, info.local_rank

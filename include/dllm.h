@@ -210,6 +210,60 @@ dllm_status dllm_masked_logits_window(const uint16_t* H, const uint8_t* M, const
                                       size_t ws_bytes, void* stream);
 
 /*
+ * dllm_masked_partials - one vocabulary shard of a vocabulary-parallel LM head.
+ *
+ * With W split by rows over GPUs (GPU g holds W[v_offset_g : v_offset_g + V_shard_g, :]),
+ * each GPU runs this call on its shard and the same H and M.  It computes exactly what
+ * dllm_masked_logits computes, over this shard's vocabulary only, and writes each masked
+ * row's softmax partial instead of the finished values (no logit is stored):
+ *     part_m[i] = max_v z_v,   part_s[i] = sum_v exp(z_v - part_m[i]),
+ *     part_a[i] = v_offset + the smallest v attaining the max        (v over the shard)
+ * and, in extended mode (stats != 0), part_t[i] = sum_v exp(z_v - m)(z_v - m) and
+ * part_m2[i] = the second-largest logit.  After the partials of every shard are gathered
+ * (one all-gather of 12 bytes per row per shard, 20 in extended mode), dllm_lse_merge
+ * turns them into tok / conf / lse (/ entropy / margin) over the whole vocabulary.  The
+ * partial algebra is the split-vocabulary merge of the Mosaic page's mask-only logits
+ * kernel, applied across GPUs instead of across tiles.
+ *
+ *   W_shard  device, bf16 [V_shard, d] row-major: rows v_offset .. v_offset+V_shard-1 of W.
+ *   v_offset first global token index of the shard (>= 0; v_offset + V_shard < 2^31).
+ *   win_lo, win_hi  device int32 [B] or both NULL: as in dllm_masked_logits_window.
+ *   stats    0, or DLLM_STAT_ENTROPY and/or DLLM_STAT_MARGIN: then part_t and part_m2 are
+ *            both required (the extended partial carries both); else both NULL.
+ *   part_m, part_s, part_a  device [B*L] capacity, compacted order (entries < count).
+ * row_idx, seq_off, count, workspace and errors as in dllm_masked_logits.
+ */
+dllm_status dllm_masked_partials(const uint16_t* H, const uint8_t* M, const uint16_t* W_shard,
+                                 int32_t B, int32_t L, int32_t d, int32_t V_shard,
+                                 int32_t v_offset, const int32_t* win_lo, const int32_t* win_hi,
+                                 uint32_t stats, float* part_m, float* part_s, int32_t* part_a,
+                                 float* part_t, float* part_m2, int32_t* row_idx,
+                                 int32_t* seq_off, int32_t* count, void* ws, size_t ws_bytes,
+                                 void* stream);
+
+/*
+ * dllm_lse_merge - merge per-shard softmax partials into the finished per-row values:
+ *     m* = max_j m_j,  s* = sum_j s_j exp(m_j - m*),  tok = a_j of the first j with m_j = m*,
+ *     lse = m* + ln s*,  conf = exp(m* - lse) = 1 / s*
+ * (extended: t* = sum_j exp(m_j - m*)(t_j + (m_j - m*) s_j), entropy = ln s* - t* / s*;
+ * m2* = second largest of all m_j and m2_j, margin = (1 - exp(m2* - m*)) / s*).
+ *
+ *   part_*   device; split j of row i at index j * split_stride + i, splits in ascending
+ *            vocabulary order (a tie of maxima keeps the lower split, i.e. the lower token).
+ *   count    device int32 [1]: rows 0 .. min(*count, n_cap)-1 are merged (the count written
+ *            by dllm_masked_partials stays on the device).
+ *   stats    as in dllm_masked_partials; entropy / margin non-NULL exactly when requested.
+ *   tok, conf, lse  device [n_cap] capacity, compacted order.
+ * Constraints: n_split >= 1, n_cap >= 1, split_stride >= n_cap.  Errors: DLLM_ERR_NULL,
+ * DLLM_ERR_ALIGN, DLLM_ERR_SHAPE, DLLM_ERR_CUDA, DLLM_ERR_DEVICE.
+ */
+dllm_status dllm_lse_merge(const float* part_m, const float* part_s, const int32_t* part_a,
+                           const float* part_t, const float* part_m2, int64_t split_stride,
+                           int32_t n_split, const int32_t* count, int32_t n_cap, uint32_t stats,
+                           int32_t* tok, float* conf, float* lse, float* entropy,
+                           float* margin, void* stream);
+
+/*
  * dllm_select_unmask - per-sequence top-k over confidences (confidence-driven unmasking,
  * dLLM inference survey page, "Main Findings").
  *

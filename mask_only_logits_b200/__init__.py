@@ -7,9 +7,10 @@ fallback: if ``libdllm.so`` is missing, loading fails loudly.
 
 Low-level calls (same names and arguments as the C ABI, tensors instead of pointers):
 ``workspace_bytes``, ``mask_compact``, ``masked_logits``, ``select_unmask``,
-``decode_step``, ``get_status``.  ``DecodeStep`` owns the buffers of one shape and runs a
-whole step on device tensors (``run``) or on host tensors with the copies included
-(``run_host``).
+``decode_step``, ``get_status``, and for a vocabulary-parallel LM head ``masked_partials``
+and ``lse_merge``.  ``DecodeStep`` owns the buffers of one shape and runs a whole step on
+device tensors (``run``) or on host tensors with the copies included (``run_host``,
+``run_host_pipeline``); ``sharded.VocabShardedStep`` runs it with W split over ranks.
 """
 from __future__ import annotations
 
@@ -22,6 +23,7 @@ from . import _abi
 __all__ = [
     "DllmError", "lib", "version", "workspace_bytes", "mask_compact", "mask_compact_noalloc",
     "masked_logits", "masked_logits_ex", "select_unmask_ex", "STAT_ENTROPY", "STAT_MARGIN",
+    "masked_partials", "lse_merge",
     "select_unmask", "decode_step", "get_status", "debug_lmhead_logits", "debug_lse_merge",
     "debug_set_gemm_variant",
     "prof_begin", "prof_end", "DecodeStep", "MAX_K",
@@ -145,6 +147,39 @@ def masked_logits_ex(H, M, W, stats, tok, conf, lse, entropy, margin, row_idx, s
         _check(lib().dllm_masked_logits_window(*ins, _ptr(win_lo, torch.int32, "win_lo"),
                                                _ptr(win_hi, torch.int32, "win_hi"), stats,
                                                *common), "dllm_masked_logits_window")
+
+
+def masked_partials(H, M, W_shard, v_offset, stats, part_m, part_s, part_a, part_t, part_m2,
+                    row_idx, seq_off, count, ws, stream=None, win_lo=None, win_hi=None) -> None:
+    """One vocabulary shard of a vocabulary-parallel LM head (W_shard = rows v_offset ..
+    v_offset + V_shard - 1 of W): per masked row, the softmax partial (max, sum of exp,
+    global argmax; plus t and second max when stats != 0) over the shard's vocabulary."""
+    B, L = M.shape
+    V_shard, d = W_shard.shape
+    _check(lib().dllm_masked_partials(
+        _ptr(H, torch.bfloat16, "H"), _ptr(M, torch.uint8, "M"),
+        _ptr(W_shard, torch.bfloat16, "W_shard"), B, L, d, V_shard, int(v_offset),
+        _ptr(win_lo, torch.int32, "win_lo"), _ptr(win_hi, torch.int32, "win_hi"), stats,
+        _ptr(part_m, torch.float32, "part_m"), _ptr(part_s, torch.float32, "part_s"),
+        _ptr(part_a, torch.int32, "part_a"), _ptr(part_t, torch.float32, "part_t"),
+        _ptr(part_m2, torch.float32, "part_m2"), _ptr(row_idx, torch.int32, "row_idx"),
+        _ptr(seq_off, torch.int32, "seq_off"), _ptr(count, torch.int32, "count"),
+        _ptr(ws, None, "ws"), ws.numel() * ws.element_size(), _stream(stream)),
+        "dllm_masked_partials")
+
+
+def lse_merge(part_m, part_s, part_a, part_t, part_m2, split_stride, n_split, count, n_cap,
+              stats, tok, conf, lse, entropy=None, margin=None, stream=None) -> None:
+    """Merge per-shard partials (split j of row i at j * split_stride + i) into tok, conf,
+    lse (and entropy / margin) for rows below the device-side count."""
+    _check(lib().dllm_lse_merge(
+        _ptr(part_m, torch.float32, "part_m"), _ptr(part_s, torch.float32, "part_s"),
+        _ptr(part_a, torch.int32, "part_a"), _ptr(part_t, torch.float32, "part_t"),
+        _ptr(part_m2, torch.float32, "part_m2"), int(split_stride), int(n_split),
+        _ptr(count, torch.int32, "count"), int(n_cap), stats, _ptr(tok, torch.int32, "tok"),
+        _ptr(conf, torch.float32, "conf"), _ptr(lse, torch.float32, "lse"),
+        _ptr(entropy, torch.float32, "entropy"), _ptr(margin, torch.float32, "margin"),
+        _stream(stream)), "dllm_lse_merge")
 
 
 def select_unmask_ex(score, row_idx, seq_off, B, L, k, threshold, min_sel, idx, n_sel,

@@ -244,20 +244,31 @@ struct LogitsArgs {
   int* tok; float* conf; float* lse; float* dbg;
   int* row_idx; int* seq_off; int* count;
   void* ws; size_t ws_bytes; cudaStream_t s;
+  lm::Partials raw = {nullptr, nullptr, nullptr, nullptr, nullptr};   // vocabulary-shard mode
+  int a_offset = 0;
 };
 
 dllm_status validate_logits(const LogitsArgs& a, bool debug) {
   if (!a.H || !a.M || !a.W || !a.row_idx || !a.seq_off || !a.count || !a.ws) return DLLM_ERR_NULL;
-  if (!debug && (!a.tok || !a.conf || !a.lse)) return DLLM_ERR_NULL;
+  const bool shard = a.raw.m != nullptr;
+  if (shard) {
+    if (!a.raw.s || !a.raw.a) return DLLM_ERR_NULL;
+    if ((a.stats != 0) != (a.raw.t != nullptr) || (a.stats != 0) != (a.raw.m2 != nullptr))
+      return DLLM_ERR_NULL;
+    if (a.a_offset < 0 || static_cast<long long>(a.a_offset) + a.V >= (1ll << 31)) return DLLM_ERR_SHAPE;
+  } else if (!debug && (!a.tok || !a.conf || !a.lse)) {
+    return DLLM_ERR_NULL;
+  }
   if (debug && !a.dbg) return DLLM_ERR_NULL;
   if ((a.win_lo == nullptr) != (a.win_hi == nullptr)) return DLLM_ERR_NULL;
   if ((a.stats & ~(DLLM_STAT_ENTROPY | DLLM_STAT_MARGIN)) != 0) return DLLM_ERR_SHAPE;
-  if (((a.stats & DLLM_STAT_ENTROPY) != 0) != (a.entropy != nullptr)) return DLLM_ERR_NULL;
-  if (((a.stats & DLLM_STAT_MARGIN) != 0) != (a.margin != nullptr)) return DLLM_ERR_NULL;
+  if (!shard && ((a.stats & DLLM_STAT_ENTROPY) != 0) != (a.entropy != nullptr)) return DLLM_ERR_NULL;
+  if (!shard && ((a.stats & DLLM_STAT_MARGIN) != 0) != (a.margin != nullptr)) return DLLM_ERR_NULL;
   if (!shapes_ok(a.B, a.L) || a.V < 1 || a.d < DLLM_D_MULTIPLE || a.d % DLLM_D_MULTIPLE != 0)
     return DLLM_ERR_SHAPE;
   const void* ptrs[] = {a.H, a.M, a.W, a.row_idx, a.seq_off, a.count, a.ws, a.tok, a.conf, a.lse,
-                        a.dbg, a.entropy, a.margin, a.win_lo, a.win_hi};
+                        a.dbg, a.entropy, a.margin, a.win_lo, a.win_hi, a.raw.m, a.raw.s,
+                        a.raw.a, a.raw.t, a.raw.m2};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return DLLM_ERR_ALIGN;
   if (a.ws_bytes < ws_layout(a.B, a.L, a.d, a.V).total) return DLLM_ERR_WORKSPACE;
@@ -280,7 +291,7 @@ dllm_status run_logits(const LogitsArgs& a, bool debug) {
   float* pm2 = reinterpret_cast<float*>(ws + w.pm2_off);
   int* ctr = reinterpret_cast<int*>(ws + w.ctr_off);
   const lm::Partials part{pm, ps, pa, pt, pm2};
-  const lm::Outputs outs{a.tok, a.conf, a.lse, a.entropy, a.margin};
+  const lm::Outputs outs{a.tok, a.conf, a.lse, a.entropy, a.margin, a.raw, a.a_offset};
   const long long n = static_cast<long long>(a.B) * a.L;
 
   // GEMM variant and its work holders (CTAs, or CTA pairs)
@@ -520,6 +531,57 @@ dllm_status dllm_masked_logits_window(const uint16_t* H, const uint8_t* M, const
   LogitsArgs a{H, M, W, B, L, d, V, win_lo, win_hi, stats, entropy, margin, tok, conf, lse, nullptr,
                row_idx, seq_off, count, ws, ws_bytes, static_cast<cudaStream_t>(stream)};
   return run_logits(a, false);
+}
+
+dllm_status dllm_masked_partials(const uint16_t* H, const uint8_t* M, const uint16_t* W_shard,
+                                 int32_t B, int32_t L, int32_t d, int32_t V_shard, int32_t v_offset,
+                                 const int32_t* win_lo, const int32_t* win_hi, uint32_t stats,
+                                 float* part_m, float* part_s, int32_t* part_a, float* part_t,
+                                 float* part_m2, int32_t* row_idx, int32_t* seq_off, int32_t* count,
+                                 void* ws, size_t ws_bytes, void* stream) {
+  if (!part_m) return DLLM_ERR_NULL;
+  LogitsArgs a{H, M, W_shard, B, L, d, V_shard, win_lo, win_hi, stats, nullptr, nullptr, nullptr,
+               nullptr, nullptr, nullptr, row_idx, seq_off, count, ws, ws_bytes,
+               static_cast<cudaStream_t>(stream)};
+  a.raw = lm::Partials{part_m, part_s, part_a, part_t, part_m2};
+  a.a_offset = v_offset;
+  return run_logits(a, false);
+}
+
+dllm_status dllm_lse_merge(const float* part_m, const float* part_s, const int32_t* part_a,
+                           const float* part_t, const float* part_m2, int64_t split_stride,
+                           int32_t n_split, const int32_t* count, int32_t n_cap, uint32_t stats,
+                           int32_t* tok, float* conf, float* lse, float* entropy, float* margin,
+                           void* stream) {
+  if (!part_m || !part_s || !part_a || !count || !tok || !conf || !lse) return DLLM_ERR_NULL;
+  if ((stats & ~(DLLM_STAT_ENTROPY | DLLM_STAT_MARGIN)) != 0) return DLLM_ERR_SHAPE;
+  if ((stats != 0) != (part_t != nullptr) || (stats != 0) != (part_m2 != nullptr)) return DLLM_ERR_NULL;
+  if (((stats & DLLM_STAT_ENTROPY) != 0) != (entropy != nullptr)) return DLLM_ERR_NULL;
+  if (((stats & DLLM_STAT_MARGIN) != 0) != (margin != nullptr)) return DLLM_ERR_NULL;
+  if (n_split < 1 || n_cap < 1 || split_stride < n_cap) return DLLM_ERR_SHAPE;
+  const void* ptrs[] = {part_m, part_s, part_a, part_t, part_m2, count, tok, conf, lse, entropy, margin};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return DLLM_ERR_ALIGN;
+  DeviceState* ds = nullptr;
+  dllm_status st = device_state(&ds);
+  if (st != DLLM_OK) return st;
+  int blocks = (n_cap + kMergeThreads - 1) / kMergeThreads;
+  if (blocks > ds->sms * 8) blocks = ds->sms * 8;
+  const lm::Partials part{const_cast<float*>(part_m), const_cast<float*>(part_s),
+                          const_cast<int*>(part_a), const_cast<float*>(part_t),
+                          const_cast<float*>(part_m2)};
+  const lm::Outputs outs{tok, conf, lse, entropy, margin, lm::Partials{nullptr, nullptr, nullptr, nullptr, nullptr}, 0};
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const cudaError_t e = stats != 0
+      ? launch_pdl(lse_merge_kernel<true>, dim3(blocks), dim3(kMergeThreads), 0, s, part,
+                   static_cast<long long>(split_stride), static_cast<int>(n_split), count,
+                   static_cast<int>(n_cap), outs)
+      : launch_pdl(lse_merge_kernel<false>, dim3(blocks), dim3(kMergeThreads), 0, s, part,
+                   static_cast<long long>(split_stride), static_cast<int>(n_split), count,
+                   static_cast<int>(n_cap), outs);
+  if (e != cudaSuccess) return DLLM_ERR_CUDA;
+  count_launch();
+  return DLLM_OK;
 }
 
 dllm_status dllm_debug_lmhead_logits(const uint16_t* H, const uint8_t* M, const uint16_t* W,

@@ -457,6 +457,11 @@ struct Outputs {
   float* lse;
   float* entropy;   // extended mode: written when not null
   float* margin;    // extended mode: written when not null
+  // Vocabulary-shard mode (raw.m not null): instead of the finished values, each row's
+  // merged state over this launch's vocabulary (a shard of a larger one) is written, with
+  // the argmax shifted by a_offset to a global token index; t and m2 in extended mode.
+  Partials raw;
+  int a_offset;
 };
 
 template <int CG, int kMode>
@@ -632,6 +637,16 @@ lmhead_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
       return true;
     };
     auto write_result = [&](int row, const RowState& st) {
+      if (out.raw.m != nullptr) {
+        out.raw.m[row] = st.m;
+        out.raw.s[row] = st.s;
+        out.raw.a[row] = st.a + out.a_offset;
+        if constexpr (kExt) {
+          if (out.raw.t) out.raw.t[row] = st.t;
+          if (out.raw.m2) out.raw.m2[row] = st.m2;
+        }
+        return;
+      }
       int t;
       float c, l, e, mg;
       state_finish(st, t, c, l, e, mg);
