@@ -51,6 +51,16 @@ PROTOTYPES = {
 _lib = None
 
 
+def load_from(path: str) -> ctypes.CDLL:
+    """Load another build of the library (e.g. a test variant) with the same prototypes."""
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in PROTOTYPES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
 def load() -> ctypes.CDLL:
     """Load libdllm.so from the package directory; raise if it has not been built."""
     global _lib

@@ -40,10 +40,13 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(f) <= t for f in SOURCES + HEADERS)
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
-    if not force and up_to_date():
+def build(force: bool = False, verbose: bool = False, extra_flags=(), out: str | None = None) -> str:
+    """Build libdllm.so in the package directory (or at `out`, e.g. a test's variant
+    built with extra -D flags; that one is always rebuilt)."""
+    target = out or LIB_PATH
+    if out is None and not force and up_to_date():
         return LIB_PATH
-    tmp = LIB_PATH + ".tmp"
+    tmp = target + ".tmp"
     cmd = [nvcc_path(), *NVCC_FLAGS, *extra_flags, "-I", os.path.join(ROOT, "include"),
            "-o", tmp, *SOURCES]
     if verbose:
@@ -53,8 +56,8 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
         raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stdout}\n{res.stderr}")
     if verbose and (res.stdout or res.stderr):
         print(res.stdout + res.stderr, flush=True)
-    os.replace(tmp, LIB_PATH)
-    return LIB_PATH
+    os.replace(tmp, target)
+    return target
 
 
 if __name__ == "__main__":

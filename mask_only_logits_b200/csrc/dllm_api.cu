@@ -12,6 +12,8 @@
 #include <mutex>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "dllm.h"
 #include "ptx.cuh"
 #include "compact.cuh"
@@ -20,6 +22,16 @@
 #include "select.cuh"
 
 namespace dllm {
+
+// An NVTX range around each entry point of the ABI, named after it, so that a timeline
+// profiler groups the kernels of one library call (header-only NVTX v3: without a tool
+// attached a range costs a null-pointer check).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // Device-side error bits (kStatusTimeout, kStatusBounds); one word per device.
 __device__ int g_status;
@@ -439,6 +451,7 @@ extern "C" {
 
 dllm_status dllm_mask_compact_noalloc(const uint8_t* M, int32_t B, int32_t L, int32_t* row_idx,
                                       int32_t* seq_off, int32_t* count, void* stream) {
+  const dllm::NvtxRange nvtx_range("dllm_mask_compact_noalloc");
   if (!M || !row_idx || !seq_off || !count) return DLLM_ERR_NULL;
   if (!shapes_ok(B, L)) return DLLM_ERR_SHAPE;
   if (static_cast<long long>(B) * L > DLLM_NOALLOC_MAX_POSITIONS) return DLLM_ERR_SCRATCH;
@@ -479,6 +492,7 @@ size_t dllm_workspace_bytes(int32_t B, int32_t L, int32_t d, int32_t V) {
 dllm_status dllm_mask_compact_window(const uint8_t* M, int32_t B, int32_t L, const int32_t* win_lo,
                                      const int32_t* win_hi, int32_t* row_idx, int32_t* seq_off,
                                      int32_t* count, void* ws, size_t ws_bytes, void* stream) {
+  const dllm::NvtxRange nvtx_range("dllm_mask_compact_window");
   if (!M || !row_idx || !seq_off || !count || !ws) return DLLM_ERR_NULL;
   if ((win_lo == nullptr) != (win_hi == nullptr)) return DLLM_ERR_NULL;
   if (!shapes_ok(B, L)) return DLLM_ERR_SHAPE;
@@ -506,6 +520,7 @@ dllm_status dllm_masked_logits(const uint16_t* H, const uint8_t* M, const uint16
                                int32_t L, int32_t d, int32_t V, int32_t* tok, float* conf,
                                float* lse, int32_t* row_idx, int32_t* seq_off, int32_t* count,
                                void* ws, size_t ws_bytes, void* stream) {
+  const dllm::NvtxRange nvtx_range("dllm_masked_logits");
   LogitsArgs a{H, M, W, B, L, d, V, nullptr, nullptr, 0u, nullptr, nullptr, tok, conf, lse, nullptr,
                row_idx, seq_off, count, ws, ws_bytes, static_cast<cudaStream_t>(stream)};
   return run_logits(a, false);
@@ -516,6 +531,7 @@ dllm_status dllm_masked_logits_ex(const uint16_t* H, const uint8_t* M, const uin
                                   float* conf, float* lse, float* entropy, float* margin,
                                   int32_t* row_idx, int32_t* seq_off, int32_t* count, void* ws,
                                   size_t ws_bytes, void* stream) {
+  const dllm::NvtxRange nvtx_range("dllm_masked_logits_ex");
   LogitsArgs a{H, M, W, B, L, d, V, nullptr, nullptr, stats, entropy, margin, tok, conf, lse, nullptr,
                row_idx, seq_off, count, ws, ws_bytes, static_cast<cudaStream_t>(stream)};
   return run_logits(a, false);
@@ -527,6 +543,7 @@ dllm_status dllm_masked_logits_window(const uint16_t* H, const uint8_t* M, const
                                       int32_t* tok, float* conf, float* lse, float* entropy,
                                       float* margin, int32_t* row_idx, int32_t* seq_off,
                                       int32_t* count, void* ws, size_t ws_bytes, void* stream) {
+  const dllm::NvtxRange nvtx_range("dllm_masked_logits_window");
   if (!win_lo || !win_hi) return DLLM_ERR_NULL;
   LogitsArgs a{H, M, W, B, L, d, V, win_lo, win_hi, stats, entropy, margin, tok, conf, lse, nullptr,
                row_idx, seq_off, count, ws, ws_bytes, static_cast<cudaStream_t>(stream)};
@@ -539,6 +556,7 @@ dllm_status dllm_masked_partials(const uint16_t* H, const uint8_t* M, const uint
                                  float* part_m, float* part_s, int32_t* part_a, float* part_t,
                                  float* part_m2, int32_t* row_idx, int32_t* seq_off, int32_t* count,
                                  void* ws, size_t ws_bytes, void* stream) {
+  const dllm::NvtxRange nvtx_range("dllm_masked_partials");
   if (!part_m) return DLLM_ERR_NULL;
   LogitsArgs a{H, M, W_shard, B, L, d, V_shard, win_lo, win_hi, stats, nullptr, nullptr, nullptr,
                nullptr, nullptr, nullptr, row_idx, seq_off, count, ws, ws_bytes,
@@ -553,6 +571,7 @@ dllm_status dllm_lse_merge(const float* part_m, const float* part_s, const int32
                            int32_t n_split, const int32_t* count, int32_t n_cap, uint32_t stats,
                            int32_t* tok, float* conf, float* lse, float* entropy, float* margin,
                            void* stream) {
+  const dllm::NvtxRange nvtx_range("dllm_lse_merge");
   if (!part_m || !part_s || !part_a || !count || !tok || !conf || !lse) return DLLM_ERR_NULL;
   if ((stats & ~(DLLM_STAT_ENTROPY | DLLM_STAT_MARGIN)) != 0) return DLLM_ERR_SHAPE;
   if ((stats != 0) != (part_t != nullptr) || (stats != 0) != (part_m2 != nullptr)) return DLLM_ERR_NULL;
@@ -627,6 +646,7 @@ dllm_status dllm_select_unmask(const float* conf, const int32_t* row_idx, const 
                                int32_t B, int32_t L, int32_t k, const int32_t* win_lo,
                                const int32_t* win_hi, const int32_t* tok, int32_t* idx,
                                int32_t* n_sel, int32_t* tok_sel, float* conf_sel, void* stream) {
+  const dllm::NvtxRange nvtx_range("dllm_select_unmask");
   return run_select(conf, row_idx, seq_off, B, L, k, false, 0.f, 0, false, win_lo, win_hi, tok, idx,
                     n_sel, tok_sel, conf_sel, stream);
 }
@@ -636,6 +656,7 @@ dllm_status dllm_select_unmask_ex(const float* score, const int32_t* row_idx, co
                                   int32_t ascending, const int32_t* win_lo, const int32_t* win_hi,
                                   const int32_t* tok, int32_t* idx, int32_t* n_sel, int32_t* tok_sel,
                                   float* score_sel, void* stream) {
+  const dllm::NvtxRange nvtx_range("dllm_select_unmask_ex");
   if (ascending != 0 && ascending != 1) return DLLM_ERR_SHAPE;
   return run_select(score, row_idx, seq_off, B, L, k, true, threshold, min_sel, ascending != 0,
                     win_lo, win_hi, tok, idx, n_sel, tok_sel, score_sel, stream);
@@ -647,6 +668,7 @@ dllm_status dllm_decode_step(const uint16_t* H, const uint8_t* M, const uint16_t
                              int32_t* row_idx, int32_t* seq_off, int32_t* count, int32_t* idx,
                              int32_t* n_sel, int32_t* tok_sel, float* conf_sel, void* ws,
                              size_t ws_bytes, void* stream) {
+  const dllm::NvtxRange nvtx_range("dllm_decode_step");
   // validate the selection's own arguments first so that nothing is launched on error
   if (!idx || !n_sel) return DLLM_ERR_NULL;
   if ((win_lo == nullptr) != (win_hi == nullptr)) return DLLM_ERR_NULL;
@@ -667,6 +689,7 @@ dllm_status dllm_decode_block_step(const uint16_t* H, const uint8_t* M, const ui
                                    int32_t* row_idx, int32_t* seq_off, int32_t* count, int32_t* idx,
                                    int32_t* n_sel, int32_t* tok_sel, float* conf_sel, void* ws,
                                    size_t ws_bytes, void* stream) {
+  const dllm::NvtxRange nvtx_range("dllm_decode_block_step");
   if (!idx || !n_sel || !win_lo || !win_hi) return DLLM_ERR_NULL;
   if (k < 1 || k > DLLM_MAX_K) return DLLM_ERR_SHAPE;
   const void* ptrs[] = {idx, n_sel, tok_sel, conf_sel};

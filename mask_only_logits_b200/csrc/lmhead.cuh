@@ -537,6 +537,11 @@ lmhead_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
           const int s = it % C::kStages;
           const uint32_t ph = (it / C::kStages) & 1u;
           if (!mbar_wait(smem_u32(&sm.empty[s]), ph ^ 1u, abort_flag, status)) return false;
+#ifdef DLLM_FAULT_SKIP_STAGE
+          // Failure-detection test builds only: this stage is never armed or loaded, so the
+          // MMA issuer's bounded wait on it runs out and the kernel unwinds with a timeout.
+          if (it == DLLM_FAULT_SKIP_STAGE) continue;
+#endif
           const uint32_t fb = smem_u32(&sm.full[s]);
           if constexpr (CG == 1) {
             mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
