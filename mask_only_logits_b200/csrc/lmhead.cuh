@@ -77,7 +77,10 @@ struct Cfg {
   static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int kStages = CG == 1 ? 4 : DLLM_STAGES2;
-  static constexpr int SMEM_BYTES = 1024 + kStages * STAGE_BYTES + 256;
+  // ring, barriers and flags, and the merge's combine buffer (4 x 128 row states)
+  static constexpr int kCombBytes = 4 * BM_CTA * 20;
+  static constexpr int SMEM_BYTES = 1024 + kStages * STAGE_BYTES + 256 + kCombBytes;
+  static_assert(SMEM_BYTES <= 232448, "exceeds the 227 KB of shared memory of one CTA");
   static constexpr int kGroupM = CG == 1 ? DLLM_GROUP_M1 : DLLM_GROUP_M2;  // m-tiles per L2 group
   // Instruction descriptor, kind::f16: fp32 accumulator (bits 4-5 = 1), A and B bf16
   // (bits 7-9 = 1, bits 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bits 17-22,
@@ -240,6 +243,8 @@ struct Smem {
   uint32_t* tmem_slot;
   int* abort_flag;
   volatile int* last_flag;   // epilogue: this CTA finished the last unit of an m-tile
+  struct RowStateRaw { float m, s, t, m2; int a; };
+  RowStateRaw* comb;         // merge: per warp quarter, the merged state of each of 128 rows
 
   __device__ __forceinline__ explicit Smem(uint8_t* raw) {
     using C = Cfg<CG>;
@@ -256,6 +261,7 @@ struct Smem {
     tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::kStages + 6);
     abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
     last_flag = abort_flag + 1;
+    comb = reinterpret_cast<RowStateRaw*>(reinterpret_cast<uint8_t*>(bars) + 256);
   }
 };
 
@@ -374,6 +380,28 @@ struct Partials {
 // through L2 (other CTAs of the running kernel may have written them) in batches of 8 whose
 // loads are all issued before any is used.
 template <bool kExt>
+__device__ __forceinline__ void merge_state(RowState& st, float m, float s, int a, float t, float m2) {
+  if (m == -INFINITY) return;           // empty partial: nothing to add
+  if (m > st.m) {                       // strict: the earlier split keeps a tie
+    const float sc = ex2_approx((st.m - m) * kLog2e);
+    if constexpr (kExt) {
+      st.t = (st.s > 0.f ? sc * (st.t + (st.m - m) * st.s) : 0.f) + t;
+      st.m2 = fmaxf(st.m, m2);
+    }
+    st.s = st.s * sc + s;
+    st.m = m;
+    st.a = a;
+  } else {
+    const float sc = ex2_approx((m - st.m) * kLog2e);
+    if constexpr (kExt) {
+      st.t += sc * (t + (m - st.m) * s);
+      st.m2 = fmaxf(st.m2, m);
+    }
+    st.s += s * sc;
+  }
+}
+
+template <bool kExt>
 __device__ __forceinline__ void merge_acc(const Partials& P, long long base, long long stride,
                                           int j0, int j1, RowState& st) {
   constexpr int kBatch = 8;
@@ -400,26 +428,7 @@ __device__ __forceinline__ void merge_acc(const Partials& P, long long base, lon
       }
     }
 #pragma unroll
-    for (int q = 0; q < kBatch; ++q) {
-      if (mb[q] == -INFINITY) continue;   // empty partial (or past j1): nothing to add
-      if (mb[q] > st.m) {                 // strict: the earlier split keeps a tie
-        const float sc = ex2_approx((st.m - mb[q]) * kLog2e);
-        if constexpr (kExt) {
-          st.t = (st.s > 0.f ? sc * (st.t + (st.m - mb[q]) * st.s) : 0.f) + tb[q];
-          st.m2 = fmaxf(st.m, m2b[q]);
-        }
-        st.s = st.s * sc + sb[q];
-        st.m = mb[q];
-        st.a = ab[q];
-      } else {
-        const float sc = ex2_approx((mb[q] - st.m) * kLog2e);
-        if constexpr (kExt) {
-          st.t += sc * (tb[q] + (mb[q] - st.m) * sb[q]);
-          st.m2 = fmaxf(st.m2, mb[q]);
-        }
-        st.s += sb[q] * sc;
-      }
-    }
+    for (int q = 0; q < kBatch; ++q) merge_state<kExt>(st, mb[q], sb[q], ab[q], tb[q], m2b[q]);
   }
 }
 
@@ -702,14 +711,74 @@ lmhead_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
       if (!epi_sync()) return false;
       if (*sm.last_flag) {
         __threadfence();
+        // The four epilogue warps split the m-tile's ordered partial slots (streams 0..P-1,
+        // then remainder holders j_lo..j_hi): warp quarter q merges slots
+        // [q * units / 4, (q + 1) * units / 4) for all 128 rows of this CTA, four rows per
+        // lane, so that 4 x kMergeBatch partials per thread are in flight per L2 round trip
+        // instead of kMergeBatch.  The quarters are then combined per row in slot order
+        // through shared memory, which keeps vocabulary order (and so the tie rule).
+        constexpr int kMergeBatch = kExt ? 4 : 8;
+        const int row0 = m_tile * C::BM + static_cast<int>(rank) * C::BM_CTA;   // CTA's first row
+        const int n_valid = pl.count - row0;
+        const long long base0 = pl.part_index(g, u.G, 0, m_local * C::BM + static_cast<int>(rank) * C::BM_CTA);
+        const long long stride = static_cast<long long>(u.G) * C::BM;
+        const int s0 = q * units / 4, s1 = (q + 1) * units / 4;
+        RowState acc[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i].reset();
+        for (int sb = s0; sb < s1; sb += kMergeBatch) {
+          float mb[4][kMergeBatch], sv[4][kMergeBatch], tb[4][kMergeBatch], m2b[4][kMergeBatch];
+          int ab[4][kMergeBatch];
+#pragma unroll
+          for (int j = 0; j < kMergeBatch; ++j) {
+            const int sl = sb + j;
+            const int slot = sl < u.P ? sl : u.P + j_lo + (sl - u.P);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int r = lane + 32 * i;
+              if (sl < s1 && r < n_valid) {
+                const long long e = base0 + slot * stride + r;
+                mb[i][j] = __ldcg(part.m + e);
+                sv[i][j] = __ldcg(part.s + e);
+                ab[i][j] = __ldcg(part.a + e);
+                if constexpr (kExt) {
+                  tb[i][j] = __ldcg(part.t + e);
+                  m2b[i][j] = __ldcg(part.m2 + e);
+                }
+              } else {
+                mb[i][j] = -INFINITY;
+                sv[i][j] = 0.f;
+                ab[i][j] = 0;
+                tb[i][j] = 0.f;
+                m2b[i][j] = -INFINITY;
+              }
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < kMergeBatch; ++j)
+              merge_state<kExt>(acc[i], mb[i][j], sv[i][j], ab[i][j], tb[i][j], m2b[i][j]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          auto& c = sm.comb[q * C::BM_CTA + lane + 32 * i];
+          c.m = acc[i].m;
+          c.s = acc[i].s;
+          c.t = acc[i].t;
+          c.m2 = acc[i].m2;
+          c.a = acc[i].a;
+        }
+        if (!epi_sync()) return false;
         if (valid) {
-          const long long base = pl.part_index(g, u.G, 0, m_local * C::BM + row_in_tile);
-          const long long stride = static_cast<long long>(u.G) * C::BM;
-          RowState mst;
-          mst.reset();
-          merge_acc<kExt>(part, base, stride, 0, u.P, mst);
-          if (j_hi >= j_lo) merge_acc<kExt>(part, base, stride, u.P + j_lo, u.P + j_hi + 1, mst);
-          write_result(row, mst);
+          RowState fin;
+          fin.reset();
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const auto& c = sm.comb[k * C::BM_CTA + row_in_cta];
+            merge_state<kExt>(fin, c.m, c.s, c.a, c.t, c.m2);
+          }
+          write_result(row, fin);
         }
       }
       return true;
