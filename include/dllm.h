@@ -32,6 +32,12 @@
  *     recorded in a per-device status word; dllm_get_status() reports and clears it.
  *   - bf16 tensors are passed as their raw 16-bit patterns (uint16_t).
  *   - Device pointers must be 16-byte aligned.
+ *   - The step inputs H and M (of dllm_masked_logits*, dllm_masked_partials,
+ *     dllm_prepare_rows and the decode-step calls) may instead be page-locked host memory
+ *     (cudaHostAlloc / cudaHostRegister / a pinned torch tensor): the kernels then read it
+ *     over the bus directly, so only the bytes they touch move -- the mask and the masked
+ *     rows of H, not all of H.  Pageable host memory gives DLLM_ERR_MEMORY.  The memory
+ *     must stay valid and unchanged until the call's kernels have run.
  */
 #ifndef DLLM_H
 #define DLLM_H
@@ -55,6 +61,7 @@ typedef int32_t dllm_status;
 #define DLLM_ERR_DEVICE     -7   /* the current device is not an sm_100 GPU                 */
 #define DLLM_ERR_BOUNDS     -8   /* a device-side bound check failed (access skipped)       */
 #define DLLM_ERR_SCRATCH    -9   /* B*L exceeds the fixed scratch of dllm_mask_compact_noalloc */
+#define DLLM_ERR_MEMORY     -10  /* an input is neither device memory nor page-locked host memory */
 
 /* Limits. */
 #define DLLM_MAX_K          1024 /* largest k accepted by dllm_select_unmask                */
@@ -208,6 +215,31 @@ dllm_status dllm_masked_logits_window(const uint16_t* H, const uint8_t* M, const
                                       float* entropy, float* margin, int32_t* row_idx,
                                       int32_t* seq_off, int32_t* count, void* ws,
                                       size_t ws_bytes, void* stream);
+
+/*
+ * dllm_prepare_rows / dllm_masked_logits_prepared - dllm_masked_logits in two calls, so
+ * that the input staging of one step (compaction of the mask and the gather of the masked
+ * rows of H into the workspace, reading H and M from device or page-locked host memory)
+ * can run on another stream while the previous step's GEMM runs.
+ *
+ * dllm_prepare_rows runs a1 (with optional windows, as in dllm_mask_compact_window) and
+ * the gather into `ws`; dllm_masked_logits_prepared then runs a2-a4 on the rows prepared in
+ * the same `ws` (it reads only `count` of the compaction outputs; row_idx and seq_off stay
+ * for dllm_select_unmask).  Both calls take the same B, L, d, V and a workspace of
+ * dllm_workspace_bytes(B, L, d, V); the caller orders the second after the first (same
+ * stream, or an event) and does not reuse `ws` for another preparation until the second
+ * has run.  Arguments, outputs and errors otherwise as in dllm_masked_logits_window /
+ * dllm_masked_logits_ex.
+ */
+dllm_status dllm_prepare_rows(const uint16_t* H, const uint8_t* M, int32_t B, int32_t L,
+                              int32_t d, int32_t V, const int32_t* win_lo,
+                              const int32_t* win_hi, int32_t* row_idx, int32_t* seq_off,
+                              int32_t* count, void* ws, size_t ws_bytes, void* stream);
+dllm_status dllm_masked_logits_prepared(const uint16_t* W, int32_t B, int32_t L, int32_t d,
+                                        int32_t V, uint32_t stats, int32_t* tok, float* conf,
+                                        float* lse, float* entropy, float* margin,
+                                        const int32_t* count, void* ws, size_t ws_bytes,
+                                        void* stream);
 
 /*
  * dllm_masked_partials - one vocabulary shard of a vocabulary-parallel LM head.

@@ -23,7 +23,7 @@ from . import _abi
 __all__ = [
     "DllmError", "lib", "version", "workspace_bytes", "mask_compact", "mask_compact_noalloc",
     "masked_logits", "masked_logits_ex", "select_unmask_ex", "STAT_ENTROPY", "STAT_MARGIN",
-    "masked_partials", "lse_merge",
+    "masked_partials", "lse_merge", "prepare_rows", "masked_logits_prepared",
     "select_unmask", "decode_step", "get_status", "debug_lmhead_logits", "debug_lse_merge",
     "debug_set_gemm_variant",
     "prof_begin", "prof_end", "DecodeStep", "MAX_K",
@@ -35,7 +35,8 @@ STAT_MARGIN = 2
 
 STATUS = {0: "DLLM_OK", -1: "DLLM_ERR_NULL", -2: "DLLM_ERR_ALIGN", -3: "DLLM_ERR_SHAPE",
           -4: "DLLM_ERR_WORKSPACE", -5: "DLLM_ERR_CUDA", -6: "DLLM_ERR_TIMEOUT",
-          -7: "DLLM_ERR_DEVICE", -8: "DLLM_ERR_BOUNDS", -9: "DLLM_ERR_SCRATCH"}
+          -7: "DLLM_ERR_DEVICE", -8: "DLLM_ERR_BOUNDS", -9: "DLLM_ERR_SCRATCH",
+          -10: "DLLM_ERR_MEMORY"}
 
 
 class DllmError(RuntimeError):
@@ -54,11 +55,15 @@ def _check(status: int, where: str) -> None:
         raise DllmError(status, where)
 
 
-def _ptr(t: torch.Tensor | None, dtype: torch.dtype | None = None, name: str = "") -> ctypes.c_void_p:
+def _ptr(t: torch.Tensor | None, dtype: torch.dtype | None = None, name: str = "",
+         host_ok: bool = False) -> ctypes.c_void_p:
+    """Device pointer of a tensor; with host_ok, a page-locked CPU tensor is also accepted
+    (the library reads it over the bus; only the step inputs H and M allow this)."""
     if t is None:
         return ctypes.c_void_p(None)
-    if not t.is_cuda:
-        raise ValueError(f"{name}: expected a CUDA tensor")
+    if not t.is_cuda and not (host_ok and t.is_pinned()):
+        raise ValueError(f"{name}: expected a CUDA tensor" +
+                         (" or a page-locked (pinned) CPU tensor" if host_ok else ""))
     if not t.is_contiguous():
         raise ValueError(f"{name}: expected a contiguous tensor")
     if dtype is not None and t.dtype != dtype:
@@ -118,7 +123,8 @@ def masked_logits(H, M, W, tok, conf, lse, row_idx, seq_off, count, ws, stream=N
     B, L = M.shape
     V, d = W.shape
     _check(lib().dllm_masked_logits(
-        _ptr(H, torch.bfloat16, "H"), _ptr(M, torch.uint8, "M"), _ptr(W, torch.bfloat16, "W"),
+        _ptr(H, torch.bfloat16, "H", True), _ptr(M, torch.uint8, "M", True),
+        _ptr(W, torch.bfloat16, "W"),
         B, L, d, V, _ptr(tok, torch.int32, "tok"), _ptr(conf, torch.float32, "conf"),
         _ptr(lse, torch.float32, "lse"), _ptr(row_idx, torch.int32, "row_idx"),
         _ptr(seq_off, torch.int32, "seq_off"), _ptr(count, torch.int32, "count"),
@@ -139,14 +145,40 @@ def masked_logits_ex(H, M, W, stats, tok, conf, lse, entropy, margin, row_idx, s
               _ptr(margin, torch.float32, "margin"), _ptr(row_idx, torch.int32, "row_idx"),
               _ptr(seq_off, torch.int32, "seq_off"), _ptr(count, torch.int32, "count"),
               _ptr(ws, None, "ws"), ws.numel() * ws.element_size(), _stream(stream))
-    ins = (_ptr(H, torch.bfloat16, "H"), _ptr(M, torch.uint8, "M"), _ptr(W, torch.bfloat16, "W"),
-           B, L, d, V)
+    ins = (_ptr(H, torch.bfloat16, "H", True), _ptr(M, torch.uint8, "M", True),
+           _ptr(W, torch.bfloat16, "W"), B, L, d, V)
     if win_lo is None and win_hi is None:
         _check(lib().dllm_masked_logits_ex(*ins, stats, *common), "dllm_masked_logits_ex")
     else:
         _check(lib().dllm_masked_logits_window(*ins, _ptr(win_lo, torch.int32, "win_lo"),
                                                _ptr(win_hi, torch.int32, "win_hi"), stats,
                                                *common), "dllm_masked_logits_window")
+
+
+def prepare_rows(H, M, d, V, row_idx, seq_off, count, ws, stream=None, win_lo=None,
+                 win_hi=None) -> None:
+    """First half of masked_logits: compaction of M (in the windows, if given) and the gather
+    of the masked rows of H into ``ws``.  H and M may be page-locked CPU tensors (read over
+    the bus: only the mask and the masked rows move)."""
+    B, L = M.shape
+    _check(lib().dllm_prepare_rows(
+        _ptr(H, torch.bfloat16, "H", True), _ptr(M, torch.uint8, "M", True), B, L, d, V,
+        _ptr(win_lo, torch.int32, "win_lo"), _ptr(win_hi, torch.int32, "win_hi"),
+        _ptr(row_idx, torch.int32, "row_idx"), _ptr(seq_off, torch.int32, "seq_off"),
+        _ptr(count, torch.int32, "count"), _ptr(ws, None, "ws"), ws.numel() * ws.element_size(),
+        _stream(stream)), "dllm_prepare_rows")
+
+
+def masked_logits_prepared(W, B, L, stats, tok, conf, lse, entropy, margin, count, ws,
+                           stream=None) -> None:
+    """Second half of masked_logits: the GEMM and its statistics on rows prepared in ``ws``."""
+    V, d = W.shape
+    _check(lib().dllm_masked_logits_prepared(
+        _ptr(W, torch.bfloat16, "W"), B, L, d, V, stats, _ptr(tok, torch.int32, "tok"),
+        _ptr(conf, torch.float32, "conf"), _ptr(lse, torch.float32, "lse"),
+        _ptr(entropy, torch.float32, "entropy"), _ptr(margin, torch.float32, "margin"),
+        _ptr(count, torch.int32, "count"), _ptr(ws, None, "ws"), ws.numel() * ws.element_size(),
+        _stream(stream)), "dllm_masked_logits_prepared")
 
 
 def masked_partials(H, M, W_shard, v_offset, stats, part_m, part_s, part_a, part_t, part_m2,
@@ -157,7 +189,7 @@ def masked_partials(H, M, W_shard, v_offset, stats, part_m, part_s, part_a, part
     B, L = M.shape
     V_shard, d = W_shard.shape
     _check(lib().dllm_masked_partials(
-        _ptr(H, torch.bfloat16, "H"), _ptr(M, torch.uint8, "M"),
+        _ptr(H, torch.bfloat16, "H", True), _ptr(M, torch.uint8, "M", True),
         _ptr(W_shard, torch.bfloat16, "W_shard"), B, L, d, V_shard, int(v_offset),
         _ptr(win_lo, torch.int32, "win_lo"), _ptr(win_hi, torch.int32, "win_hi"), stats,
         _ptr(part_m, torch.float32, "part_m"), _ptr(part_s, torch.float32, "part_s"),
@@ -218,7 +250,8 @@ def decode_step(H, M, W, k, tok, conf, lse, row_idx, seq_off, count, idx, n_sel,
     fn, name = ((lib().dllm_decode_block_step, "dllm_decode_block_step") if block_only
                 else (lib().dllm_decode_step, "dllm_decode_step"))
     _check(fn(
-        _ptr(H, torch.bfloat16, "H"), _ptr(M, torch.uint8, "M"), _ptr(W, torch.bfloat16, "W"),
+        _ptr(H, torch.bfloat16, "H", True), _ptr(M, torch.uint8, "M", True),
+        _ptr(W, torch.bfloat16, "W"),
         B, L, d, V, k, _ptr(win_lo, torch.int32, "win_lo"), _ptr(win_hi, torch.int32, "win_hi"),
         _ptr(tok, torch.int32, "tok"), _ptr(conf, torch.float32, "conf"),
         _ptr(lse, torch.float32, "lse"), _ptr(row_idx, torch.int32, "row_idx"),
@@ -291,15 +324,28 @@ class DecodeStep:
         self.row_idx = torch.empty(n, **i32)
         self.seq_off = torch.empty(B + 1, **i32)
         self.count = torch.empty(4, **i32)          # 16 bytes: keeps the next buffer aligned
-        self.idx = torch.empty(B, k, **i32)
-        self.n_sel = torch.empty(B, **i32)
-        self.tok_sel = torch.empty(B, k, **i32)
-        self.conf_sel = torch.empty(B, k, dtype=torch.float32, device=self.device)
+        # the selection outputs share one buffer (each part starts 16-byte aligned), so that
+        # one copy brings a step's whole selection back to the host
+        self._sel_parts = [B * k, B, B * k, B * k]            # idx, n_sel, tok_sel, conf_sel
+        self._sel_off = [0]
+        for n_part in self._sel_parts:
+            self._sel_off.append(self._sel_off[-1] + (n_part + 3) // 4 * 4)
+        self.sel_buf = torch.empty(self._sel_off[-1], **i32)
+        self.idx, self.n_sel, self.tok_sel, self.conf_sel = self._sel_views(self.sel_buf)
         nbytes = workspace_bytes(B, L, d, V)
         if nbytes == 0:
             raise ValueError("invalid shapes (d must be a positive multiple of 64)")
         self.ws = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
         self._host = None
+
+    def _sel_views(self, buf):
+        """idx [B, k], n_sel [B], tok_sel [B, k] (int32) and conf_sel [B, k] (float32) views
+        of a selection buffer laid out like ``sel_buf`` (device or host)."""
+        B, k = self.B, self.k
+        o = self._sel_off
+        return (buf[o[0]:o[0] + B * k].view(B, k), buf[o[1]:o[1] + B],
+                buf[o[2]:o[2] + B * k].view(B, k),
+                buf[o[3]:o[3] + B * k].view(torch.float32).view(B, k))
 
     def run(self, H, M, W, win_lo=None, win_hi=None, stream=None, block_only=False) -> dict:
         """One step on device tensors.  block_only=True (windows required): logits for the
@@ -314,20 +360,16 @@ class DecodeStep:
     # -- end-to-end from host memory ---------------------------------------------------------
     def _host_buffers(self):
         if self._host is None:
-            B, L, d, k = self.B, self.L, self.d, self.k
-            pin = dict(pin_memory=True)
+            B, L, d = self.B, self.L, self.d
             self._host = dict(
                 H=torch.empty(B * L, d, dtype=torch.bfloat16, device=self.device),
                 M=torch.empty(B, L, dtype=torch.uint8, device=self.device),
-                idx=torch.empty(B, k, dtype=torch.int32, **pin),
-                n_sel=torch.empty(B, dtype=torch.int32, **pin),
-                tok_sel=torch.empty(B, k, dtype=torch.int32, **pin),
-                conf_sel=torch.empty(B, k, dtype=torch.float32, **pin))
+                sel=torch.empty(self.sel_buf.numel(), dtype=torch.int32, pin_memory=True))
         return self._host
 
     def run_host(self, H_host, M_host, W, win_lo=None, win_hi=None, stream=None,
                  block_only=False) -> dict:
-        """One step from pinned host H and M: copy them in, run, copy the selection back.
+        """One step from host H and M: copy them in, run, copy the selection back.
 
         W (the resident vocabulary projection) and the windows are device tensors.  Returns
         host tensors idx, n_sel, tok_sel, conf_sel; synchronises the stream.
@@ -338,83 +380,105 @@ class DecodeStep:
             hb["H"].copy_(H_host, non_blocking=True)
             hb["M"].copy_(M_host, non_blocking=True)
             self.run(hb["H"], hb["M"], W, win_lo, win_hi, s, block_only)
-            hb["idx"].copy_(self.idx, non_blocking=True)
-            hb["n_sel"].copy_(self.n_sel, non_blocking=True)
-            hb["tok_sel"].copy_(self.tok_sel, non_blocking=True)
-            hb["conf_sel"].copy_(self.conf_sel, non_blocking=True)
+            hb["sel"].copy_(self.sel_buf, non_blocking=True)
         s.synchronize()
-        return dict(idx=hb["idx"], n_sel=hb["n_sel"], tok_sel=hb["tok_sel"], conf_sel=hb["conf_sel"])
+        return dict(zip(("idx", "n_sel", "tok_sel", "conf_sel"), self._sel_views(hb["sel"])))
 
     def run_host_pipeline(self, batches, W, win_lo=None, win_hi=None, stream=None,
-                          copy_stream=None, block_only=False):
-        """Decode steps over host batches [(H_host, M_host), ...] (pinned), with the copy of
-        batch i+1 into the device overlapping the step of batch i.
+                          prep_stream=None, block_only=False):
+        """Decode steps over host batches [(H_host, M_host), ...] in page-locked host memory,
+        with the input staging of step i+1 overlapping step i.
 
-        Two device input buffers alternate; a copy stream loads batch i+1 while the compute
-        stream runs step i and copies its selection back to pinned host memory.  Yields, per
-        step, host tensors idx, n_sel, tok_sel, conf_sel (valid until the next iteration).
+        Staging (``prepare_rows``: compaction of the mask and the gather of only the masked
+        rows of H, both read straight from host memory over the bus) runs on a second
+        stream into one of two workspaces, while the compute stream runs the previous
+        step's GEMM and selection on the other (``masked_logits_prepared``,
+        ``select_unmask``) and copies the selection back to page-locked host memory.
+        Yields, per step, host tensors idx, n_sel, tok_sel, conf_sel (valid until the next
+        iteration).  Each batch's H_host and M_host must stay valid and unchanged until its
+        step has been yielded.
         """
-        B, L, d, k = self.B, self.L, self.d, self.k
+        B, L, d, V, k = self.B, self.L, self.d, self.V, self.k
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
-        cs = copy_stream if copy_stream is not None else torch.cuda.Stream(self.device)
+        ps = prep_stream if prep_stream is not None else torch.cuda.Stream(self.device)
         if getattr(self, "_pipe", None) is None:
             pin = dict(pin_memory=True)
+            i32 = dict(dtype=torch.int32, device=self.device)
             self._pipe = dict(
-                H=[torch.empty(B * L, d, dtype=torch.bfloat16, device=self.device) for _ in range(2)],
-                M=[torch.empty(B, L, dtype=torch.uint8, device=self.device) for _ in range(2)],
-                out=[dict(idx=torch.empty(B, k, dtype=torch.int32, **pin),
-                          n_sel=torch.empty(B, dtype=torch.int32, **pin),
-                          tok_sel=torch.empty(B, k, dtype=torch.int32, **pin),
-                          conf_sel=torch.empty(B, k, dtype=torch.float32, **pin)) for _ in range(2)])
+                ws=[self.ws, torch.empty_like(self.ws)],
+                row_idx=[self.row_idx, torch.empty(B * L, **i32)],
+                seq_off=[self.seq_off, torch.empty(B + 1, **i32)],
+                count=[self.count, torch.empty(4, **i32)],
+                out_buf=[torch.empty(self.sel_buf.numel(), dtype=torch.int32, **pin)
+                         for _ in range(2)],
+                copy_stream=torch.cuda.Stream(self.device))
+            self._pipe["out"] = [dict(zip(("idx", "n_sel", "tok_sel", "conf_sel"),
+                                          self._sel_views(b))) for b in self._pipe["out_buf"]]
         pb = self._pipe
-        loaded = [torch.cuda.Event() for _ in range(2)]
-        freed = [torch.cuda.Event() for _ in range(2)]
+        cs = pb["copy_stream"]
+        prepped = [torch.cuda.Event() for _ in range(2)]
+        used = [torch.cuda.Event() for _ in range(2)]
+        selected = [torch.cuda.Event() for _ in range(2)]
         done = [torch.cuda.Event() for _ in range(2)]
+        pw = (win_lo, win_hi) if block_only else (None, None)
 
-        def load(i, Hh, Mh):
+        def prep(i, Hh, Mh):
+            if not (Hh.is_pinned() and Mh.is_pinned()):
+                raise ValueError("host batches must be page-locked (pinned) CPU tensors")
             b = i & 1
-            with torch.cuda.stream(cs):
+            with torch.cuda.stream(ps):
                 if i >= 2:
-                    cs.wait_event(freed[b])          # step i-2 no longer reads this buffer
-                pb["H"][b].copy_(Hh, non_blocking=True)
-                pb["M"][b].copy_(Mh, non_blocking=True)
-                loaded[b].record(cs)
+                    ps.wait_event(used[b])           # step i-2 no longer reads this workspace
+                prepare_rows(Hh, Mh, d, V, pb["row_idx"][b], pb["seq_off"][b], pb["count"][b],
+                             pb["ws"][b], ps, *pw)
+                prepped[b].record(ps)
+
+        def compute(i):
+            b = i & 1
+            with torch.cuda.stream(s):
+                s.wait_event(prepped[b])
+                masked_logits_prepared(W, B, L, 0, self.tok, self.conf, self.lse, None, None,
+                                       pb["count"][b], pb["ws"][b], s)
+                if i >= 1:
+                    s.wait_event(done[(i - 1) & 1])  # step i-1's selection has been copied out
+                select_unmask(self.conf, pb["row_idx"][b], pb["seq_off"][b], B, L, k, self.idx,
+                              self.n_sel, win_lo, win_hi, self.tok, self.tok_sel, self.conf_sel, s)
+                used[b].record(s)
+                selected[b].record(s)
+            # the selection goes back on the copy stream: the next step's GEMM does not wait
+            with torch.cuda.stream(cs):
+                cs.wait_event(selected[b])
+                pb["out_buf"][b].copy_(self.sel_buf, non_blocking=True)
+                done[b].record(cs)
 
         it = iter(batches)
-        first = next(it, None)
-        if first is None:
+        cur = next(it, None)
+        if cur is None:
             return
-        load(0, *first)
+        prep(0, *cur)
         i = 0
         pending = None
-        nxt = next(it, None)
         while True:
-            b = i & 1
+            nxt = next(it, None)
             if nxt is not None:
-                load(i + 1, *nxt)                    # overlaps step i below
-            with torch.cuda.stream(s):
-                s.wait_event(loaded[b])
-                self.run(pb["H"][b], pb["M"][b], W, win_lo, win_hi, s, block_only)
-                freed[b].record(s)
-                o = pb["out"][b]
-                o["idx"].copy_(self.idx, non_blocking=True)
-                o["n_sel"].copy_(self.n_sel, non_blocking=True)
-                o["tok_sel"].copy_(self.tok_sel, non_blocking=True)
-                o["conf_sel"].copy_(self.conf_sel, non_blocking=True)
-                done[b].record(s)
+                prep(i + 1, *nxt)                    # overlaps the compute of step i
+            compute(i)
             if pending is not None:
                 done[pending].synchronize()
                 yield pb["out"][pending]
-            pending = b
+            pending = i & 1
             if nxt is None:
                 break
-            nxt = next(it, None)
             i += 1
         done[pending].synchronize()
         yield pb["out"][pending]
+
+    def h2d_bytes_zero_copy(self, count: int) -> int:
+        """Bytes one pipelined step reads from host memory: the mask and the masked rows."""
+        return self.B * self.L + count * self.d * 2
 
     def h2d_bytes(self) -> int:
         return self.B * self.L * self.d * 2 + self.B * self.L
 
     def d2h_bytes(self) -> int:
-        return self.B * self.k * 4 * 3 + self.B * 4
+        return self.sel_buf.numel() * 4

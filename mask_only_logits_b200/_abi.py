@@ -27,6 +27,9 @@ PROTOTYPES = {
     "dllm_masked_logits_window": (_st, [_p, _p, _p, _i32, _i32, _i32, _i32, _p, _p,
                                         ctypes.c_uint32, _p, _p, _p, _p, _p, _p, _p, _p, _p, _sz,
                                         _p]),
+    "dllm_prepare_rows": (_st, [_p, _p, _i32, _i32, _i32, _i32, _p, _p, _p, _p, _p, _p, _sz, _p]),
+    "dllm_masked_logits_prepared": (_st, [_p, _i32, _i32, _i32, _i32, ctypes.c_uint32, _p, _p, _p,
+                                          _p, _p, _p, _p, _sz, _p]),
     "dllm_masked_partials": (_st, [_p, _p, _p, _i32, _i32, _i32, _i32, _i32, _p, _p,
                                    ctypes.c_uint32, _p, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
     "dllm_lse_merge": (_st, [_p, _p, _p, _p, _p, ctypes.c_int64, _i32, _p, _i32, ctypes.c_uint32,

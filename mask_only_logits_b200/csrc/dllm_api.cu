@@ -213,6 +213,27 @@ WsLayout ws_layout(int B, int L, int d, int V) {
   return w;
 }
 
+// A step input (H or M) may live in device memory or in page-locked host memory that the
+// device can read over PCIe (zero-copy: only the bytes the kernels touch cross the bus,
+// e.g. just the masked rows of H).  Resolves the pointer the kernels use; pageable host
+// memory is rejected (DLLM_ERR_MEMORY) because the device cannot read it.
+dllm_status resolve_input(const void* p, const void** dev) {
+  cudaPointerAttributes at{};
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();                       // clear the sticky-free error of the query
+    return DLLM_ERR_MEMORY;
+  }
+  if (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) {
+    *dev = p;
+    return DLLM_OK;
+  }
+  if (at.type == cudaMemoryTypeHost && at.devicePointer != nullptr) {
+    *dev = at.devicePointer;
+    return aligned16(*dev) ? DLLM_OK : DLLM_ERR_ALIGN;
+  }
+  return DLLM_ERR_MEMORY;
+}
+
 bool shapes_ok(int B, int L) {
   return B >= 1 && L >= 1 && static_cast<long long>(B) * L < (1ll << 31);
 }
@@ -260,8 +281,9 @@ struct LogitsArgs {
   int a_offset = 0;
 };
 
-dllm_status validate_logits(const LogitsArgs& a, bool debug) {
-  if (!a.H || !a.M || !a.W || !a.row_idx || !a.seq_off || !a.count || !a.ws) return DLLM_ERR_NULL;
+dllm_status validate_logits(const LogitsArgs& a, bool debug, bool prepared = false) {
+  if ((!prepared && (!a.H || !a.M || !a.row_idx || !a.seq_off)) || !a.W || !a.count || !a.ws)
+    return DLLM_ERR_NULL;
   const bool shard = a.raw.m != nullptr;
   if (shard) {
     if (!a.raw.s || !a.raw.a) return DLLM_ERR_NULL;
@@ -287,14 +309,39 @@ dllm_status validate_logits(const LogitsArgs& a, bool debug) {
   return DLLM_OK;
 }
 
-dllm_status run_logits(const LogitsArgs& a, bool debug) {
-  dllm_status st = validate_logits(a, debug);
+// a1 + gather: compaction of the mask (in the windows, if any) and the copy of the masked
+// rows of H into the workspace's dense Hm; H and M may be page-locked host memory.
+dllm_status prepare_rows(const LogitsArgs& a, const DeviceState& ds, const WsLayout& w) {
+  const void* Hd = nullptr;
+  const void* Md = nullptr;
+  dllm_status st = resolve_input(a.H, &Hd);
+  if (st != DLLM_OK) return st;
+  if ((st = resolve_input(a.M, &Md)) != DLLM_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(a.ws);
+  int* tiles = reinterpret_cast<int*>(ws + w.tiles_off);
+  uint16_t* Hm = reinterpret_cast<uint16_t*>(ws + w.hm_off);
+  int* ctr = reinterpret_cast<int*>(ws + w.ctr_off);
+  const long long n = static_cast<long long>(a.B) * a.L;
+  if ((st = launch_compact(static_cast<const uint8_t*>(Md), a.B, a.L, a.win_lo, a.win_hi, a.row_idx,
+                           a.seq_off, a.count, tiles, ds.status, a.s)) != DLLM_OK)
+    return st;
+  if (launch_pdl(gather_rows_kernel, dim3(ds.sms * 4), dim3(kGatherThreads), 0, a.s,
+                 static_cast<const uint16_t*>(Hd), (const int*)a.row_idx, (const int*)a.count, n,
+                 a.d, Hm, ctr, w.n_ctr, ds.status) != cudaSuccess)
+    return DLLM_ERR_CUDA;
+  count_launch();
+  return DLLM_OK;
+}
+
+// skip_prepare: the rows were prepared by an earlier dllm_prepare_rows into the same
+// workspace (H and M are then not read).
+dllm_status run_logits(const LogitsArgs& a, bool debug, bool skip_prepare = false) {
+  dllm_status st = validate_logits(a, debug, skip_prepare);
   if (st != DLLM_OK) return st;
   DeviceState* ds = nullptr;
   if ((st = device_state(&ds)) != DLLM_OK) return st;
   const WsLayout w = ws_layout(a.B, a.L, a.d, a.V);
   uint8_t* ws = static_cast<uint8_t*>(a.ws);
-  int* tiles = reinterpret_cast<int*>(ws + w.tiles_off);
   uint16_t* Hm = reinterpret_cast<uint16_t*>(ws + w.hm_off);
   float* pm = reinterpret_cast<float*>(ws + w.pm_off);
   float* ps = reinterpret_cast<float*>(ws + w.ps_off);
@@ -326,15 +373,9 @@ dllm_status run_logits(const LogitsArgs& a, bool debug) {
     if (need > w.part_cap) return DLLM_ERR_WORKSPACE;                  // cannot happen on B200
   }
 
-  if ((st = launch_compact(a.M, a.B, a.L, a.win_lo, a.win_hi, a.row_idx, a.seq_off, a.count, tiles,
-                           ds->status, a.s)) != DLLM_OK)
-    return st;
-
-  if (launch_pdl(gather_rows_kernel, dim3(ds->sms * 4), dim3(kGatherThreads), 0, a.s, a.H,
-                 (const int*)a.row_idx, (const int*)a.count, n, a.d, Hm, ctr, w.n_ctr,
-                 ds->status) != cudaSuccess)
-    return DLLM_ERR_CUDA;
-  count_launch();
+  if (!skip_prepare) {
+    if ((st = prepare_rows(a, *ds, w)) != DLLM_OK) return st;
+  }
 
   CUtensorMap tmA, tmB;
   if (make_tmap(&tmA, Hm, static_cast<uint64_t>(n), a.d, 128) != DLLM_OK) return DLLM_ERR_CUDA;
@@ -480,6 +521,7 @@ const char* dllm_status_string(dllm_status s) {
     case DLLM_ERR_DEVICE: return "device is not an sm_100 GPU";
     case DLLM_ERR_BOUNDS: return "a device-side bound check failed";
     case DLLM_ERR_SCRATCH: return "B*L exceeds the fixed scratch of the allocation-free entry point";
+    case DLLM_ERR_MEMORY: return "an input is neither device memory nor page-locked host memory";
     default: return "unknown status";
   }
 }
@@ -601,6 +643,38 @@ dllm_status dllm_lse_merge(const float* part_m, const float* part_s, const int32
   if (e != cudaSuccess) return DLLM_ERR_CUDA;
   count_launch();
   return DLLM_OK;
+}
+
+dllm_status dllm_prepare_rows(const uint16_t* H, const uint8_t* M, int32_t B, int32_t L, int32_t d,
+                              int32_t V, const int32_t* win_lo, const int32_t* win_hi,
+                              int32_t* row_idx, int32_t* seq_off, int32_t* count, void* ws,
+                              size_t ws_bytes, void* stream) {
+  const dllm::NvtxRange nvtx_range("dllm_prepare_rows");
+  if (!H || !M || !row_idx || !seq_off || !count || !ws) return DLLM_ERR_NULL;
+  if ((win_lo == nullptr) != (win_hi == nullptr)) return DLLM_ERR_NULL;
+  if (!shapes_ok(B, L) || V < 1 || d < DLLM_D_MULTIPLE || d % DLLM_D_MULTIPLE != 0) return DLLM_ERR_SHAPE;
+  const void* ptrs[] = {H, M, row_idx, seq_off, count, ws, win_lo, win_hi};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return DLLM_ERR_ALIGN;
+  const WsLayout w = ws_layout(B, L, d, V);
+  if (ws_bytes < w.total) return DLLM_ERR_WORKSPACE;
+  DeviceState* ds = nullptr;
+  dllm_status st = device_state(&ds);
+  if (st != DLLM_OK) return st;
+  LogitsArgs a{H, M, nullptr, B, L, d, V, win_lo, win_hi, 0u, nullptr, nullptr, nullptr, nullptr, nullptr,
+               nullptr, row_idx, seq_off, count, ws, ws_bytes, static_cast<cudaStream_t>(stream)};
+  return prepare_rows(a, *ds, w);
+}
+
+dllm_status dllm_masked_logits_prepared(const uint16_t* W, int32_t B, int32_t L, int32_t d, int32_t V,
+                                        uint32_t stats, int32_t* tok, float* conf, float* lse,
+                                        float* entropy, float* margin, const int32_t* count,
+                                        void* ws, size_t ws_bytes, void* stream) {
+  const dllm::NvtxRange nvtx_range("dllm_masked_logits_prepared");
+  LogitsArgs a{nullptr, nullptr, W, B, L, d, V, nullptr, nullptr, stats, entropy, margin, tok, conf,
+               lse, nullptr, nullptr, nullptr, const_cast<int32_t*>(count), ws, ws_bytes,
+               static_cast<cudaStream_t>(stream)};
+  return run_logits(a, false, true);
 }
 
 dllm_status dllm_debug_lmhead_logits(const uint16_t* H, const uint8_t* M, const uint16_t* W,

@@ -210,7 +210,7 @@ def test_pair_variant_large(dl):
 
 
 def test_run_host_pipeline_matches_device_steps(dl):
-    """Overlapped copies must not mix batches: each yielded selection equals that batch's
+    """Overlapped staging must not mix batches: each yielded selection equals that batch's
     device-resident step."""
     cfg = WL.CONFIGS["cfg0"]
     inps = [WL.make_inputs(cfg, seed=s) for s in (0, 1, 2, 3, 4)]
@@ -228,3 +228,71 @@ def test_run_host_pipeline_matches_device_steps(dl):
     for (gi, gn, gt), (ei, en, et) in zip(got, expected):
         assert torch.equal(gi, ei) and torch.equal(gn, en) and torch.equal(gt, et)
     assert not all(torch.equal(got[0][0], g[0]) for g in got[1:])   # batches really differ
+
+
+def test_pinned_host_inputs_match_device(dl):
+    """H and the mask in page-locked host memory (read over the bus by the compaction and
+    gather kernels) give bit-identical results to the same inputs in device memory."""
+    for name, variant in (("cfg0", 0), ("cfg4", 0), ("cfg1_m64", 1)):
+        inp = WL.make_inputs(WL.CONFIGS[name], seed=1)
+        cfg = inp["cfg"]
+        dev = GU.to_device(inp)
+        dl.debug_set_gemm_variant(variant)
+        try:
+            step = dl.DecodeStep(cfg.B, cfg.L, cfg.d, cfg.V, cfg.k)
+            a = {k: v.clone() for k, v in step.run(dev["H"], dev["M"], dev["W"], dev["win_lo"],
+                                                   dev["win_hi"]).items()}
+            b = step.run(inp["H"].pin_memory(), inp["M"].pin_memory(), dev["W"], dev["win_lo"],
+                         dev["win_hi"])
+            torch.cuda.synchronize()
+            assert dl.get_status() == 0
+            c = int(a["count"][0])
+            assert int(b["count"][0]) == c
+            for key in ("tok", "conf", "lse", "row_idx"):
+                assert torch.equal(a[key][:c], b[key][:c]), (name, key)
+            for key in ("idx", "n_sel", "tok_sel", "conf_sel", "seq_off"):
+                assert torch.equal(a[key], b[key]), (name, key)
+        finally:
+            dl.debug_set_gemm_variant(0)
+
+
+def test_pageable_host_input_rejected(dl):
+    """Pageable host memory cannot be read by the kernels: rejected before any launch."""
+    import ctypes
+    inp = WL.make_inputs(WL.CONFIGS["cfg0"], seed=0)
+    cfg = inp["cfg"]
+    H_pageable = np.ascontiguousarray(WL.bf16_bits(inp["H"]))        # plain host memory
+    n = cfg.B * cfg.L
+    i32 = dict(dtype=torch.int32, device="cuda")
+    outs = [torch.empty(n, **i32), torch.empty(n, device="cuda"), torch.empty(n, device="cuda"),
+            torch.empty(n, **i32), torch.empty(cfg.B + 1, **i32), torch.empty(4, **i32)]
+    ws = torch.empty(dl.workspace_bytes(cfg.B, cfg.L, cfg.d, cfg.V), dtype=torch.uint8, device="cuda")
+    M, W = inp["M"].cuda(), inp["W"].cuda()
+    P = lambda t: ctypes.c_void_p(t.data_ptr())
+    st = dl.lib().dllm_masked_logits(ctypes.c_void_p(H_pageable.ctypes.data), P(M), P(W), cfg.B,
+                                     cfg.L, cfg.d, cfg.V, *[P(t) for t in outs], P(ws), ws.numel(),
+                                     ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == -10                                                   # DLLM_ERR_MEMORY
+    assert dl.get_status() == 0
+
+
+def test_host_pipeline_block_only_and_windows(dl):
+    """The two-stream pipeline with current-block-only steps and with selection windows."""
+    cfg = WL.custom_config(4, 1024, 128, 3000, 4, mask="semi_ar", block=32)
+    inps = [WL.make_inputs(cfg, seed=s) for s in (3, 4, 5)]
+    W = inps[0]["W"].cuda()
+    lo, hi = WL.make_windows(cfg)
+    lo_d, hi_d = torch.from_numpy(lo).cuda(), torch.from_numpy(hi).cuda()
+    for block_only in (False, True):
+        step = dl.DecodeStep(cfg.B, cfg.L, cfg.d, cfg.V, cfg.k)
+        expected = []
+        for inp in inps:
+            out = step.run(inp["H"].cuda(), inp["M"].cuda(), W, lo_d, hi_d, block_only=block_only)
+            expected.append((out["idx"].cpu().clone(), out["n_sel"].cpu().clone()))
+        batches = [(inp["H"].pin_memory(), inp["M"].pin_memory()) for inp in inps]
+        got = [(o["idx"].clone(), o["n_sel"].clone())
+               for o in step.run_host_pipeline(batches, W, lo_d, hi_d, block_only=block_only)]
+        assert len(got) == len(expected)
+        for (gi, gn), (ei, en) in zip(got, expected):
+            assert torch.equal(gi, ei) and torch.equal(gn, en)
+        assert dl.get_status() == 0
