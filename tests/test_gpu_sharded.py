@@ -146,3 +146,35 @@ def test_vocab_sharded_step_single_rank(dl):
     GU.check_selection_exact(out["idx"].cpu().numpy(), out["n_sel"].cpu().numpy(),
                              out["conf"][:c].cpu().numpy(), row_idx, seq_off, cfg.L, cfg.k,
                              None, None, O)
+
+
+def test_sharded_block_only_windows(dl):
+    """Vocabulary shards with current-block-only rows (windows applied at compaction)."""
+    cfg = WL.custom_config(4, 1024, 128, 3001, 4, mask="semi_ar", block=32)
+    inp = WL.make_inputs(cfg, seed=6)
+    lo, hi = WL.make_windows(cfg)
+    dev = GU.to_device(inp)
+    lo_d, hi_d = torch.from_numpy(lo).cuda(), torch.from_numpy(hi).cuda()
+    from mask_only_logits_b200.sharded import PartialLayout
+    S, n = 3, cfg.B * cfg.L
+    lay = PartialLayout(n, extended=False)
+    gathered = lay.empty(S, "cuda")
+    i32 = dict(dtype=torch.int32, device="cuda")
+    row_idx, seq_off, count = torch.empty(n, **i32), torch.empty(cfg.B + 1, **i32), torch.empty(4, **i32)
+    for j in range(S):
+        v0, v1 = D.shard_range(cfg.V, j, S)
+        ws = torch.empty(dl.workspace_bytes(cfg.B, cfg.L, cfg.d, v1 - v0), dtype=torch.uint8, device="cuda")
+        f = lay.fields_of(gathered[j])
+        dl.masked_partials(dev["H"], dev["M"], dev["W"][v0:v1].contiguous(), v0, 0, f["m"], f["s"],
+                           f["a"], None, None, row_idx, seq_off, count, ws, win_lo=lo_d, win_hi=hi_d)
+    gf = lay.fields_of(gathered)
+    tok, conf, lse = torch.empty(n, **i32), torch.empty(n, device="cuda"), torch.empty(n, device="cuda")
+    dl.lse_merge(gf["m"], gf["s"], gf["a"], None, None, lay.split_stride, S, count, n, 0, tok, conf, lse)
+    assert dl.get_status() == 0
+    c = int(count[0])
+    Mw = O.window_mask(inp["M"].numpy(), lo, hi)
+    ref = O.oracle_rows(WL.bf16_bits(inp["H"]), WL.bf16_bits(inp["W"]), Mw)
+    assert c == ref["count"] == cfg.B * 32
+    np.testing.assert_array_equal(row_idx[:c].cpu().numpy(), ref["row_idx"])
+    GU.check_rows(tok[:c].cpu().numpy(), conf[:c].cpu().numpy(), lse[:c].cpu().numpy(), ref,
+                  np.arange(c), "sharded-block")
