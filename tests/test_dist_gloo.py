@@ -149,3 +149,49 @@ def test_vocab_sharded_exchange_two_gloo_ranks():
         assert tok_ok
         assert e_lse < 1e-6 and e_conf < 1e-5, (e_lse, e_conf)     # fp32 packing of partials
         assert bounds == D.shard_range(1001, r, world)
+
+
+def _dead_rank_worker(rank: int, world: int, port: int, q):
+    """Rank 1 leaves before the step's exchange; rank 0 must get an error, not hang."""
+    import time
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    try:
+        from mask_only_logits_b200.sharded import PartialLayout, exchange_partials
+        dist = D.init_process_group("gloo", timeout_s=5)
+        dist.barrier()                                     # both ranks were up
+        if rank == 1:
+            q.put((rank, "left"))
+            q.close()
+            q.join_thread()                                # the message is out before dying
+            os._exit(0)                                    # dies between steps, no goodbye
+        lay = PartialLayout(64, extended=False)
+        local, gathered = lay.empty(None, "cpu").zero_(), lay.empty(world, "cpu")
+        t0 = time.monotonic()
+        try:
+            exchange_partials(local, gathered)
+            q.put((rank, "no error", time.monotonic() - t0))
+        except Exception as e:  # noqa: BLE001 - the collective must fail
+            q.put((rank, "raised", time.monotonic() - t0, type(e).__name__))
+    except Exception as e:  # noqa: BLE001
+        q.put((rank, "setup failed: " + repr(e)))
+
+
+@pytest.mark.timeout(300)
+def test_dead_rank_is_detected_by_the_exchange():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_dead_rank_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = {}
+    for _ in range(world):
+        item = q.get(timeout=240)
+        results[item[0]] = item
+    for p in procs:
+        p.join(timeout=60)
+    assert results[1][1] == "left", results[1]
+    assert results[0][1] == "raised", results[0]
+    assert results[0][2] < 120.0                           # within the group's timeout budget
