@@ -380,6 +380,8 @@ def main() -> None:
     ap.add_argument("--no-full-baseline", action="store_true",
                     help="skip timing the full-logits torch path the method replaces")
     ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--graph", action="store_true",
+                    help="time replays of the step captured in a CUDA graph (one launch per step)")
     ap.add_argument("--shard", default="replica", choices=["replica", "vocab"],
                     help="replica: one independent step per rank (weak scaling); vocab: one "
                          "step with W split by rows over the ranks (strong scaling)")
@@ -442,12 +444,24 @@ def main() -> None:
         torch.cuda.synchronize(dev)
 
     # ---- device-resident timed region: the steps alone ----
+    if args.graph:
+        step.capture(H, M, W, win_lo, win_hi, blk)
+        for _ in range(3):
+            step.replay(stream)
+        torch.cuda.synchronize(dev)
+
+    def one_step():
+        if args.graph:
+            step.replay(stream)
+        else:
+            step.run(H, M, W, win_lo, win_hi, stream, blk)
+
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev.index if dev.index is not None else 0) as clk:
         barrier()
         ev0.record(stream)
         for _ in range(args.steps):
-            step.run(H, M, W, win_lo, win_hi, stream, blk)
+            one_step()
         ev1.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
@@ -508,7 +522,7 @@ def main() -> None:
             metric=METRIC, value=rows_s, unit=UNIT, n_gpus=world, steps=args.steps,
             warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True, scaling="weak",
             vs_baseline=None, dtype="bf16", data="synthetic",
-            config=workload_config(cfg, count),
+            config=dict(workload_config(cfg, count), **({"launch": "CUDA graph replay"} if args.graph else {})),
             tflops=step_tflops, gbs=step_gbs,
             roofline_frac_step=roof / (ms_step / 1e3),
             roofline_ms=roof * 1e3,

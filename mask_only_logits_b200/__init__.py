@@ -358,6 +358,37 @@ class DecodeStep:
                     tok_sel=self.tok_sel, conf_sel=self.conf_sel)
 
     # -- end-to-end from host memory ---------------------------------------------------------
+    def capture(self, H, M, W, win_lo=None, win_hi=None, block_only=False):
+        """Capture one step on these device tensors into a CUDA graph.  ``replay()`` then
+        reruns the whole step (every kernel, with the programmatic-launch edges between them)
+        on whatever those tensors hold at replay time, for one launch of CPU work; the
+        outputs are this object's buffers as after ``run``.  Tensors must keep their
+        addresses while the graph is used."""
+        side = torch.cuda.Stream(self.device)
+        side.wait_stream(torch.cuda.current_stream(self.device))
+        with torch.cuda.stream(side):
+            for _ in range(2):                   # one-time device set-up happens outside capture
+                self.run(H, M, W, win_lo, win_hi, side, block_only)
+        torch.cuda.current_stream(self.device).wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, capture_error_mode="thread_local"):
+            self.run(H, M, W, win_lo, win_hi, None, block_only)
+        self._graph = graph
+        return graph
+
+    def replay(self, stream=None) -> dict:
+        """Rerun the captured step (``capture`` first) on the current (or given) stream."""
+        if getattr(self, "_graph", None) is None:
+            raise RuntimeError("capture() a step first")
+        if stream is None:
+            self._graph.replay()
+        else:
+            with torch.cuda.stream(stream):
+                self._graph.replay()
+        return dict(tok=self.tok, conf=self.conf, lse=self.lse, row_idx=self.row_idx,
+                    seq_off=self.seq_off, count=self.count[:1], idx=self.idx, n_sel=self.n_sel,
+                    tok_sel=self.tok_sel, conf_sel=self.conf_sel)
+
     def _host_buffers(self):
         if self._host is None:
             B, L, d = self.B, self.L, self.d

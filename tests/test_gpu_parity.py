@@ -169,6 +169,8 @@ def test_block_only_random_windows(dl, B, L, d, V, k, r):
     (1, 2048, 128, 5000, 16, "bernoulli", 1.0),      # 8 m-tiles of 256 rows
     (1, 1000, 64, 37800, 32, "bernoulli", 1.0),      # remainder holders (both variants)
     (1, 12000, 64, 3000, 8, "bernoulli", 0.08),      # sparse mask, few m-tiles of a long L
+    (1, 3840, 64, 20000, 8, "bernoulli", 1.0),       # 30 m-tiles: tail split 18 + 12
+    (1, 13300, 64, 5000, 8, "bernoulli", 1.0),       # 104 m-tiles: 2 full groups + 18 + 12
 ])
 def test_edge_shapes(dl, B, L, d, V, k, mask, r):
     cfg = WL.custom_config(B, L, d, V, k, mask=mask, r=r)
@@ -296,3 +298,32 @@ def test_host_pipeline_block_only_and_windows(dl):
         for (gi, gn), (ei, en) in zip(got, expected):
             assert torch.equal(gi, ei) and torch.equal(gn, en)
         assert dl.get_status() == 0
+
+
+@pytest.mark.parametrize("name,block_only", [("cfg0", False), ("cfg4_block", True), ("cfg1", False)])
+def test_cuda_graph_replay_matches_eager(dl, name, block_only):
+    """A captured step replayed on new contents of its input buffers gives the eager step's
+    results bit for bit (same kernels, same launch shapes)."""
+    cfg = WL.CONFIGS[name]
+    inps = [WL.make_inputs(cfg, seed=s) for s in (0, 1)]
+    W = inps[0]["W"].cuda()
+    H = inps[0]["H"].cuda()
+    M = inps[0]["M"].cuda()
+    lo = None if inps[0]["win_lo"] is None else torch.from_numpy(inps[0]["win_lo"]).cuda()
+    hi = None if inps[0]["win_hi"] is None else torch.from_numpy(inps[0]["win_hi"]).cuda()
+    eager = dl.DecodeStep(cfg.B, cfg.L, cfg.d, cfg.V, cfg.k)
+    graphed = dl.DecodeStep(cfg.B, cfg.L, cfg.d, cfg.V, cfg.k)
+    graphed.capture(H, M, W, lo, hi, block_only=block_only)
+    for inp in inps:
+        H.copy_(inp["H"])
+        M.copy_(inp["M"])
+        e = {k: v.clone() for k, v in eager.run(H, M, W, lo, hi, block_only=block_only).items()}
+        g = graphed.replay()
+        torch.cuda.synchronize()
+        assert dl.get_status() == 0
+        c = int(e["count"][0])
+        assert int(g["count"][0]) == c
+        for key in ("tok", "conf", "lse", "row_idx"):
+            assert torch.equal(e[key][:c], g[key][:c]), key
+        for key in ("idx", "n_sel", "tok_sel", "conf_sel"):
+            assert torch.equal(e[key], g[key]), key
