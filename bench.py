@@ -479,6 +479,9 @@ def main() -> None:
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
     t_ms, gemm_ms = D.max_over_ranks([t_ms, gemm_ms], dev)
+    # rows processed by the whole job per step: every rank's own batch (seeded per rank, so
+    # Bernoulli masks give each rank its own count)
+    job_rows = int(round(D.sum_over_ranks([count], dev)[0]))
     full_base = (full_logits_baseline(H, M, W, cfg.k, win_lo, win_hi, blk, dev)
                  if world == 1 and not args.no_full_baseline else None)
 
@@ -510,7 +513,7 @@ def main() -> None:
         peaks = load_peaks()
         a = algorithmic(cfg, count)
         ms_step = t_ms / args.steps
-        rows_s = count * world * args.steps / (t_ms / 1e3)
+        rows_s = job_rows * args.steps / (t_ms / 1e3)
         gemm_avg_s = gemm_ms / max(1, gemm_launches) / 1e3
         roof = roofline_s(cfg, count, peaks)
         step_tflops = a["flops"] / (ms_step / 1e3) / 1e12
@@ -522,7 +525,8 @@ def main() -> None:
             metric=METRIC, value=rows_s, unit=UNIT, n_gpus=world, steps=args.steps,
             warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True, scaling="weak",
             vs_baseline=None, dtype="bf16", data="synthetic",
-            config=dict(workload_config(cfg, count), **({"launch": "CUDA graph replay"} if args.graph else {})),
+            config=dict(workload_config(cfg, count), masked_rows_all_ranks=job_rows,
+                        **({"launch": "CUDA graph replay"} if args.graph else {})),
             tflops=step_tflops, gbs=step_gbs,
             roofline_frac_step=roof / (ms_step / 1e3),
             roofline_ms=roof * 1e3,
@@ -532,7 +536,7 @@ def main() -> None:
                         full_logits_fp32_bytes=int(full_logits),
                         note="peak = torch allocations of the step (outputs + workspace) over the "
                              "resident inputs; full_logits_fp32_bytes = B*L*V fp32 logits"),
-            e2e=dict(value=count * world * e2e_steps / (e2e_ms / 1e3), unit=UNIT,
+            e2e=dict(value=job_rows * e2e_steps / (e2e_ms / 1e3), unit=UNIT,
                      h2d_bytes_per_step=step.h2d_bytes_zero_copy(count),
                      d2h_bytes_per_step=step.d2h_bytes(),
                      ms_per_step=e2e_ms / e2e_steps,
