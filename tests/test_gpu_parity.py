@@ -327,3 +327,35 @@ def test_cuda_graph_replay_matches_eager(dl, name, block_only):
             assert torch.equal(e[key][:c], g[key][:c]), key
         for key in ("idx", "n_sel", "tok_sel", "conf_sel"):
             assert torch.equal(e[key], g[key]), key
+
+
+def test_step_memory_is_far_below_full_logits(dl):
+    """The step allocates no [B*L, V] buffer and the library allocates no device memory:
+    after warm-up, running steps changes neither torch's allocations nor the device's free
+    memory, and everything the step owns (outputs + workspace) is a small fraction of the
+    bf16 full-logits tensor it avoids."""
+    for name in ("cfg1", "cfg4"):
+        inp = WL.make_inputs(WL.CONFIGS[name], seed=0)
+        cfg = inp["cfg"]
+        dev = GU.to_device(inp)
+        step = dl.DecodeStep(cfg.B, cfg.L, cfg.d, cfg.V, cfg.k)
+        for _ in range(2):
+            step.run(dev["H"], dev["M"], dev["W"], dev["win_lo"], dev["win_hi"])
+        torch.cuda.synchronize()
+        torch.cuda.reset_peak_memory_stats()
+        before_alloc = torch.cuda.memory_allocated()
+        free_before, _ = torch.cuda.mem_get_info()
+        for _ in range(3):
+            step.run(dev["H"], dev["M"], dev["W"], dev["win_lo"], dev["win_hi"])
+        torch.cuda.synchronize()
+        free_after, _ = torch.cuda.mem_get_info()
+        assert dl.get_status() == 0
+        assert torch.cuda.max_memory_allocated() == before_alloc, name   # nothing allocated
+        assert free_after >= free_before, name                          # not even by the library
+        owned = step.ws.numel() + sum(t.numel() * t.element_size() for t in
+                                      (step.tok, step.conf, step.lse, step.row_idx, step.seq_off,
+                                       step.count, step.sel_buf))
+        full_logits_bf16 = cfg.B * cfg.L * cfg.V * 2
+        assert owned < full_logits_bf16 / 10, (name, owned, full_logits_bf16)
+        del step, dev
+        torch.cuda.empty_cache()
