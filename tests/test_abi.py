@@ -123,3 +123,15 @@ def test_window_entry_points_validate_on_host(lib):
                                       _p(a), 1 << 30, nul) == -1
     assert lib.dllm_decode_block_step(*ins, 0, _p(a), _p(a), *[_p(a)] * 6, _p(a), _p(a), nul, nul,
                                       _p(a), 1 << 30, nul) == -3
+
+
+def test_graft_entry_build_accepts_this_library(lib, monkeypatch):
+    """__graft_entry__.build() imports the package and checks the ABI version; run it here
+    with the (already built) library so that a version bump cannot break it unnoticed."""
+    import importlib
+    import sys
+    monkeypatch.syspath_prepend(ROOT)
+    entry = importlib.import_module("__graft_entry__")
+    monkeypatch.setattr(build, "build", lambda *a, **k: _abi.LIB_PATH)
+    entry.build()
+    assert "mask_only_logits_b200" in sys.modules
