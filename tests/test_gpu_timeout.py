@@ -19,11 +19,13 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.fixture(scope="module")
-def injected(tmp_path_factory):
+def injected():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
+    import os
     from mask_only_logits_b200 import _abi, build
-    out = str(tmp_path_factory.mktemp("inject") / "libdllm_skip_stage.so")
+    # built next to libdllm.so (in the package directory, never committed)
+    out = os.path.join(build.PKG_DIR, "libdllm_fault_skip_stage.so")
     build.build(extra_flags=["-DDLLM_FAULT_SKIP_STAGE=1"], out=out)
     return _abi.load_from(out)
 
