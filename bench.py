@@ -325,17 +325,17 @@ def run_vocab_sharded(args, cfg) -> None:
     if dl.get_status(stream) != 0:
         raise RuntimeError("device status after the timed region")
     t_ms, gemm_ms = D.max_over_ranks([t_ms, gemm_ms], dev)
-    # end to end: H and the mask from pinned host memory, the selection back, every step
+    # end to end: H and the mask read from pinned host memory by the library's compaction
+    # and gather kernels (only the mask and the masked rows cross the bus), the selection
+    # copied back, every step
     e2e_steps = args.e2e_steps or max(10, min(args.steps, 200))
     H_host, M_host = inp["H"].pin_memory(), inp["M"].pin_memory()
-    H_dev, M_dev = torch.empty_like(H), torch.empty_like(M)
     idx_host = torch.empty(cfg.B, cfg.k, dtype=torch.int32).pin_memory()
+    step.run(H_host, M_host, W_shard, win_lo, win_hi, stream, blk)
     barrier()
     t0 = time.perf_counter()
     for _ in range(e2e_steps):
-        H_dev.copy_(H_host, non_blocking=True)
-        M_dev.copy_(M_host, non_blocking=True)
-        step.run(H_dev, M_dev, W_shard, win_lo, win_hi, stream, blk)
+        step.run(H_host, M_host, W_shard, win_lo, win_hi, stream, blk)
         idx_host.copy_(step.idx, non_blocking=True)
     torch.cuda.synchronize(dev)
     e2e_ms = D.max_over_ranks([(time.perf_counter() - t0) * 1e3], dev)[0]
@@ -356,10 +356,11 @@ def run_vocab_sharded(args, cfg) -> None:
             config=dict(workload_config(cfg, count), parallelism=f"vocabulary-parallel over {world} GPU(s)"),
             roofline=roof, gpu_launches=launches,
             e2e=dict(value=count * e2e_steps / (e2e_ms / 1e3), unit=UNIT,
-                     h2d_bytes_per_step=cfg.B * cfg.L * (2 * cfg.d + 1),
+                     h2d_bytes_per_step=cfg.B * cfg.L + 2 * cfg.d * count,
                      d2h_bytes_per_step=cfg.B * cfg.k * 4, ms_per_step=e2e_ms / e2e_steps,
-                     note="every rank copies H and the mask in from pinned host memory and "
-                          "its selection back each step; wall clock, max over ranks"),
+                     note="every rank's kernels read the mask and the masked rows of H from "
+                          "pinned host memory and the selection is copied back each step (no "
+                          "overlap between steps); wall clock, max over ranks"),
             clocks=clk.summary())
         if cpu is not None:
             line["cpu_baseline"] = cpu
