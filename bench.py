@@ -100,8 +100,9 @@ def gemm_roofline(cfg, count: int, peaks: dict, gemm_s: float, paired: bool, ker
     gemm_bytes = 2.0 * cfg.V * cfg.d + 2.0 * count * cfg.d
     tensor_bound = flops / (peaks["bf16_tflops"] * 1e12) >= gemm_bytes / (peaks["hbm_gbs"] * 1e9)
     out = dict(bound="tensor" if tensor_bound else "hbm",
-               kernel=("masked_lmhead, paired-SM tcgen05 (lmhead_kernel<2, 0>)" if paired else
-                       "masked_lmhead, single-SM tcgen05 (lmhead_kernel<1, 0>)"))
+               kernel=("masked_lmhead, " + ("paired-SM" if paired else "single-SM") +
+                       f" tcgen05 ({kernel})" if kernel.startswith("lmhead_kernel") else
+                       "masked_lmhead, " + kernel))
     tflops = flops / gemm_s / 1e12
     gbs = gemm_bytes / gemm_s / 1e9
     if tensor_bound:
@@ -395,6 +396,11 @@ def main() -> None:
     ap.add_argument("--shard", default="replica", choices=["replica", "vocab"],
                     help="replica: one independent step per rank (weak scaling); vocab: one "
                          "step with W split by rows over the ranks (strong scaling)")
+    ap.add_argument("--policy", default="confidence", choices=["confidence", "entropy", "margin"],
+                    help="score the positions to unmask are ranked by (entropy / margin run the "
+                         "GEMM's extended epilogue)")
+    ap.add_argument("--threshold", type=float, default=None,
+                    help="threshold-based parallel unmasking on the policy's score (default: top-k)")
     ap.add_argument("--gemm-variant", type=int, default=0, choices=[0, 1, 2],
                     help="0 = library default, 1 = single-SM GEMM, 2 = paired-SM GEMM")
     args = ap.parse_args()
@@ -435,7 +441,8 @@ def main() -> None:
     torch.cuda.reset_peak_memory_stats(dev)
     base_mem = torch.cuda.memory_allocated(dev)
     dl.debug_set_gemm_variant(args.gemm_variant)
-    step = dl.DecodeStep(cfg.B, cfg.L, cfg.d, cfg.V, cfg.k, device=dev)
+    step = dl.DecodeStep(cfg.B, cfg.L, cfg.d, cfg.V, cfg.k, device=dev, policy=args.policy,
+                         threshold=args.threshold)
     stream = torch.cuda.current_stream(dev)
 
     for _ in range(args.warmup):
@@ -531,12 +538,14 @@ def main() -> None:
         step_gbs = a["bytes"] / (ms_step / 1e3) / 1e9
         full_logits = cfg.B * cfg.L * cfg.V * 4
         paired = args.gemm_variant == 2 or (args.gemm_variant == 0 and cfg.B * cfg.L <= 16384)
-        gemm_kernel_name = "lmhead_kernel<2, 0>" if paired else "lmhead_kernel<1, 0>"
+        mode = 1 if step.stats else 0
+        gemm_kernel_name = f"lmhead_kernel<{2 if paired else 1}, {mode}>"
         line = dict(
             metric=METRIC, value=rows_s, unit=UNIT, n_gpus=world, steps=args.steps,
             warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True, scaling="weak",
             vs_baseline=None, dtype="bf16", data="synthetic",
             config=dict(workload_config(cfg, count), masked_rows_all_ranks=job_rows,
+                        policy=args.policy, threshold=args.threshold,
                         **({"launch": "CUDA graph replay"} if args.graph else {})),
             tflops=step_tflops, gbs=step_gbs,
             roofline_frac_step=roof / (ms_step / 1e3),

@@ -304,23 +304,42 @@ def prof_end() -> tuple[float, int, int]:
     return ms.value, g.value, kcount.value
 
 
+POLICIES = ("confidence", "entropy", "margin")
+
+
 class DecodeStep:
     """Buffers for one decode-step shape (B, L, d, V, k) on one device, and the step itself.
+
+    ``policy`` picks the score the positions to unmask are ranked by: "confidence" (largest
+    softmax probability, higher is better), "entropy" (of the row's softmax, lower is
+    better) or "margin" (top-1 minus top-2 probability, higher is better).  With
+    ``threshold`` set, every candidate whose score is at least as good as the threshold is
+    unmasked, at most k and at least min(min_sel, candidates) per sequence; without it, the k
+    best.  ``conf_sel`` then holds the policy's score of each selected position.
 
     Outputs are views into buffers owned by this object; their first ``count`` entries are
     valid (``count`` stays on the device unless read).
     """
 
-    def __init__(self, B: int, L: int, d: int, V: int, k: int, device="cuda"):
+    def __init__(self, B: int, L: int, d: int, V: int, k: int, device="cuda",
+                 policy: str = "confidence", threshold: float | None = None, min_sel: int = 1):
         if k < 1 or k > MAX_K:
             raise ValueError(f"k must be in [1, {MAX_K}]")
+        if policy not in POLICIES:
+            raise ValueError(f"policy must be one of {POLICIES}")
         self.B, self.L, self.d, self.V, self.k = B, L, d, V, k
+        self.policy, self.threshold, self.min_sel = policy, threshold, min_sel
+        self.stats = {"confidence": 0, "entropy": STAT_ENTROPY, "margin": STAT_MARGIN}[policy]
         self.device = torch.device(device)
         n = B * L
         i32 = dict(dtype=torch.int32, device=self.device)
         self.tok = torch.empty(n, **i32)
         self.conf = torch.empty(n, dtype=torch.float32, device=self.device)
         self.lse = torch.empty(n, dtype=torch.float32, device=self.device)
+        self.entropy = torch.empty(n, dtype=torch.float32, device=self.device) \
+            if policy == "entropy" else None
+        self.margin = torch.empty(n, dtype=torch.float32, device=self.device) \
+            if policy == "margin" else None
         self.row_idx = torch.empty(n, **i32)
         self.seq_off = torch.empty(B + 1, **i32)
         self.count = torch.empty(4, **i32)          # 16 bytes: keeps the next buffer aligned
@@ -347,15 +366,48 @@ class DecodeStep:
                 buf[o[2]:o[2] + B * k].view(B, k),
                 buf[o[3]:o[3] + B * k].view(torch.float32).view(B, k))
 
+    def _plain(self) -> bool:
+        return self.policy == "confidence" and self.threshold is None
+
+    def _select(self, row_idx, seq_off, win_lo, win_hi, stream) -> None:
+        """The selection of this step's policy on the scores the logits call left."""
+        if self._plain():
+            select_unmask(self.conf, row_idx, seq_off, self.B, self.L, self.k, self.idx,
+                          self.n_sel, win_lo, win_hi, self.tok, self.tok_sel, self.conf_sel,
+                          stream)
+            return
+        score = {"confidence": self.conf, "entropy": self.entropy, "margin": self.margin}[self.policy]
+        ascending = self.policy == "entropy"
+        tau = self.threshold
+        if tau is None:                                  # plain top-k of this score
+            tau = float("inf") if ascending else float("-inf")
+        select_unmask_ex(score, row_idx, seq_off, self.B, self.L, self.k, tau, self.min_sel,
+                         self.idx, self.n_sel, ascending, win_lo, win_hi, self.tok, self.tok_sel,
+                         self.conf_sel, stream)
+
+    def _outputs(self) -> dict:
+        out = dict(tok=self.tok, conf=self.conf, lse=self.lse, row_idx=self.row_idx,
+                   seq_off=self.seq_off, count=self.count[:1], idx=self.idx, n_sel=self.n_sel,
+                   tok_sel=self.tok_sel, conf_sel=self.conf_sel)
+        if self.entropy is not None:
+            out["entropy"] = self.entropy
+        if self.margin is not None:
+            out["margin"] = self.margin
+        return out
+
     def run(self, H, M, W, win_lo=None, win_hi=None, stream=None, block_only=False) -> dict:
         """One step on device tensors.  block_only=True (windows required): logits for the
         masked rows inside the windows only; tok/conf/lse/row_idx then cover those rows."""
-        decode_step(H, M, W, self.k, self.tok, self.conf, self.lse, self.row_idx, self.seq_off,
-                    self.count, self.idx, self.n_sel, self.ws, win_lo, win_hi, self.tok_sel,
-                    self.conf_sel, stream, block_only)
-        return dict(tok=self.tok, conf=self.conf, lse=self.lse, row_idx=self.row_idx,
-                    seq_off=self.seq_off, count=self.count[:1], idx=self.idx, n_sel=self.n_sel,
-                    tok_sel=self.tok_sel, conf_sel=self.conf_sel)
+        if self._plain():
+            decode_step(H, M, W, self.k, self.tok, self.conf, self.lse, self.row_idx,
+                        self.seq_off, self.count, self.idx, self.n_sel, self.ws, win_lo, win_hi,
+                        self.tok_sel, self.conf_sel, stream, block_only)
+        else:
+            masked_logits_ex(H, M, W, self.stats, self.tok, self.conf, self.lse, self.entropy,
+                             self.margin, self.row_idx, self.seq_off, self.count, self.ws,
+                             stream, *((win_lo, win_hi) if block_only else (None, None)))
+            self._select(self.row_idx, self.seq_off, win_lo, win_hi, stream)
+        return self._outputs()
 
     # -- end-to-end from host memory ---------------------------------------------------------
     def capture(self, H, M, W, win_lo=None, win_hi=None, block_only=False):
@@ -385,9 +437,7 @@ class DecodeStep:
         else:
             with torch.cuda.stream(stream):
                 self._graph.replay()
-        return dict(tok=self.tok, conf=self.conf, lse=self.lse, row_idx=self.row_idx,
-                    seq_off=self.seq_off, count=self.count[:1], idx=self.idx, n_sel=self.n_sel,
-                    tok_sel=self.tok_sel, conf_sel=self.conf_sel)
+        return self._outputs()
 
     def _host_buffers(self):
         if self._host is None:
@@ -468,12 +518,11 @@ class DecodeStep:
             b = i & 1
             with torch.cuda.stream(s):
                 s.wait_event(prepped[b])
-                masked_logits_prepared(W, B, L, 0, self.tok, self.conf, self.lse, None, None,
-                                       pb["count"][b], pb["ws"][b], s)
+                masked_logits_prepared(W, B, L, self.stats, self.tok, self.conf, self.lse,
+                                       self.entropy, self.margin, pb["count"][b], pb["ws"][b], s)
                 if i >= 1:
                     s.wait_event(done[(i - 1) & 1])  # step i-1's selection has been copied out
-                select_unmask(self.conf, pb["row_idx"][b], pb["seq_off"][b], B, L, k, self.idx,
-                              self.n_sel, win_lo, win_hi, self.tok, self.tok_sel, self.conf_sel, s)
+                self._select(pb["row_idx"][b], pb["seq_off"][b], win_lo, win_hi, s)
                 used[b].record(s)
                 selected[b].record(s)
             # the selection goes back on the copy stream: the next step's GEMM does not wait

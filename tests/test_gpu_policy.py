@@ -201,3 +201,63 @@ def test_entropy_driven_step(dl):
     ref_idx, ref_n = O.select_unmask_threshold(-e64, g["row_idx"], g["seq_off"], L, 8, -tau, 1)
     np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
     np.testing.assert_array_equal(n_sel.cpu().numpy(), ref_n)
+
+
+# thresholds exactly representable in float32, so that the fp32 comparison on the GPU and
+# the fp64 one of the oracle agree for every score
+@pytest.mark.parametrize("policy,threshold,min_sel", [("entropy", None, 1), ("margin", None, 1),
+                                                     ("confidence", 0.015625, 2),
+                                                     ("entropy", 9.0, 0), ("margin", 2.0 ** -10, 1)])
+def test_decode_step_policies(dl, policy, threshold, min_sel):
+    """DecodeStep with an unmasking policy: the selection equals the oracle's threshold
+    selection on the step's own GPU scores (bit-exact), and the per-row scores match the
+    oracle's within the policy tolerances."""
+    inp = WL.make_inputs(WL.CONFIGS["cfg4"] if policy == "margin" else WL.CONFIGS["cfg0"], seed=7)
+    cfg = inp["cfg"]
+    step = dl.DecodeStep(cfg.B, cfg.L, cfg.d, cfg.V, cfg.k, policy=policy, threshold=threshold,
+                         min_sel=min_sel)
+    lo = None if inp["win_lo"] is None else torch.from_numpy(inp["win_lo"]).cuda()
+    hi = None if inp["win_hi"] is None else torch.from_numpy(inp["win_hi"]).cuda()
+    out = step.run(inp["H"].cuda(), inp["M"].cuda(), inp["W"].cuda(), lo, hi)
+    assert dl.get_status() == 0
+    c = int(out["count"][0])
+    score = out["conf"] if policy == "confidence" else out[policy]
+    s32 = score[:c].cpu().numpy().astype(np.float64)
+    row_idx, seq_off = out["row_idx"][:c].cpu().numpy(), out["seq_off"].cpu().numpy()
+    asc = policy == "entropy"
+    tau = threshold if threshold is not None else (np.inf if asc else -np.inf)
+    ref_idx, ref_n = O.select_unmask_threshold(-s32 if asc else s32, row_idx, seq_off, cfg.L, cfg.k,
+                                               -tau if asc else tau, min_sel, inp["win_lo"],
+                                               inp["win_hi"])
+    np.testing.assert_array_equal(out["n_sel"].cpu().numpy(), ref_n)
+    np.testing.assert_array_equal(out["idx"].cpu().numpy(), ref_idx)
+    # the selected scores are those of the selected rows
+    for b in range(cfg.B):
+        n = int(ref_n[b])
+        r = [np.searchsorted(row_idx, b * cfg.L + p) for p in ref_idx[b, :n]]
+        np.testing.assert_array_equal(out["conf_sel"][b, :n].cpu().numpy(), s32[r].astype(np.float32))
+    # scores against the oracle on a sample of rows
+    rows = np.arange(c) if c <= 600 else WL.sample_rows(c, 300, seed=1)
+    ref = O.oracle_rows(WL.bf16_bits(inp["H"]), WL.bf16_bits(inp["W"]), inp["M"].numpy(), rows)
+    if policy == "entropy":
+        e = s32[rows]
+        assert np.all(np.abs(e - ref["entropy"]) <= 2e-3 * np.abs(ref["entropy"]) + 2e-5)
+    elif policy == "margin":
+        m = s32[rows]
+        assert np.all(np.abs(m - ref["margin"]) <= 2e-3 * np.abs(ref["margin"]) + 1e-4 * ref["conf"])
+
+
+def test_policy_pipeline_matches_device_steps(dl):
+    """The host pipeline with an entropy policy selects what device-resident steps select."""
+    cfg = WL.CONFIGS["cfg0"]
+    inps = [WL.make_inputs(cfg, seed=s) for s in (11, 12, 13)]
+    W = inps[0]["W"].cuda()
+    step = dl.DecodeStep(cfg.B, cfg.L, cfg.d, cfg.V, cfg.k, policy="entropy", threshold=7.0)
+    expected = []
+    for inp in inps:
+        out = step.run(inp["H"].cuda(), inp["M"].cuda(), W)
+        expected.append((out["idx"].cpu().clone(), out["n_sel"].cpu().clone()))
+    batches = [(inp["H"].pin_memory(), inp["M"].pin_memory()) for inp in inps]
+    got = [(o["idx"].clone(), o["n_sel"].clone()) for o in step.run_host_pipeline(batches, W)]
+    for (gi, gn), (ei, en) in zip(got, expected):
+        assert torch.equal(gi, ei) and torch.equal(gn, en)
