@@ -87,6 +87,12 @@ def roofline_s(cfg, M: int, peaks: dict) -> float:
     return max(a["flops"] / (peaks["bf16_tflops"] * 1e12), a["bytes"] / (peaks["hbm_gbs"] * 1e9))
 
 
+def gemm_paired(variant: int, count: int) -> bool:
+    """Whether the GEMM runs on CTA pairs: forced (1, 2), or the library's choice from the
+    masked count (pairs for 129..16384 rows)."""
+    return variant == 2 or (variant == 0 and 128 < count <= 16384)
+
+
 def gemm_roofline(cfg, count: int, peaks: dict, gemm_s: float, paired: bool, kernel: str,
                   power_capped: bool = False) -> dict:
     """Roofline of the dominant kernel (the masked LM-head GEMM with its fused epilogue):
@@ -355,7 +361,7 @@ def run_vocab_sharded(args, cfg) -> None:
         ms_step = t_ms / args.steps
         clk_summary = clk.summary()
         roof = gemm_roofline(shard_cfg, count, peaks, gemm_ms / max(1, gemm_launches) / 1e3,
-                             args.gemm_variant == 2 or (args.gemm_variant == 0 and cfg.B * cfg.L <= 16384),
+                             gemm_paired(args.gemm_variant, count),
                              "vocabulary shard", "sw_power_cap" in clk_summary["reasons"])
         roof["traffic"] = None
         roof["shard"] = f"rows [{step.v0}, {step.v1}) of W on rank 0"
@@ -537,9 +543,10 @@ def main() -> None:
         step_tflops = a["flops"] / (ms_step / 1e3) / 1e12
         step_gbs = a["bytes"] / (ms_step / 1e3) / 1e9
         full_logits = cfg.B * cfg.L * cfg.V * 4
-        paired = args.gemm_variant == 2 or (args.gemm_variant == 0 and cfg.B * cfg.L <= 16384)
+        paired = gemm_paired(args.gemm_variant, count)
         mode = 1 if step.stats else 0
-        gemm_kernel_name = f"lmhead_kernel<{2 if paired else 1}, {mode}>"
+        gemm_kernel_name = (f"lmhead_auto_kernel<{mode}>" if args.gemm_variant == 0 else
+                            f"lmhead_kernel<{args.gemm_variant}, {mode}>")
         line = dict(
             metric=METRIC, value=rows_s, unit=UNIT, n_gpus=world, steps=args.steps,
             warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True, scaling="weak",

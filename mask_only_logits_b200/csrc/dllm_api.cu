@@ -49,12 +49,12 @@ struct DeviceState {
 };
 
 // GEMM variant: 2 = CTA pairs (cta_group::2, 256x256 tiles), 1 = single CTAs
-// (cta_group::1, 128x256 tiles).  0 = default: pairs when B*L <= kPairMaxPositions (few
-// m-tiles: the larger tile does more work per clock), single CTAs above (measured under the
-// 1 kW power cap, the single-CTA kernel does more work per joule and sustains a higher clock
-// on long GEMMs).
+// (cta_group::1, 128x256 tiles), both forced (test hook).  0 = default: chosen on the
+// device from the masked count (lm::auto_variant): pairs for 129..16384 rows (the larger
+// tile does more work per clock), single CTAs for one m-tile (a pair would compute 128
+// empty rows) and for long GEMMs (measured under the 1 kW power cap, the single-CTA kernel
+// does more work per joule and sustains a higher clock).
 std::atomic<int> g_gemm_variant{0};
-constexpr long long kPairMaxPositions = 16384;
 
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
@@ -129,7 +129,10 @@ dllm_status device_state(DeviceState** out) {
            cudaFuncSetAttribute(lm::lmhead_kernel<1, lm::kModeDebugStore>, smem_attr, lm::Cfg<1>::SMEM_BYTES) ||
            cudaFuncSetAttribute(lm::lmhead_kernel<2, lm::kModeStats>, smem_attr, lm::Cfg<2>::SMEM_BYTES) ||
            cudaFuncSetAttribute(lm::lmhead_kernel<2, lm::kModeStatsExt>, smem_attr, lm::Cfg<2>::SMEM_BYTES) ||
-           cudaFuncSetAttribute(lm::lmhead_kernel<2, lm::kModeDebugStore>, smem_attr, lm::Cfg<2>::SMEM_BYTES)))
+           cudaFuncSetAttribute(lm::lmhead_kernel<2, lm::kModeDebugStore>, smem_attr, lm::Cfg<2>::SMEM_BYTES) ||
+           cudaFuncSetAttribute(lm::lmhead_auto_kernel<lm::kModeStats>, smem_attr, lm::kAutoSmemBytes) ||
+           cudaFuncSetAttribute(lm::lmhead_auto_kernel<lm::kModeStatsExt>, smem_attr, lm::kAutoSmemBytes) ||
+           cudaFuncSetAttribute(lm::lmhead_auto_kernel<lm::kModeDebugStore>, smem_attr, lm::kAutoSmemBytes)))
         st.err = DLLM_ERR_CUDA;
       if (st.err == DLLM_OK) {
         // how many CTA pairs of the paired GEMM can be resident at once (a persistent grid
@@ -353,16 +356,18 @@ dllm_status run_logits(const LogitsArgs& a, bool debug, bool skip_prepare = fals
   const lm::Outputs outs{a.tok, a.conf, a.lse, a.entropy, a.margin, a.raw, a.a_offset};
   const long long n = static_cast<long long>(a.B) * a.L;
 
-  // GEMM variant and its work holders (CTAs, or CTA pairs)
+  // GEMM variant: 0 = chosen on the device from the masked count (lm::auto_variant, one
+  // launch in clusters of two CTAs), 1 / 2 = forced single CTAs / CTA pairs (test hook)
   int cg = g_gemm_variant.load();
-  if (cg == 0) cg = n <= kPairMaxPositions ? 2 : 1;
-  if (cg == 2 && ds->pairs < 1) cg = 1;
-  const int holders = cg == 2 ? ds->pairs : (ds->sms < lm::kMaxCtas ? ds->sms : lm::kMaxCtas);
-  const int bm = cg == 2 ? lm::Cfg<2>::BM : lm::Cfg<1>::BM;
-  const int gmax = cg == 2 ? lm::Cfg<2>::kGroupM : lm::Cfg<1>::kGroupM;
-  {
-    // largest partial footprint over every masked count: all positions masked, or any
-    // count that fits one group of m-tiles (remainder holders)
+  if (ds->pairs < 1) cg = 1;                                   // no CTA pairs on this device
+  const int single_holders = cg == 0 ? 2 * ds->pairs : (ds->sms < lm::kMaxCtas ? ds->sms : lm::kMaxCtas);
+  for (int v = 1; v <= 2; ++v) {
+    if (cg != 0 && cg != v) continue;
+    // largest partial footprint over every masked count this variant may run: all
+    // positions masked, or any count that fits one group of m-tiles (remainder holders)
+    const int holders = v == 2 ? ds->pairs : single_holders;
+    const int bm = v == 2 ? lm::Cfg<2>::BM : lm::Cfg<1>::BM;
+    const int gmax = v == 2 ? lm::Cfg<2>::kGroupM : lm::Cfg<1>::kGroupM;
     long long need = lm::Plan::make(static_cast<int>(n), a.V, holders, gmax, bm).part_entries();
     const long long mt = (n + bm - 1) / bm;
     for (long long m = 1; m <= mt && m <= gmax; ++m) {
@@ -377,9 +382,13 @@ dllm_status run_logits(const LogitsArgs& a, bool debug, bool skip_prepare = fals
     if ((st = prepare_rows(a, *ds, w)) != DLLM_OK) return st;
   }
 
-  CUtensorMap tmA, tmB;
+  // W is staged 256 rows per CTA by single CTAs and 128 rows per CTA by pairs
+  CUtensorMap tmA, tmB1, tmB2;
   if (make_tmap(&tmA, Hm, static_cast<uint64_t>(n), a.d, 128) != DLLM_OK) return DLLM_ERR_CUDA;
-  if (make_tmap(&tmB, a.W, static_cast<uint64_t>(a.V), a.d, lm::BN / cg) != DLLM_OK) return DLLM_ERR_CUDA;
+  if (cg != 2 && make_tmap(&tmB1, a.W, static_cast<uint64_t>(a.V), a.d, lm::BN) != DLLM_OK)
+    return DLLM_ERR_CUDA;
+  if (cg != 1 && make_tmap(&tmB2, a.W, static_cast<uint64_t>(a.V), a.d, lm::BN / 2) != DLLM_OK)
+    return DLLM_ERR_CUDA;
 
   cudaEvent_t e0 = nullptr, e1 = nullptr;
   if (g_prof.on) {
@@ -404,16 +413,16 @@ dllm_status run_logits(const LogitsArgs& a, bool debug, bool skip_prepare = fals
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cg == 2) {
+    if (cg != 1) {
       attr[1].id = cudaLaunchAttributeClusterDimension;
       attr[1].val.clusterDim.x = 2;
       attr[1].val.clusterDim.y = 1;
       attr[1].val.clusterDim.z = 1;
       cfg.numAttrs = 2;
-      cfg.gridDim = dim3(2 * holders, 1, 1);
-      cfg.dynamicSmemBytes = lm::Cfg<2>::SMEM_BYTES;
+      cfg.gridDim = dim3(2 * ds->pairs, 1, 1);
+      cfg.dynamicSmemBytes = cg == 0 ? lm::kAutoSmemBytes : lm::Cfg<2>::SMEM_BYTES;
     } else {
-      cfg.gridDim = dim3(holders, 1, 1);
+      cfg.gridDim = dim3(single_holders, 1, 1);
       cfg.dynamicSmemBytes = lm::Cfg<1>::SMEM_BYTES;
     }
     const int n_cap = static_cast<int>(n);
@@ -421,18 +430,26 @@ dllm_status run_logits(const LogitsArgs& a, bool debug, bool skip_prepare = fals
     const int mode = debug ? lm::kModeDebugStore : (a.stats ? lm::kModeStatsExt : lm::kModeStats);
     const int* cnt = a.count;
     cudaError_t e;
-#define DLLM_LAUNCH_GEMM(CGV, MODE)                                                            \
-  cudaLaunchKernelEx(&cfg, lm::lmhead_kernel<CGV, MODE>, tmA, tmB, cnt, n_cap, a.V, a.d, gmax, \
+#define DLLM_LAUNCH_GEMM(CGV, MODE, TMB)                                                      \
+  cudaLaunchKernelEx(&cfg, lm::lmhead_kernel<CGV, MODE>, tmA, TMB, cnt, n_cap, a.V, a.d,      \
+                     lm::Cfg<CGV>::kGroupM, part, w.part_cap, ctr, outs, dbg, ds->status)
+#define DLLM_LAUNCH_AUTO(MODE)                                                                 \
+  cudaLaunchKernelEx(&cfg, lm::lmhead_auto_kernel<MODE>, tmA, tmB1, tmB2, cnt, n_cap, a.V, a.d, \
                      part, w.part_cap, ctr, outs, dbg, ds->status)
-    if (cg == 2)
-      e = mode == lm::kModeStats ? DLLM_LAUNCH_GEMM(2, lm::kModeStats)
-        : mode == lm::kModeStatsExt ? DLLM_LAUNCH_GEMM(2, lm::kModeStatsExt)
-        : DLLM_LAUNCH_GEMM(2, lm::kModeDebugStore);
+    if (cg == 0)
+      e = mode == lm::kModeStats ? DLLM_LAUNCH_AUTO(lm::kModeStats)
+        : mode == lm::kModeStatsExt ? DLLM_LAUNCH_AUTO(lm::kModeStatsExt)
+        : DLLM_LAUNCH_AUTO(lm::kModeDebugStore);
+    else if (cg == 2)
+      e = mode == lm::kModeStats ? DLLM_LAUNCH_GEMM(2, lm::kModeStats, tmB2)
+        : mode == lm::kModeStatsExt ? DLLM_LAUNCH_GEMM(2, lm::kModeStatsExt, tmB2)
+        : DLLM_LAUNCH_GEMM(2, lm::kModeDebugStore, tmB2);
     else
-      e = mode == lm::kModeStats ? DLLM_LAUNCH_GEMM(1, lm::kModeStats)
-        : mode == lm::kModeStatsExt ? DLLM_LAUNCH_GEMM(1, lm::kModeStatsExt)
-        : DLLM_LAUNCH_GEMM(1, lm::kModeDebugStore);
+      e = mode == lm::kModeStats ? DLLM_LAUNCH_GEMM(1, lm::kModeStats, tmB1)
+        : mode == lm::kModeStatsExt ? DLLM_LAUNCH_GEMM(1, lm::kModeStatsExt, tmB1)
+        : DLLM_LAUNCH_GEMM(1, lm::kModeDebugStore, tmB1);
 #undef DLLM_LAUNCH_GEMM
+#undef DLLM_LAUNCH_AUTO
     if (e != cudaSuccess) return DLLM_ERR_CUDA;
   }
   count_launch();

@@ -473,16 +473,20 @@ struct Outputs {
   int a_offset;
 };
 
+// The GEMM of one launch on a CTA (CG = 1) or on one CTA of a pair (CG = 2).  tmA / tmB
+// point at the kernel's own __grid_constant__ tensor-map parameters (TMA needs their
+// parameter-space address, never a copy).  waited: the kernel already passed
+// griddepcontrol.wait (then the set-up below no longer overlaps the previous kernel).
 template <int CG, int kMode>
-__global__ void __launch_bounds__(kThreads, 1)
-lmhead_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-              const int* __restrict__ count_ptr, int n_cap, int V, int d, int gmax,
-              const Partials part, long long part_cap, int* __restrict__ unit_ctr,
-              const Outputs out, float* __restrict__ dbg_logits, int* __restrict__ status) {
+__device__ __forceinline__ void lmhead_run(uint8_t* smem_raw, const CUtensorMap* tmA,
+                                           const CUtensorMap* tmB, const int* __restrict__ count_ptr,
+                                           bool waited, int n_cap, int V, int d, int gmax,
+                                           const Partials& part, long long part_cap,
+                                           int* __restrict__ unit_ctr, const Outputs& out,
+                                           float* __restrict__ dbg_logits, int* __restrict__ status) {
   using C = Cfg<CG>;
   constexpr bool kDebugStore = kMode == kModeDebugStore;
   constexpr bool kExt = kMode == kModeStatsExt;
-  extern __shared__ uint8_t smem_raw[];
   Smem<CG> sm(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = CG == 1 ? 0u : cluster_ctarank();   // rank inside the CTA pair
@@ -503,8 +507,8 @@ lmhead_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(tmA);
+    tma_prefetch_desc(tmB);
   }
   if (warp == 1) {
     if constexpr (CG == 1) {
@@ -524,8 +528,10 @@ lmhead_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
 
   // everything above touched only this CTA's own resources; from here on the kernel reads
   // what the compaction and gather kernels wrote
-  pdl_wait();
-  pdl_launch_dependents();
+  if (!waited) {
+    pdl_wait();
+    pdl_launch_dependents();
+  }
   const int count = *count_ptr;
   const Plan pl = Plan::make(count < 0 ? 0 : (count > n_cap ? n_cap : count), V,
                              static_cast<int>(gridDim.x) / CG, gmax, C::BM);
@@ -554,13 +560,13 @@ lmhead_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
           const uint32_t fb = smem_u32(&sm.full[s]);
           if constexpr (CG == 1) {
             mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
-            tma_load_2d(smem_u32(sm.a + s * C::A_BYTES), &tmA, fb, kb * BK, a_row);
-            tma_load_2d(smem_u32(sm.b + s * C::B_BYTES), &tmB, fb, kb * BK, b_row);
+            tma_load_2d(smem_u32(sm.a + s * C::A_BYTES), tmA, fb, kb * BK, a_row);
+            tma_load_2d(smem_u32(sm.b + s * C::B_BYTES), tmB, fb, kb * BK, b_row);
           } else {
             if (leader) mbar_arrive_expect_tx(fb, CG * C::STAGE_BYTES);
             const uint32_t fb_leader = fb & kPeerBitMask;
-            tma_load_2d_pair(smem_u32(sm.a + s * C::A_BYTES), &tmA, fb_leader, kb * BK, a_row);
-            tma_load_2d_pair(smem_u32(sm.b + s * C::B_BYTES), &tmB, fb_leader, kb * BK, b_row);
+            tma_load_2d_pair(smem_u32(sm.a + s * C::A_BYTES), tmA, fb_leader, kb * BK, a_row);
+            tma_load_2d_pair(smem_u32(sm.b + s * C::B_BYTES), tmB, fb_leader, kb * BK, b_row);
           }
         }
         return true;
@@ -827,6 +833,53 @@ lmhead_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     if constexpr (CG == 1) tmem_dealloc(tmem_base, kTmemCols);
     else tmem_dealloc_pair(tmem_base, kTmemCols);
   }
+}
+
+// One GEMM variant, fixed at launch (CG = 2 needs a launch in clusters of two CTAs).  Its
+// set-up (barriers, TMEM, tensor-map prefetch) runs before griddepcontrol.wait, overlapping
+// the previous kernel on the stream.
+template <int CG, int kMode>
+__global__ void __launch_bounds__(kThreads, 1)
+lmhead_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              const int* __restrict__ count_ptr, int n_cap, int V, int d, int gmax,
+              const Partials part, long long part_cap, int* __restrict__ unit_ctr,
+              const Outputs out, float* __restrict__ dbg_logits, int* __restrict__ status) {
+  extern __shared__ uint8_t smem_raw[];
+  lmhead_run<CG, kMode>(smem_raw, &tmA, &tmB, count_ptr, false, n_cap, V, d, gmax, part, part_cap,
+                        unit_ctr, out, dbg_logits, status);
+}
+
+// The variant chosen on the device from the masked count, which the host does not know:
+// one m-tile of 128 rows or fewer runs on single CTAs (a pair would compute 128 empty
+// rows), up to kPairMaxRows rows on CTA pairs (per SM half the W bytes staged per flop),
+// more on single CTAs (longer GEMMs, where the pairs' higher power draw costs clock under
+// the power cap).  Launched in clusters of two CTAs with the shared memory of the larger
+// variant; the count is read first, so the set-up follows griddepcontrol.wait.
+constexpr int kSingleMaxRows = 128;
+constexpr int kPairMaxRows = 16384;
+__host__ __device__ inline int auto_variant(int count) {
+  return count > kSingleMaxRows && count <= kPairMaxRows ? 2 : 1;
+}
+constexpr int kAutoSmemBytes = Cfg<1>::SMEM_BYTES > Cfg<2>::SMEM_BYTES ? Cfg<1>::SMEM_BYTES
+                                                                        : Cfg<2>::SMEM_BYTES;
+
+template <int kMode>
+__global__ void __launch_bounds__(kThreads, 1)
+lmhead_auto_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB1,
+                   const __grid_constant__ CUtensorMap tmB2, const int* __restrict__ count_ptr,
+                   int n_cap, int V, int d, const Partials part, long long part_cap,
+                   int* __restrict__ unit_ctr, const Outputs out, float* __restrict__ dbg_logits,
+                   int* __restrict__ status) {
+  extern __shared__ uint8_t smem_raw[];
+  pdl_wait();
+  pdl_launch_dependents();
+  const int c = *count_ptr;
+  if (auto_variant(c) == 2)
+    lmhead_run<2, kMode>(smem_raw, &tmA, &tmB2, count_ptr, true, n_cap, V, d, Cfg<2>::kGroupM,
+                         part, part_cap, unit_ctr, out, dbg_logits, status);
+  else
+    lmhead_run<1, kMode>(smem_raw, &tmA, &tmB1, count_ptr, true, n_cap, V, d, Cfg<1>::kGroupM,
+                         part, part_cap, unit_ctr, out, dbg_logits, status);
 }
 
 }  // namespace lm
