@@ -51,10 +51,16 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "lmhead_traffic.json")
 
 
 def gemm_source_hash() -> str:
+    """SHA-256 of the GEMM's code: its sources with comments and whitespace removed, so that
+    an edited comment does not void a capture while any change to the code does."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for rel in GEMM_SOURCES:
-        h.update(open(os.path.join(ROOT, rel), "rb").read())
+        text = open(os.path.join(ROOT, rel)).read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)        # block comments
+        text = re.sub(r"//[^\n]*", " ", text)                      # line comments
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()
 
 

@@ -5,14 +5,16 @@
 // C[i, v] = sum_k Hm[i, k] * W[v, k] for the compacted masked rows Hm (bf16, K-major) and
 // the vocabulary projection W (bf16, K-major), fp32 accumulation in tensor memory.
 //
-// Persistent, warp-specialised kernel, one CTA per SM, 192 threads, templated on the CTA
-// group size CG:
+// Persistent, warp-specialised GEMM, one CTA per SM, 192 threads, in two bodies (the
+// device function lmhead_run, templated on the CTA group size CG):
 //   CG = 1  each CTA owns a 128 x 256 tile (tcgen05.mma.cta_group::1, M=128, N=256)
 //   CG = 2  a cluster of two CTAs on paired SMs owns a 256 x 256 tile
 //           (tcgen05.mma.cta_group::2, M=256, N=256): each CTA stages 128 rows of Hm and
 //           128 rows of W per stage, the leader CTA issues the MMAs for both, and each CTA's
 //           TMEM holds its own 128 rows of the accumulator.  Per SM this halves the W bytes
 //           staged per flop.
+// lmhead_auto_kernel (the default) is launched in clusters of two CTAs and picks the body
+// on the device from the masked count; lmhead_kernel<CG> runs one body fixed at launch.
 // Roles (per CTA):
 //   warp 0      TMA producer: a 128x64 tile of Hm and a (256/CG)x64 tile of W per stage
 //               (128-byte swizzle) into a kStages-deep shared-memory ring
@@ -30,7 +32,8 @@
 // W tiles at the same time (each W tile is fetched from HBM about once per group and served
 // from L2 to the others) while the group's Hm tiles stay resident in L2.  Per row, the
 // partials of the P streams are merged (lse_merge) by the epilogue of whichever CTA finishes
-// the m-tile's last unit; with P = 1 the unit's statistics are the result.
+// the m-tile's last unit (its four epilogue warps each merge a quarter of the partials, then
+// combine in order); with P = 1 the unit's statistics are the result.
 //
 // Every wait is bounded (ptx.cuh).  On a timeout the CTA raises its abort flag, every role
 // unwinds, the MMA issuer waits (bounded) for its issued MMAs, the CTA lingers 2 ms so that
