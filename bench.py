@@ -225,7 +225,8 @@ def blas_threads() -> int:
 
 def cpu_baseline(inp: dict, budget_s: float = 10.0) -> dict:
     """The oracle on a bounded sample of the workload's masked rows: the sample doubles until
-    one run takes about budget_s (or covers every masked row); the last run is reported."""
+    one run takes about budget_s; when every masked row fits in less, whole passes over the
+    workload repeat until budget_s is spent.  Rows per second over the reported runs."""
     cfg = inp["cfg"]
     count = rows_of_step(inp)
     rng = np.random.default_rng(0)
@@ -236,9 +237,15 @@ def cpu_baseline(inp: dict, budget_s: float = 10.0) -> dict:
         if t >= budget_s or n_rows == count:
             break
         n_rows = min(count, max(2 * n_rows, int(n_rows * budget_s / max(t, 1e-3))))
+    passes = 1
+    while t < budget_s and n_rows == count:           # the whole workload, again
+        t1, n1 = oracle_rate(inp, rows)
+        t, n, passes = t + t1, n + n1, passes + 1
+    what = (f"{n_rows} of {count} masked rows" if passes == 1 else
+            f"all {count} masked rows, {passes} passes")
     return dict(value=n / t, unit=UNIT, cores=blas_threads(), kind="oracle",
-                sample=f"{n_rows} of {count} masked rows of {cfg.name} (fp64 NumPy logits over all "
-                       f"V={cfg.V}, statistics, top-k over the sample), {t:.1f} s")
+                sample=f"{what} of {cfg.name} (fp64 NumPy logits over all V={cfg.V}, statistics, "
+                       f"top-k over the sample), {t:.1f} s")
 
 
 def run_reference(args, cfg) -> None:
