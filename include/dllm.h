@@ -15,6 +15,17 @@
  *      (confidence-driven unmasking, dLLM inference survey page, "Main Findings";
  *      an optional per-sequence window restricts candidates to the current
  *      semi-autoregressive block, Sparse-dLLM page, "Experiment")  (dllm_select_unmask).
+ * and around these:
+ *   - the whole step in one call (dllm_decode_step), or with logits for the current
+ *     block's rows only (dllm_decode_block_step, dllm_masked_logits_window,
+ *     dllm_mask_compact_window);
+ *   - entropy / top-2 margin scores and threshold-based parallel unmasking
+ *     (dllm_masked_logits_ex, dllm_select_unmask_ex);
+ *   - the staging of a step split from its GEMM, for overlapping steps
+ *     (dllm_prepare_rows, dllm_masked_logits_prepared);
+ *   - a vocabulary-parallel LM head over several GPUs: per-shard softmax partials and their
+ *     merge (dllm_masked_partials, dllm_lse_merge);
+ *   - compaction without a workspace (dllm_mask_compact_noalloc).
  *
  * Conventions for every call:
  *   - Pointers marked "device" must point to memory of the current CUDA device; the caller
