@@ -121,13 +121,15 @@ def row_policy_stats(Z: np.ndarray):
 
 
 def rows_stats_chunked(H_rows_bits: np.ndarray, W_bits: np.ndarray, chunk: int = V_CHUNK,
-                       with_policy: bool = False):
+                       with_policy: bool = False, W64: np.ndarray | None = None):
     """(tok, m, lse, conf, top2_gap) for rows of H given as bf16 bits, W as bf16 bits.
 
     Logits are formed chunk by chunk over the vocabulary and kept whole per row before the
     statistics are taken (the statistics are those of ``row_stats`` on the full row); the
     chunking only bounds the fp64 copy of W held at once.  top2_gap = m - (second largest
-    logit), used to exempt near-ties from exact argmax comparison.
+    logit), used to exempt near-ties from exact argmax comparison.  W64, when given, is
+    bf16_bits_to_f64(W_bits) computed once by the caller (the same values; callers that run
+    many row sets against one W skip converting it every time).
     """
     H64 = bf16_bits_to_f64(H_rows_bits)
     n = H64.shape[0]
@@ -135,7 +137,8 @@ def rows_stats_chunked(H_rows_bits: np.ndarray, W_bits: np.ndarray, chunk: int =
     Z = np.empty((n, V), dtype=np.float64)
     for v0 in range(0, V, chunk):
         v1 = min(V, v0 + chunk)
-        Z[:, v0:v1] = logits_rows(H64, bf16_bits_to_f64(W_bits[v0:v1]))
+        Wc = W64[v0:v1] if W64 is not None else bf16_bits_to_f64(W_bits[v0:v1])
+        Z[:, v0:v1] = logits_rows(H64, Wc)
     tok, m, lse, conf = row_stats(Z)
     gap = top2_gap(Z)
     if with_policy:
