@@ -432,6 +432,9 @@ def main() -> None:
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--graph", action="store_true",
                     help="time replays of the step captured in a CUDA graph (one launch per step)")
+    ap.add_argument("--serial", action="store_true",
+                    help="run each step's staging (compaction, gather) on the compute stream "
+                         "instead of overlapping it with the previous step's GEMM")
     ap.add_argument("--shard", default="replica", choices=["replica", "vocab"],
                     help="replica: one independent step per rank (weak scaling); vocab: one "
                          "step with W split by rows over the ranks (strong scaling)")
@@ -506,6 +509,14 @@ def main() -> None:
             step.replay(stream)
         torch.cuda.synchronize(dev)
 
+    overlap = not (args.graph or args.serial)
+    if overlap:
+        # the staging of step i+1 (compaction of the mask, gather of the masked rows) runs
+        # on a second stream while step i's GEMM and selection run on this one
+        prep_stream = torch.cuda.Stream(dev)
+        step.run_overlapped([(H, M)] * 3, W, win_lo, win_hi, stream, prep_stream, blk)
+        torch.cuda.synchronize(dev)
+
     def one_step():
         if args.graph:
             step.replay(stream)
@@ -516,8 +527,12 @@ def main() -> None:
     with ClockSampler(dev.index if dev.index is not None else 0) as clk:
         barrier()
         ev0.record(stream)
-        for _ in range(args.steps):
-            one_step()
+        if overlap:
+            step.run_overlapped([(H, M)] * args.steps, W, win_lo, win_hi, stream, prep_stream,
+                                blk)
+        else:
+            for _ in range(args.steps):
+                one_step()
         ev1.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
@@ -586,7 +601,9 @@ def main() -> None:
             vs_baseline=None, dtype="bf16", data="synthetic",
             config=dict(workload_config(cfg, count), masked_rows_all_ranks=job_rows,
                         policy=args.policy, threshold=args.threshold,
-                        **({"launch": "CUDA graph replay"} if args.graph else {})),
+                        launch=("CUDA graph replay" if args.graph else
+                                "one stream, steps in sequence" if args.serial else
+                                "two streams: staging of step i+1 overlaps step i")),
             tflops=step_tflops, gbs=step_gbs,
             roofline_frac_step=roof / (ms_step / 1e3),
             roofline_ms=roof * 1e3,

@@ -465,6 +465,17 @@ class DecodeStep:
         s.synchronize()
         return dict(zip(("idx", "n_sel", "tok_sel", "conf_sel"), self._sel_views(hb["sel"])))
 
+    def _double(self) -> dict:
+        """Two sets of (workspace, row_idx, seq_off, count): this object's own and a second
+        one, so that staging of one step can run while the previous step computes."""
+        if getattr(self, "_dbl", None) is None:
+            i32 = dict(dtype=torch.int32, device=self.device)
+            self._dbl = dict(ws=[self.ws, torch.empty_like(self.ws)],
+                             row_idx=[self.row_idx, torch.empty(self.B * self.L, **i32)],
+                             seq_off=[self.seq_off, torch.empty(self.B + 1, **i32)],
+                             count=[self.count, torch.empty(4, **i32)])
+        return self._dbl
+
     def run_host_pipeline(self, batches, W, win_lo=None, win_hi=None, stream=None,
                           prep_stream=None, block_only=False):
         """Decode steps over host batches [(H_host, M_host), ...] in page-locked host memory,
@@ -483,14 +494,9 @@ class DecodeStep:
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
         ps = prep_stream if prep_stream is not None else torch.cuda.Stream(self.device)
         if getattr(self, "_pipe", None) is None:
-            pin = dict(pin_memory=True)
-            i32 = dict(dtype=torch.int32, device=self.device)
             self._pipe = dict(
-                ws=[self.ws, torch.empty_like(self.ws)],
-                row_idx=[self.row_idx, torch.empty(B * L, **i32)],
-                seq_off=[self.seq_off, torch.empty(B + 1, **i32)],
-                count=[self.count, torch.empty(4, **i32)],
-                out_buf=[torch.empty(self.sel_buf.numel(), dtype=torch.int32, **pin)
+                self._double(),
+                out_buf=[torch.empty(self.sel_buf.numel(), dtype=torch.int32, pin_memory=True)
                          for _ in range(2)],
                 copy_stream=torch.cuda.Stream(self.device))
             self._pipe["out"] = [dict(zip(("idx", "n_sel", "tok_sel", "conf_sel"),
@@ -552,6 +558,48 @@ class DecodeStep:
             i += 1
         done[pending].synchronize()
         yield pb["out"][pending]
+
+    def run_overlapped(self, batches, W, win_lo=None, win_hi=None, stream=None,
+                       prep_stream=None, block_only=False, sel_out=None) -> dict:
+        """Whole steps over device-resident batches [(H, M), ...] (or pinned host ones), each
+        step's staging (compaction and gather, ``prepare_rows``) on a second stream during
+        the previous step's GEMM, with no host synchronisation: the throughput loop of a
+        serving process whose inputs are already on the GPU.  sel_out, if given, is a list
+        (one per batch) of int32 device buffers shaped like ``sel_buf`` that receive each
+        step's packed selection; otherwise only the last step's outputs remain (this
+        object's buffers)."""
+        B, L, d, V, k = self.B, self.L, self.d, self.V, self.k
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        ps = prep_stream if prep_stream is not None else torch.cuda.Stream(self.device)
+        ob = self._double()
+        prepped = [torch.cuda.Event() for _ in range(2)]
+        used = [torch.cuda.Event() for _ in range(2)]
+        pw = (win_lo, win_hi) if block_only else (None, None)
+        ps.wait_stream(s)                            # inputs written before the call are ready
+        last = 0
+        for i, (H, M) in enumerate(batches):
+            b = i & 1
+            with torch.cuda.stream(ps):
+                if i >= 2:
+                    ps.wait_event(used[b])           # step i-2 no longer reads this workspace
+                prepare_rows(H, M, d, V, ob["row_idx"][b], ob["seq_off"][b], ob["count"][b],
+                             ob["ws"][b], ps, *pw)
+                prepped[b].record(ps)
+            with torch.cuda.stream(s):
+                s.wait_event(prepped[b])
+                masked_logits_prepared(W, B, L, self.stats, self.tok, self.conf, self.lse,
+                                       self.entropy, self.margin, ob["count"][b], ob["ws"][b], s)
+                self._select(ob["row_idx"][b], ob["seq_off"][b], win_lo, win_hi, s)
+                used[b].record(s)
+                if sel_out is not None:
+                    sel_out[i].copy_(self.sel_buf, non_blocking=True)
+            last = b
+        if last == 1:                                # leave the last step's compaction in place
+            with torch.cuda.stream(s):
+                self.row_idx.copy_(ob["row_idx"][1])
+                self.seq_off.copy_(ob["seq_off"][1])
+                self.count.copy_(ob["count"][1])
+        return self._outputs()
 
     def h2d_bytes_zero_copy(self, count: int) -> int:
         """Bytes one pipelined step reads from host memory: the mask and the masked rows."""

@@ -359,3 +359,30 @@ def test_step_memory_is_far_below_full_logits(dl):
         assert owned < full_logits_bf16 / 10, (name, owned, full_logits_bf16)
         del step, dev
         torch.cuda.empty_cache()
+
+
+def test_overlapped_steps_match_single_steps(dl):
+    """Steps overlapped on two streams (staging of step i+1 during step i) select exactly
+    what single steps select, batch by batch, and leave the last step's outputs."""
+    for name in ("cfg0", "cfg4"):
+        cfg = WL.CONFIGS[name]
+        inps = [WL.make_inputs(cfg, seed=s) for s in (21, 22, 23, 24, 25)]
+        W = inps[0]["W"].cuda()
+        lo = None if inps[0]["win_lo"] is None else torch.from_numpy(inps[0]["win_lo"]).cuda()
+        hi = None if inps[0]["win_hi"] is None else torch.from_numpy(inps[0]["win_hi"]).cuda()
+        step = dl.DecodeStep(cfg.B, cfg.L, cfg.d, cfg.V, cfg.k)
+        dev = [(inp["H"].cuda(), inp["M"].cuda()) for inp in inps]
+        expected = []
+        for H, M in dev:
+            step.run(H, M, W, lo, hi)
+            expected.append(step.sel_buf.clone())
+        sel_out = [torch.empty_like(step.sel_buf) for _ in dev]
+        out = step.run_overlapped(dev, W, lo, hi, sel_out=sel_out)
+        torch.cuda.synchronize()
+        assert dl.get_status() == 0
+        for got, exp in zip(sel_out, expected):
+            assert torch.equal(got, exp), name
+        assert torch.equal(step.sel_buf, expected[-1])
+        c = int(out["count"][0])
+        ref_rows, _, ref_c = O.mask_compact(inps[-1]["M"].numpy())
+        assert c == ref_c and np.array_equal(out["row_idx"][:c].cpu().numpy(), ref_rows)
