@@ -24,6 +24,10 @@
 //   3. one ordered pass collects every candidate above T and the first needed ones equal
 //      to T (block-wide ballot scan keeps them in row order)
 //   4. bitonic sort of the (at most k_eff) keys, descending; write positions, tokens, scores.
+// Up to kSelRankMax candidates (e.g. one 32-token block) skip steps 2-4: keys are distinct,
+// so the number of candidates whose key is larger is a candidate's place in the sorted
+// output, and each thread writes its own candidate there if that place is below k_eff
+// (about n^2 / 32 cycles, against ~25 CTA-wide barriers for steps 2-4).
 #pragma once
 #include "ptx.cuh"
 
@@ -32,6 +36,8 @@ namespace dllm {
 constexpr int kSelThreads = 1024;
 constexpr int kSelMaxK = 1024;
 constexpr int kSelStage = 4096;     // up to this many candidates: keys staged in shared memory
+constexpr int kSelRankMax = 256;    // up to this many: output place by rank, no select or sort
+static_assert(kSelRankMax <= kSelThreads && kSelRankMax <= kSelStage, "one staged key per thread");
 
 // Float -> unsigned with the same order (for non-NaN values).
 __device__ __forceinline__ uint32_t ordered_bits(float f) {
@@ -112,6 +118,32 @@ select_unmask_kernel(const float* __restrict__ conf, const int* __restrict__ row
     k_eff = want < k ? want : k;
   }
   const int nsel = k_eff;
+
+  if (n <= kSelRankMax) {            // uniform over the CTA: every thread returns here
+    if (tid < n) {
+      const uint32_t mine = skey[tid];
+      int place = 0;                   // candidates ahead: larger key, or equal and lower row
+      for (int j = 0; j < n; ++j) {
+        const uint32_t other = skey[j];
+        place += (other > mine || (other == mine && j < tid)) ? 1 : 0;
+      }
+      if (place < nsel) {
+        const int r = c0 + tid;
+        const size_t o = static_cast<size_t>(b) * k + place;
+        idx[o] = static_cast<int>(row_idx[r] - seq_base);
+        if (tok_sel) tok_sel[o] = tok[r];
+        if (conf_sel) conf_sel[o] = conf[r];
+      }
+    }
+    for (int j = nsel + tid; j < k; j += kSelThreads) {
+      const size_t o = static_cast<size_t>(b) * k + j;
+      idx[o] = -1;
+      if (tok_sel) tok_sel[o] = -1;
+      if (conf_sel) conf_sel[o] = 0.f;
+    }
+    if (tid == 0) n_sel[b] = nsel;
+    return;
+  }
 
   if (tid == 0) sh_n = 0;
   __syncthreads();

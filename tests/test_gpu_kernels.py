@@ -250,3 +250,22 @@ def test_select_windows_and_empty(dl):
     M2[1, 10:20] = 1
     _select_case(dl, rng.random(10).astype(np.float32), M2, 5)
     _select_case(dl, np.zeros(0, np.float32), np.zeros((2, 40), np.uint8), 3)
+
+
+@pytest.mark.parametrize("k", [1, 4, 64, 300])
+def test_select_rank_path_boundary(dl, k):
+    """Sequences with 255, 256 (placed by rank) and 257 (radix select) candidates, one per
+    sequence in one launch, with exact ties: every path gives the oracle's selection."""
+    rng = np.random.default_rng(k)
+    B, L = 3, 400
+    M = np.zeros((B, L), np.uint8)
+    for b, n_b in enumerate((255, 256, 257)):
+        M[b, rng.choice(L, n_b, replace=False)] = 1
+    n = int(M.sum())
+    conf = (rng.integers(1, 17, size=n) / 16.0).astype(np.float32)
+    tok = rng.integers(0, 1000, size=n).astype(np.int32)
+    _select_case(dl, conf, M, k, tok_np=tok)
+    # a window that leaves 256 candidates in one sequence and 257 in another
+    lo = np.array([0, 0, 0], np.int32)
+    hi = np.array([L, L, L], np.int32)
+    _select_case(dl, conf, M, k, (lo, hi))

@@ -261,3 +261,49 @@ def test_policy_pipeline_matches_device_steps(dl):
     got = [(o["idx"].clone(), o["n_sel"].clone()) for o in step.run_host_pipeline(batches, W)]
     for (gi, gn), (ei, en) in zip(got, expected):
         assert torch.equal(gi, ei) and torch.equal(gn, en)
+
+
+@pytest.mark.parametrize("policy,threshold", [("entropy", 7.0), ("margin", None),
+                                              ("confidence", 0.015625)])
+def test_policy_overlapped_steps_block_only(dl, policy, threshold):
+    """Overlapped steps (staging on a second stream) with a policy and current-block-only
+    logits select what single device-resident steps select, batch by batch."""
+    cfg = WL.CONFIGS["cfg4_block"]
+    inps = [WL.make_inputs(cfg, seed=s) for s in (31, 32, 33)]
+    W = inps[0]["W"].cuda()
+    lo = torch.from_numpy(inps[0]["win_lo"]).cuda()
+    hi = torch.from_numpy(inps[0]["win_hi"]).cuda()
+    step = dl.DecodeStep(cfg.B, cfg.L, cfg.d, cfg.V, cfg.k, policy=policy, threshold=threshold)
+    dev = [(inp["H"].cuda(), inp["M"].cuda()) for inp in inps]
+    expected = []
+    for H, M in dev:
+        step.run(H, M, W, lo, hi, block_only=True)
+        expected.append(step.sel_buf.clone())
+    sel_out = [torch.empty_like(step.sel_buf) for _ in dev]
+    step.run_overlapped(dev, W, lo, hi, block_only=True, sel_out=sel_out)
+    torch.cuda.synchronize()
+    assert dl.get_status() == 0
+    for got, exp in zip(sel_out, expected):
+        assert torch.equal(got, exp)
+    # the block-only row set of the last batch: the masked positions inside the windows
+    c = int(step.count[0])
+    Mw = O.window_mask(inps[-1]["M"].numpy(), inps[0]["win_lo"], inps[0]["win_hi"])
+    assert c == int(Mw.sum())
+    assert np.array_equal(step.row_idx[:c].cpu().numpy(), np.flatnonzero(Mw.reshape(-1)))
+
+
+@pytest.mark.parametrize("ascending", [False, True])
+def test_threshold_select_rank_path_boundary(dl, ascending):
+    """Threshold selection on 255 / 256 / 257 candidates (the rank placement and the radix
+    select meet at 256), exact ties, min_sel floors above and below the passing count."""
+    rng = np.random.default_rng(5)
+    B, L = 3, 300
+    M = np.zeros((B, L), np.uint8)
+    for b, n_b in enumerate((255, 256, 257)):
+        M[b, rng.choice(L, n_b, replace=False)] = 1
+    n = int(M.sum())
+    score = (rng.integers(0, 32, size=n) / 32.0).astype(np.float32)
+    if ascending:
+        score = -score + 0.25
+    for tau, min_sel, k in ((0.5, 1, 256), (0.97, 20, 64), (0.0, 0, 300), (2.0, 5, 8)):
+        _select_ex(dl, score, M, k, tau, min_sel, ascending)
