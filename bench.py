@@ -236,6 +236,17 @@ def blas_threads() -> int:
         return os.cpu_count() or 1
 
 
+def blas_backend() -> str:
+    """The BLAS library NumPy's matmul runs on, with its version (e.g. "openblas 0.3.29")."""
+    try:
+        from threadpoolctl import threadpool_info
+        libs = [f"{i.get('internal_api')} {i.get('version')}" for i in threadpool_info()
+                if i.get("user_api") == "blas"]
+        return ", ".join(libs) or "unknown"
+    except Exception:  # noqa: BLE001
+        return "unknown"
+
+
 def cpu_baseline(inp: dict, budget_s: float = 10.0) -> dict:
     """The oracle on a bounded sample of the workload's masked rows: the sample doubles until
     one run takes about budget_s; when every masked row fits in less, whole passes over the
@@ -258,6 +269,7 @@ def cpu_baseline(inp: dict, budget_s: float = 10.0) -> dict:
     what = (f"{n_rows} of {count} masked rows" if passes == 1 else
             f"all {count} masked rows, {passes} passes")
     return dict(value=n / t, unit=UNIT, cores=blas_threads(), kind="oracle",
+                host_cpus=os.cpu_count(), blas=blas_backend(),
                 sample=f"{what} of {cfg.name} (fp64 NumPy logits over all V={cfg.V} with W "
                        f"converted once, statistics, top-k over the sample), {t:.1f} s")
 
@@ -293,6 +305,7 @@ def run_reference(args, cfg) -> None:
                 scaling="weak", vs_baseline=None, dtype="f64", data="synthetic", impl="reference",
                 config=workload_config(cfg, count),
                 cpu_baseline=dict(value=value, unit=UNIT, cores=blas_threads(), kind="oracle",
+                                  host_cpus=os.cpu_count(), blas=blas_backend(),
                                   sample=f"{rows_per_step} random masked rows per step of "
                                          f"{cfg.name} (W converted to fp64 once)"),
                 e2e=dict(value=value, unit=UNIT, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
