@@ -277,7 +277,7 @@ def cpu_baseline(inp: dict, budget_s: float = 10.0) -> dict:
 def run_reference(args, cfg) -> None:
     """The oracle as the reference arm: rank 0 only, on the host cores.  Each step times the
     oracle on a random sample of the workload's masked rows, sized from a measured per-row
-    cost so that warm-up and timed steps together take about two minutes."""
+    cost so that warm-up and timed steps together take about --ref-seconds (two minutes)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
@@ -290,7 +290,7 @@ def run_reference(args, cfg) -> None:
     t32, n32 = run.time_rows(pick(32))
     per_row = max((t32 - t8) / max(n32 - n8, 1.0), t32 / max(n32, 1.0) * 0.5, 1e-6)
     fixed = max(t8 - n8 * per_row, 0.0)
-    per_step = 120.0 / max(1, args.steps + args.warmup)
+    per_step = args.ref_seconds / max(1, args.steps + args.warmup)
     rows_per_step = int(max(1, min(count, (per_step - fixed) / per_row)))
     for _ in range(args.warmup):
         run.time_rows(pick(rows_per_step))
@@ -440,6 +440,8 @@ def main() -> None:
     ap.add_argument("--config", default="cfg1")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-seconds", type=float, default=120.0,
+                    help="--impl reference: oracle seconds that warm-up and timed steps take together")
     ap.add_argument("--no-full-baseline", action="store_true",
                     help="skip timing the full-logits torch path the method replaces")
     ap.add_argument("--e2e-steps", type=int, default=None)
