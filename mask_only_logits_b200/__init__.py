@@ -490,7 +490,7 @@ class DecodeStep:
         iteration).  Each batch's H_host and M_host must stay valid and unchanged until its
         step has been yielded.
         """
-        B, L, d, V, k = self.B, self.L, self.d, self.V, self.k
+        B, L, d, V = self.B, self.L, self.d, self.V
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
         ps = prep_stream if prep_stream is not None else torch.cuda.Stream(self.device)
         if getattr(self, "_pipe", None) is None:
@@ -568,7 +568,7 @@ class DecodeStep:
         (one per batch) of int32 device buffers shaped like ``sel_buf`` that receive each
         step's packed selection; otherwise only the last step's outputs remain (this
         object's buffers)."""
-        B, L, d, V, k = self.B, self.L, self.d, self.V, self.k
+        B, L, d, V = self.B, self.L, self.d, self.V
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
         ps = prep_stream if prep_stream is not None else torch.cuda.Stream(self.device)
         ob = self._double()
