@@ -531,6 +531,7 @@ def main() -> None:
         prep_stream = torch.cuda.Stream(dev)
         step.run_overlapped([(H, M)] * 3, W, win_lo, win_hi, stream, prep_stream, blk)
         torch.cuda.synchronize(dev)
+        step_peak = torch.cuda.max_memory_allocated(dev) - base_mem   # with the 2nd workspace
 
     def one_step():
         if args.graph:
@@ -631,7 +632,9 @@ def main() -> None:
             gpu_launches=launches,
             memory=dict(peak_step_bytes=int(step_peak),
                         full_logits_fp32_bytes=int(full_logits),
-                        note="peak = torch allocations of the step (outputs + workspace) over the "
+                        workspaces=1 if not overlap else 2,
+                        note="peak = torch allocations of the step (outputs + workspace; two "
+                             "workspaces when staging overlaps the previous step) over the "
                              "resident inputs; full_logits_fp32_bytes = B*L*V fp32 logits"),
             e2e=dict(value=job_rows * e2e_steps / (e2e_ms / 1e3), unit=UNIT,
                      h2d_bytes_per_step=step.h2d_bytes_zero_copy(count),
