@@ -55,13 +55,23 @@ def _check(status: int, where: str) -> None:
         raise DllmError(status, where)
 
 
+def _on_device(t: torch.Tensor, host_ok: bool) -> bool:
+    """Whether the library's kernels can read t: device memory, or (host_ok) page-locked
+    host memory."""
+    return t.is_cuda or (host_ok and t.is_pinned())
+
+
 def _ptr(t: torch.Tensor | None, dtype: torch.dtype | None = None, name: str = "",
-         host_ok: bool = False) -> ctypes.c_void_p:
-    """Device pointer of a tensor; with host_ok, a page-locked CPU tensor is also accepted
-    (the library reads it over the bus; only the step inputs H and M allow this)."""
+         host_ok: bool = False, n: int = 0) -> ctypes.c_void_p:
+    """Device pointer of a tensor of at least n elements; with host_ok, a page-locked CPU
+    tensor is also accepted (the library reads it over the bus; only the step inputs H and
+    M allow this).  The library sees only pointers, so the sizes are checked here: a short
+    buffer is refused before any launch could run past its end."""
     if t is None:
         return ctypes.c_void_p(None)
-    if not t.is_cuda and not (host_ok and t.is_pinned()):
+    if t.numel() < n:
+        raise ValueError(f"{name}: needs at least {n} elements, got {t.numel()}")
+    if not _on_device(t, host_ok):
         raise ValueError(f"{name}: expected a CUDA tensor" +
                          (" or a page-locked (pinned) CPU tensor" if host_ok else ""))
     if not t.is_contiguous():
@@ -91,18 +101,18 @@ def mask_compact(M, row_idx, seq_off, count, ws, stream=None, win_lo=None, win_h
     B, L = M.shape
     if win_lo is None and win_hi is None:
         _check(lib().dllm_mask_compact(_ptr(M, torch.uint8, "M"), B, L,
-                                       _ptr(row_idx, torch.int32, "row_idx"),
-                                       _ptr(seq_off, torch.int32, "seq_off"),
-                                       _ptr(count, torch.int32, "count"), _ptr(ws, None, "ws"),
+                                       _ptr(row_idx, torch.int32, "row_idx", n=B * L),
+                                       _ptr(seq_off, torch.int32, "seq_off", n=B + 1),
+                                       _ptr(count, torch.int32, "count", n=1), _ptr(ws, None, "ws"),
                                        ws.numel() * ws.element_size(), _stream(stream)),
                "dllm_mask_compact")
         return
     _check(lib().dllm_mask_compact_window(_ptr(M, torch.uint8, "M"), B, L,
-                                          _ptr(win_lo, torch.int32, "win_lo"),
-                                          _ptr(win_hi, torch.int32, "win_hi"),
-                                          _ptr(row_idx, torch.int32, "row_idx"),
-                                          _ptr(seq_off, torch.int32, "seq_off"),
-                                          _ptr(count, torch.int32, "count"), _ptr(ws, None, "ws"),
+                                          _ptr(win_lo, torch.int32, "win_lo", n=B),
+                                          _ptr(win_hi, torch.int32, "win_hi", n=B),
+                                          _ptr(row_idx, torch.int32, "row_idx", n=B * L),
+                                          _ptr(seq_off, torch.int32, "seq_off", n=B + 1),
+                                          _ptr(count, torch.int32, "count", n=1), _ptr(ws, None, "ws"),
                                           ws.numel() * ws.element_size(), _stream(stream)),
            "dllm_mask_compact_window")
 
@@ -113,21 +123,22 @@ def mask_compact_noalloc(M, row_idx, seq_off, count, stream=None) -> None:
     on the GPU race on that scratch)."""
     B, L = M.shape
     _check(lib().dllm_mask_compact_noalloc(_ptr(M, torch.uint8, "M"), B, L,
-                                           _ptr(row_idx, torch.int32, "row_idx"),
-                                           _ptr(seq_off, torch.int32, "seq_off"),
-                                           _ptr(count, torch.int32, "count"), _stream(stream)),
+                                           _ptr(row_idx, torch.int32, "row_idx", n=B * L),
+                                           _ptr(seq_off, torch.int32, "seq_off", n=B + 1),
+                                           _ptr(count, torch.int32, "count", n=1), _stream(stream)),
            "dllm_mask_compact_noalloc")
 
 
 def masked_logits(H, M, W, tok, conf, lse, row_idx, seq_off, count, ws, stream=None) -> None:
     B, L = M.shape
     V, d = W.shape
+    n = B * L
     _check(lib().dllm_masked_logits(
-        _ptr(H, torch.bfloat16, "H", True), _ptr(M, torch.uint8, "M", True),
+        _ptr(H, torch.bfloat16, "H", True, n * d), _ptr(M, torch.uint8, "M", True),
         _ptr(W, torch.bfloat16, "W"),
-        B, L, d, V, _ptr(tok, torch.int32, "tok"), _ptr(conf, torch.float32, "conf"),
-        _ptr(lse, torch.float32, "lse"), _ptr(row_idx, torch.int32, "row_idx"),
-        _ptr(seq_off, torch.int32, "seq_off"), _ptr(count, torch.int32, "count"),
+        B, L, d, V, _ptr(tok, torch.int32, "tok", n=n), _ptr(conf, torch.float32, "conf", n=n),
+        _ptr(lse, torch.float32, "lse", n=n), _ptr(row_idx, torch.int32, "row_idx", n=n),
+        _ptr(seq_off, torch.int32, "seq_off", n=B + 1), _ptr(count, torch.int32, "count", n=1),
         _ptr(ws, None, "ws"), ws.numel() * ws.element_size(), _stream(stream)),
         "dllm_masked_logits")
 
@@ -140,18 +151,20 @@ def masked_logits_ex(H, M, W, stats, tok, conf, lse, entropy, margin, row_idx, s
     [win_lo[b], win_hi[b]) get logits (current-block-only decoding)."""
     B, L = M.shape
     V, d = W.shape
-    common = (_ptr(tok, torch.int32, "tok"), _ptr(conf, torch.float32, "conf"),
-              _ptr(lse, torch.float32, "lse"), _ptr(entropy, torch.float32, "entropy"),
-              _ptr(margin, torch.float32, "margin"), _ptr(row_idx, torch.int32, "row_idx"),
-              _ptr(seq_off, torch.int32, "seq_off"), _ptr(count, torch.int32, "count"),
+    n = B * L
+    common = (_ptr(tok, torch.int32, "tok", n=n), _ptr(conf, torch.float32, "conf", n=n),
+              _ptr(lse, torch.float32, "lse", n=n), _ptr(entropy, torch.float32, "entropy", n=n),
+              _ptr(margin, torch.float32, "margin", n=n),
+              _ptr(row_idx, torch.int32, "row_idx", n=n),
+              _ptr(seq_off, torch.int32, "seq_off", n=B + 1), _ptr(count, torch.int32, "count", n=1),
               _ptr(ws, None, "ws"), ws.numel() * ws.element_size(), _stream(stream))
-    ins = (_ptr(H, torch.bfloat16, "H", True), _ptr(M, torch.uint8, "M", True),
+    ins = (_ptr(H, torch.bfloat16, "H", True, n * d), _ptr(M, torch.uint8, "M", True),
            _ptr(W, torch.bfloat16, "W"), B, L, d, V)
     if win_lo is None and win_hi is None:
         _check(lib().dllm_masked_logits_ex(*ins, stats, *common), "dllm_masked_logits_ex")
     else:
-        _check(lib().dllm_masked_logits_window(*ins, _ptr(win_lo, torch.int32, "win_lo"),
-                                               _ptr(win_hi, torch.int32, "win_hi"), stats,
+        _check(lib().dllm_masked_logits_window(*ins, _ptr(win_lo, torch.int32, "win_lo", n=B),
+                                               _ptr(win_hi, torch.int32, "win_hi", n=B), stats,
                                                *common), "dllm_masked_logits_window")
 
 
@@ -162,10 +175,10 @@ def prepare_rows(H, M, d, V, row_idx, seq_off, count, ws, stream=None, win_lo=No
     the bus: only the mask and the masked rows move)."""
     B, L = M.shape
     _check(lib().dllm_prepare_rows(
-        _ptr(H, torch.bfloat16, "H", True), _ptr(M, torch.uint8, "M", True), B, L, d, V,
-        _ptr(win_lo, torch.int32, "win_lo"), _ptr(win_hi, torch.int32, "win_hi"),
-        _ptr(row_idx, torch.int32, "row_idx"), _ptr(seq_off, torch.int32, "seq_off"),
-        _ptr(count, torch.int32, "count"), _ptr(ws, None, "ws"), ws.numel() * ws.element_size(),
+        _ptr(H, torch.bfloat16, "H", True, B * L * d), _ptr(M, torch.uint8, "M", True), B, L, d, V,
+        _ptr(win_lo, torch.int32, "win_lo", n=B), _ptr(win_hi, torch.int32, "win_hi", n=B),
+        _ptr(row_idx, torch.int32, "row_idx", n=B * L), _ptr(seq_off, torch.int32, "seq_off", n=B + 1),
+        _ptr(count, torch.int32, "count", n=1), _ptr(ws, None, "ws"), ws.numel() * ws.element_size(),
         _stream(stream)), "dllm_prepare_rows")
 
 
@@ -173,11 +186,12 @@ def masked_logits_prepared(W, B, L, stats, tok, conf, lse, entropy, margin, coun
                            stream=None) -> None:
     """Second half of masked_logits: the GEMM and its statistics on rows prepared in ``ws``."""
     V, d = W.shape
+    n = B * L
     _check(lib().dllm_masked_logits_prepared(
-        _ptr(W, torch.bfloat16, "W"), B, L, d, V, stats, _ptr(tok, torch.int32, "tok"),
-        _ptr(conf, torch.float32, "conf"), _ptr(lse, torch.float32, "lse"),
-        _ptr(entropy, torch.float32, "entropy"), _ptr(margin, torch.float32, "margin"),
-        _ptr(count, torch.int32, "count"), _ptr(ws, None, "ws"), ws.numel() * ws.element_size(),
+        _ptr(W, torch.bfloat16, "W"), B, L, d, V, stats, _ptr(tok, torch.int32, "tok", n=n),
+        _ptr(conf, torch.float32, "conf", n=n), _ptr(lse, torch.float32, "lse", n=n),
+        _ptr(entropy, torch.float32, "entropy", n=n), _ptr(margin, torch.float32, "margin", n=n),
+        _ptr(count, torch.int32, "count", n=1), _ptr(ws, None, "ws"), ws.numel() * ws.element_size(),
         _stream(stream)), "dllm_masked_logits_prepared")
 
 
@@ -188,14 +202,15 @@ def masked_partials(H, M, W_shard, v_offset, stats, part_m, part_s, part_a, part
     global argmax; plus t and second max when stats != 0) over the shard's vocabulary."""
     B, L = M.shape
     V_shard, d = W_shard.shape
+    n = B * L
     _check(lib().dllm_masked_partials(
-        _ptr(H, torch.bfloat16, "H", True), _ptr(M, torch.uint8, "M", True),
+        _ptr(H, torch.bfloat16, "H", True, n * d), _ptr(M, torch.uint8, "M", True),
         _ptr(W_shard, torch.bfloat16, "W_shard"), B, L, d, V_shard, int(v_offset),
-        _ptr(win_lo, torch.int32, "win_lo"), _ptr(win_hi, torch.int32, "win_hi"), stats,
-        _ptr(part_m, torch.float32, "part_m"), _ptr(part_s, torch.float32, "part_s"),
-        _ptr(part_a, torch.int32, "part_a"), _ptr(part_t, torch.float32, "part_t"),
-        _ptr(part_m2, torch.float32, "part_m2"), _ptr(row_idx, torch.int32, "row_idx"),
-        _ptr(seq_off, torch.int32, "seq_off"), _ptr(count, torch.int32, "count"),
+        _ptr(win_lo, torch.int32, "win_lo", n=B), _ptr(win_hi, torch.int32, "win_hi", n=B), stats,
+        _ptr(part_m, torch.float32, "part_m", n=n), _ptr(part_s, torch.float32, "part_s", n=n),
+        _ptr(part_a, torch.int32, "part_a", n=n), _ptr(part_t, torch.float32, "part_t", n=n),
+        _ptr(part_m2, torch.float32, "part_m2", n=n), _ptr(row_idx, torch.int32, "row_idx", n=n),
+        _ptr(seq_off, torch.int32, "seq_off", n=B + 1), _ptr(count, torch.int32, "count", n=1),
         _ptr(ws, None, "ws"), ws.numel() * ws.element_size(), _stream(stream)),
         "dllm_masked_partials")
 
@@ -204,13 +219,16 @@ def lse_merge(part_m, part_s, part_a, part_t, part_m2, split_stride, n_split, co
               stats, tok, conf, lse, entropy=None, margin=None, stream=None) -> None:
     """Merge per-shard partials (split j of row i at j * split_stride + i) into tok, conf,
     lse (and entropy / margin) for rows below the device-side count."""
+    np_ = max(0, (int(n_split) - 1) * int(split_stride) + int(n_cap))   # partial entries read
     _check(lib().dllm_lse_merge(
-        _ptr(part_m, torch.float32, "part_m"), _ptr(part_s, torch.float32, "part_s"),
-        _ptr(part_a, torch.int32, "part_a"), _ptr(part_t, torch.float32, "part_t"),
-        _ptr(part_m2, torch.float32, "part_m2"), int(split_stride), int(n_split),
-        _ptr(count, torch.int32, "count"), int(n_cap), stats, _ptr(tok, torch.int32, "tok"),
-        _ptr(conf, torch.float32, "conf"), _ptr(lse, torch.float32, "lse"),
-        _ptr(entropy, torch.float32, "entropy"), _ptr(margin, torch.float32, "margin"),
+        _ptr(part_m, torch.float32, "part_m", n=np_), _ptr(part_s, torch.float32, "part_s", n=np_),
+        _ptr(part_a, torch.int32, "part_a", n=np_), _ptr(part_t, torch.float32, "part_t", n=np_),
+        _ptr(part_m2, torch.float32, "part_m2", n=np_), int(split_stride), int(n_split),
+        _ptr(count, torch.int32, "count", n=1), int(n_cap), stats,
+        _ptr(tok, torch.int32, "tok", n=n_cap),
+        _ptr(conf, torch.float32, "conf", n=n_cap), _ptr(lse, torch.float32, "lse", n=n_cap),
+        _ptr(entropy, torch.float32, "entropy", n=n_cap),
+        _ptr(margin, torch.float32, "margin", n=n_cap),
         _stream(stream)), "dllm_lse_merge")
 
 
@@ -219,24 +237,33 @@ def select_unmask_ex(score, row_idx, seq_off, B, L, k, threshold, min_sel, idx, 
                      score_sel=None, stream=None) -> None:
     """Threshold-based selection: per sequence min(k, max(min(min_sel, n), #qualifying))
     best candidates; qualifying = score >= threshold (<= with ascending=True)."""
+    # the per-row inputs are read below the device-side seq_off[B] only (callers may pass
+    # exactly that many entries), so only the [B+1], [B] and [B, k] buffers are checked
+    n, nk = 0, B * k
     _check(lib().dllm_select_unmask_ex(
-        _ptr(score, torch.float32, "score"), _ptr(row_idx, torch.int32, "row_idx"),
-        _ptr(seq_off, torch.int32, "seq_off"), B, L, k, float(threshold), min_sel,
-        1 if ascending else 0, _ptr(win_lo, torch.int32, "win_lo"),
-        _ptr(win_hi, torch.int32, "win_hi"), _ptr(tok, torch.int32, "tok"),
-        _ptr(idx, torch.int32, "idx"), _ptr(n_sel, torch.int32, "n_sel"),
-        _ptr(tok_sel, torch.int32, "tok_sel"), _ptr(score_sel, torch.float32, "score_sel"),
+        _ptr(score, torch.float32, "score", n=n), _ptr(row_idx, torch.int32, "row_idx", n=n),
+        _ptr(seq_off, torch.int32, "seq_off", n=B + 1), B, L, k, float(threshold), min_sel,
+        1 if ascending else 0, _ptr(win_lo, torch.int32, "win_lo", n=B),
+        _ptr(win_hi, torch.int32, "win_hi", n=B), _ptr(tok, torch.int32, "tok", n=n),
+        _ptr(idx, torch.int32, "idx", n=nk), _ptr(n_sel, torch.int32, "n_sel", n=B),
+        _ptr(tok_sel, torch.int32, "tok_sel", n=nk),
+        _ptr(score_sel, torch.float32, "score_sel", n=nk),
         _stream(stream)), "dllm_select_unmask_ex")
 
 
 def select_unmask(conf, row_idx, seq_off, B, L, k, idx, n_sel, win_lo=None, win_hi=None,
                   tok=None, tok_sel=None, conf_sel=None, stream=None) -> None:
+    # the per-row inputs are read below the device-side seq_off[B] only (callers may pass
+    # exactly that many entries), so only the [B+1], [B] and [B, k] buffers are checked
+    n, nk = 0, B * k
     _check(lib().dllm_select_unmask(
-        _ptr(conf, torch.float32, "conf"), _ptr(row_idx, torch.int32, "row_idx"),
-        _ptr(seq_off, torch.int32, "seq_off"), B, L, k, _ptr(win_lo, torch.int32, "win_lo"),
-        _ptr(win_hi, torch.int32, "win_hi"), _ptr(tok, torch.int32, "tok"),
-        _ptr(idx, torch.int32, "idx"), _ptr(n_sel, torch.int32, "n_sel"),
-        _ptr(tok_sel, torch.int32, "tok_sel"), _ptr(conf_sel, torch.float32, "conf_sel"),
+        _ptr(conf, torch.float32, "conf", n=n), _ptr(row_idx, torch.int32, "row_idx", n=n),
+        _ptr(seq_off, torch.int32, "seq_off", n=B + 1), B, L, k,
+        _ptr(win_lo, torch.int32, "win_lo", n=B), _ptr(win_hi, torch.int32, "win_hi", n=B),
+        _ptr(tok, torch.int32, "tok", n=n),
+        _ptr(idx, torch.int32, "idx", n=nk), _ptr(n_sel, torch.int32, "n_sel", n=B),
+        _ptr(tok_sel, torch.int32, "tok_sel", n=nk),
+        _ptr(conf_sel, torch.float32, "conf_sel", n=nk),
         _stream(stream)), "dllm_select_unmask")
 
 
@@ -249,15 +276,18 @@ def decode_step(H, M, W, k, tok, conf, lse, row_idx, seq_off, count, idx, n_sel,
     V, d = W.shape
     fn, name = ((lib().dllm_decode_block_step, "dllm_decode_block_step") if block_only
                 else (lib().dllm_decode_step, "dllm_decode_step"))
+    n, nk = B * L, B * k
     _check(fn(
-        _ptr(H, torch.bfloat16, "H", True), _ptr(M, torch.uint8, "M", True),
+        _ptr(H, torch.bfloat16, "H", True, n * d), _ptr(M, torch.uint8, "M", True),
         _ptr(W, torch.bfloat16, "W"),
-        B, L, d, V, k, _ptr(win_lo, torch.int32, "win_lo"), _ptr(win_hi, torch.int32, "win_hi"),
-        _ptr(tok, torch.int32, "tok"), _ptr(conf, torch.float32, "conf"),
-        _ptr(lse, torch.float32, "lse"), _ptr(row_idx, torch.int32, "row_idx"),
-        _ptr(seq_off, torch.int32, "seq_off"), _ptr(count, torch.int32, "count"),
-        _ptr(idx, torch.int32, "idx"), _ptr(n_sel, torch.int32, "n_sel"),
-        _ptr(tok_sel, torch.int32, "tok_sel"), _ptr(conf_sel, torch.float32, "conf_sel"),
+        B, L, d, V, k, _ptr(win_lo, torch.int32, "win_lo", n=B),
+        _ptr(win_hi, torch.int32, "win_hi", n=B),
+        _ptr(tok, torch.int32, "tok", n=n), _ptr(conf, torch.float32, "conf", n=n),
+        _ptr(lse, torch.float32, "lse", n=n), _ptr(row_idx, torch.int32, "row_idx", n=n),
+        _ptr(seq_off, torch.int32, "seq_off", n=B + 1), _ptr(count, torch.int32, "count", n=1),
+        _ptr(idx, torch.int32, "idx", n=nk), _ptr(n_sel, torch.int32, "n_sel", n=B),
+        _ptr(tok_sel, torch.int32, "tok_sel", n=nk),
+        _ptr(conf_sel, torch.float32, "conf_sel", n=nk),
         _ptr(ws, None, "ws"), ws.numel() * ws.element_size(), _stream(stream)), name)
 
 
@@ -268,20 +298,25 @@ def get_status(stream=None) -> int:
 def debug_lmhead_logits(H, M, W, logits_out, row_idx, seq_off, count, ws, stream=None) -> None:
     B, L = M.shape
     V, d = W.shape
+    n = B * L
     _check(lib().dllm_debug_lmhead_logits(
-        _ptr(H, torch.bfloat16, "H"), _ptr(M, torch.uint8, "M"), _ptr(W, torch.bfloat16, "W"),
-        B, L, d, V, _ptr(logits_out, torch.float32, "logits_out"),
-        _ptr(row_idx, torch.int32, "row_idx"), _ptr(seq_off, torch.int32, "seq_off"),
-        _ptr(count, torch.int32, "count"), _ptr(ws, None, "ws"), ws.numel() * ws.element_size(),
+        _ptr(H, torch.bfloat16, "H", n=n * d), _ptr(M, torch.uint8, "M"),
+        _ptr(W, torch.bfloat16, "W"),
+        B, L, d, V, _ptr(logits_out, torch.float32, "logits_out", n=n * V),
+        _ptr(row_idx, torch.int32, "row_idx", n=n), _ptr(seq_off, torch.int32, "seq_off", n=B + 1),
+        _ptr(count, torch.int32, "count", n=1), _ptr(ws, None, "ws"), ws.numel() * ws.element_size(),
         _stream(stream)), "dllm_debug_lmhead_logits")
 
 
 def debug_lse_merge(part_m, part_s, part_a, tok, conf, lse, stream=None) -> None:
     n_split, n_rows = part_m.shape
+    np_ = n_split * n_rows
     _check(lib().dllm_debug_lse_merge(
-        _ptr(part_m, torch.float32, "part_m"), _ptr(part_s, torch.float32, "part_s"),
-        _ptr(part_a, torch.int32, "part_a"), n_rows, n_split, _ptr(tok, torch.int32, "tok"),
-        _ptr(conf, torch.float32, "conf"), _ptr(lse, torch.float32, "lse"), _stream(stream)),
+        _ptr(part_m, torch.float32, "part_m"), _ptr(part_s, torch.float32, "part_s", n=np_),
+        _ptr(part_a, torch.int32, "part_a", n=np_), n_rows, n_split,
+        _ptr(tok, torch.int32, "tok", n=n_rows),
+        _ptr(conf, torch.float32, "conf", n=n_rows), _ptr(lse, torch.float32, "lse", n=n_rows),
+        _stream(stream)),
         "dllm_debug_lse_merge")
 
 

@@ -46,13 +46,16 @@ class PartialLayout:
         return torch.empty(shape, dtype=torch.float32, device=device)
 
     def fields_of(self, buf: torch.Tensor) -> dict:
-        """Views of the fields of a packed buffer (local or gathered); for a gathered buffer
-        each view starts at rank 0's field and steps by ``split_stride`` per rank, which is
-        how the merge reads it (only the base pointer and the stride are passed on)."""
+        """Views of the fields of a packed buffer (local [fields, n_pad] or gathered [world,
+        fields, n_pad]).  A local field is its n_pad entries.  A gathered field starts at
+        rank 0's field and runs to the end of the buffer: the merge reads field f of rank j
+        at j * split_stride past that start (only the base pointer and the stride are passed
+        on), and the view covers every entry it reads."""
         flat = buf.reshape(-1)
+        gathered = buf.dim() == 3
         out = {}
         for f, name in enumerate(("m", "s", "a", "t", "m2")[:self.fields]):
-            v = flat[f * self.n_pad:(f + 1) * self.n_pad]
+            v = flat[f * self.n_pad:] if gathered else flat[f * self.n_pad:(f + 1) * self.n_pad]
             out[name] = v.view(torch.int32) if name == "a" else v
         return out
 

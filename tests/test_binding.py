@@ -1,0 +1,169 @@
+"""The Python binding's marshalling on a machine without a GPU, against a fake library: every
+wrapper passes as many arguments as the C prototype declares, and refuses a buffer smaller
+than the call may touch (the library sees only pointers, so a short tensor would otherwise
+let a kernel run past its end) before anything is launched."""
+import pytest
+import torch
+
+import mask_only_logits_b200 as dl
+from mask_only_logits_b200 import _abi
+from mask_only_logits_b200.sharded import PartialLayout
+
+B, L, d, V, k = 2, 40, 64, 100, 4
+N = B * L
+S = 0                                               # explicit stream: no CUDA call needed
+
+
+class FakeLib:
+    def __init__(self):
+        self.calls = []
+
+    def __getattr__(self, name):
+        if name not in _abi.PROTOTYPES:
+            raise AttributeError(name)
+
+        def call(*args):
+            assert len(args) == len(_abi.PROTOTYPES[name][1]), (name, len(args))
+            self.calls.append(name)
+            return 0
+        return call
+
+
+@pytest.fixture
+def fake(monkeypatch):
+    lib = FakeLib()
+    monkeypatch.setattr(dl, "lib", lambda: lib)
+    monkeypatch.setattr(dl, "_on_device", lambda t, host_ok: True)
+    return lib
+
+
+def i32(n):
+    return torch.zeros(n, dtype=torch.int32)
+
+
+def f32(n):
+    return torch.zeros(n, dtype=torch.float32)
+
+
+def bufs():
+    return dict(H=torch.zeros(N, d, dtype=torch.bfloat16), M=torch.zeros(B, L, dtype=torch.uint8),
+                W=torch.zeros(V, d, dtype=torch.bfloat16), tok=i32(N), conf=f32(N), lse=f32(N),
+                ent=f32(N), mar=f32(N), row_idx=i32(N), seq_off=i32(B + 1), count=i32(4),
+                idx=i32(B * k), n_sel=i32(B), tok_sel=i32(B * k), conf_sel=f32(B * k),
+                lo=i32(B), hi=i32(B), ws=torch.zeros(64, dtype=torch.uint8))
+
+
+CALLS = {
+    "mask_compact": lambda b: dl.mask_compact(b["M"], b["row_idx"], b["seq_off"], b["count"], b["ws"], S),
+    "mask_compact_window": lambda b: dl.mask_compact(b["M"], b["row_idx"], b["seq_off"], b["count"],
+                                                     b["ws"], S, b["lo"], b["hi"]),
+    "mask_compact_noalloc": lambda b: dl.mask_compact_noalloc(b["M"], b["row_idx"], b["seq_off"],
+                                                              b["count"], S),
+    "masked_logits": lambda b: dl.masked_logits(b["H"], b["M"], b["W"], b["tok"], b["conf"], b["lse"],
+                                                b["row_idx"], b["seq_off"], b["count"], b["ws"], S),
+    "masked_logits_ex": lambda b: dl.masked_logits_ex(
+        b["H"], b["M"], b["W"], 3, b["tok"], b["conf"], b["lse"], b["ent"], b["mar"], b["row_idx"],
+        b["seq_off"], b["count"], b["ws"], S),
+    "masked_logits_window": lambda b: dl.masked_logits_ex(
+        b["H"], b["M"], b["W"], 3, b["tok"], b["conf"], b["lse"], b["ent"], b["mar"], b["row_idx"],
+        b["seq_off"], b["count"], b["ws"], S, b["lo"], b["hi"]),
+    "prepare_rows": lambda b: dl.prepare_rows(b["H"], b["M"], d, V, b["row_idx"], b["seq_off"],
+                                              b["count"], b["ws"], S, b["lo"], b["hi"]),
+    "masked_logits_prepared": lambda b: dl.masked_logits_prepared(
+        b["W"], B, L, 3, b["tok"], b["conf"], b["lse"], b["ent"], b["mar"], b["count"], b["ws"], S),
+    "select_unmask": lambda b: dl.select_unmask(b["conf"], b["row_idx"], b["seq_off"], B, L, k,
+                                                b["idx"], b["n_sel"], b["lo"], b["hi"], b["tok"],
+                                                b["tok_sel"], b["conf_sel"], S),
+    "select_unmask_ex": lambda b: dl.select_unmask_ex(b["conf"], b["row_idx"], b["seq_off"], B, L, k,
+                                                      0.5, 1, b["idx"], b["n_sel"], False, b["lo"],
+                                                      b["hi"], b["tok"], b["tok_sel"], b["conf_sel"], S),
+    "decode_step": lambda b: dl.decode_step(b["H"], b["M"], b["W"], k, b["tok"], b["conf"], b["lse"],
+                                            b["row_idx"], b["seq_off"], b["count"], b["idx"],
+                                            b["n_sel"], b["ws"], b["lo"], b["hi"], b["tok_sel"],
+                                            b["conf_sel"], S),
+    "decode_block_step": lambda b: dl.decode_step(b["H"], b["M"], b["W"], k, b["tok"], b["conf"],
+                                                  b["lse"], b["row_idx"], b["seq_off"], b["count"],
+                                                  b["idx"], b["n_sel"], b["ws"], b["lo"], b["hi"],
+                                                  b["tok_sel"], b["conf_sel"], S, block_only=True),
+    "debug_lmhead_logits": lambda b: dl.debug_lmhead_logits(b["H"], b["M"], b["W"], f32(N * V),
+                                                            b["row_idx"], b["seq_off"], b["count"],
+                                                            b["ws"], S),
+}
+
+# buffers each call must check, with the size it needs
+NEEDS = {
+    "mask_compact": ["row_idx", "seq_off"],
+    "mask_compact_window": ["row_idx", "seq_off", "lo", "hi"],
+    "mask_compact_noalloc": ["row_idx", "seq_off"],
+    "masked_logits": ["H", "tok", "conf", "lse", "row_idx", "seq_off"],
+    "masked_logits_ex": ["H", "tok", "conf", "lse", "ent", "mar", "row_idx", "seq_off"],
+    "masked_logits_window": ["H", "tok", "conf", "lse", "ent", "mar", "row_idx", "seq_off", "lo", "hi"],
+    "prepare_rows": ["H", "row_idx", "seq_off", "lo", "hi"],
+    "masked_logits_prepared": ["tok", "conf", "lse", "ent", "mar"],
+    "select_unmask": ["seq_off", "idx", "n_sel", "tok_sel", "conf_sel", "lo", "hi"],
+    "select_unmask_ex": ["seq_off", "idx", "n_sel", "tok_sel", "conf_sel", "lo", "hi"],
+    "decode_step": ["H", "tok", "conf", "lse", "row_idx", "seq_off", "idx", "n_sel", "tok_sel",
+                    "conf_sel", "lo", "hi"],
+    "decode_block_step": ["H", "tok", "conf", "lse", "row_idx", "seq_off", "idx", "n_sel",
+                          "tok_sel", "conf_sel", "lo", "hi"],
+    "debug_lmhead_logits": ["H", "row_idx", "seq_off"],
+}
+
+
+@pytest.mark.parametrize("name", sorted(CALLS))
+def test_wrapper_arity_and_sizes(fake, name):
+    CALLS[name](bufs())                               # every buffer large enough: one C call
+    assert len(fake.calls) == 1
+    for key in NEEDS[name]:
+        b = bufs()
+        t = b[key]
+        b[key] = t.reshape(-1)[:-1]                   # one element short
+        with pytest.raises(ValueError, match="needs at least"):
+            CALLS[name](b)
+    assert len(fake.calls) == 1                       # nothing reached the library
+
+
+def test_vocab_partials_and_merge_sizes(fake):
+    """Per-shard partials take B*L entries per field; the merge reads n_split strided splits,
+    which the gathered layout's field views cover exactly."""
+    world = 3
+    lay = PartialLayout(N, extended=True)
+    local, gathered = lay.empty(None, "cpu"), lay.empty(world, "cpu")
+    b = bufs()
+    lf, gf = lay.fields_of(local), lay.fields_of(gathered)
+    dl.masked_partials(b["H"], b["M"], b["W"][:50], 0, 3, lf["m"], lf["s"], lf["a"], lf["t"],
+                       lf["m2"], b["row_idx"], b["seq_off"], b["count"], b["ws"], S)
+    dl.lse_merge(gf["m"], gf["s"], gf["a"], gf["t"], gf["m2"], lay.split_stride, world, b["count"],
+                 N, 3, b["tok"], b["conf"], b["lse"], b["ent"], b["mar"], S)
+    assert fake.calls == ["dllm_masked_partials", "dllm_lse_merge"]
+    with pytest.raises(ValueError, match="part_m: needs at least"):
+        dl.masked_partials(b["H"], b["M"], b["W"][:50], 0, 0, f32(N - 1), lf["s"], lf["a"], None,
+                           None, b["row_idx"], b["seq_off"], b["count"], b["ws"], S)
+    short = gathered.reshape(-1)[:(world - 1) * lay.split_stride + N - 1]
+    with pytest.raises(ValueError, match="part_m: needs at least"):
+        dl.lse_merge(short, gf["s"], gf["a"], None, None, lay.split_stride, world, b["count"], N, 0,
+                     b["tok"], b["conf"], b["lse"], stream=S)
+    with pytest.raises(ValueError, match="tok: needs at least"):
+        dl.lse_merge(gf["m"], gf["s"], gf["a"], None, None, lay.split_stride, world, b["count"], N,
+                     0, i32(N - 1), b["conf"], b["lse"], stream=S)
+    # the gathered views reach the last rank's field
+    for v in (gf["m"], gf["s"], gf["a"], gf["t"], gf["m2"]):
+        assert v.numel() >= (world - 1) * lay.split_stride + lay.n_cap
+
+
+def test_debug_merge_sizes(fake):
+    pm, ps, pa = f32(6), f32(6), i32(6)
+    dl.debug_lse_merge(pm.view(2, 3), ps, pa, i32(3), f32(3), f32(3), S)
+    with pytest.raises(ValueError, match="part_s: needs at least"):
+        dl.debug_lse_merge(pm.view(2, 3), f32(5), pa, i32(3), f32(3), f32(3), S)
+    with pytest.raises(ValueError, match="lse: needs at least"):
+        dl.debug_lse_merge(pm.view(2, 3), ps, pa, i32(3), f32(3), f32(2), S)
+
+
+def test_cpu_tensors_are_refused_without_the_fake(monkeypatch):
+    """Without the stand-in device check, an ordinary CPU tensor is refused by name."""
+    monkeypatch.setattr(dl, "lib", lambda: FakeLib())
+    b = bufs()
+    with pytest.raises(ValueError, match="M: expected a CUDA tensor"):
+        dl.mask_compact(torch.zeros(B, L, dtype=torch.uint8), b["row_idx"], b["seq_off"],
+                        b["count"], b["ws"], S)
