@@ -167,3 +167,40 @@ def test_cpu_tensors_are_refused_without_the_fake(monkeypatch):
     with pytest.raises(ValueError, match="M: expected a CUDA tensor"):
         dl.mask_compact(torch.zeros(B, L, dtype=torch.uint8), b["row_idx"], b["seq_off"],
                         b["count"], b["ws"], S)
+
+
+@pytest.mark.parametrize("Bq,kq", [(1, 1), (3, 5), (8, 4), (2, 1024), (7, 3)])
+def test_decode_step_selection_layout(Bq, kq):
+    """The packed selection buffer (one copy brings a step's selection to the host): four
+    parts idx, n_sel, tok_sel, conf_sel, each starting 16-byte aligned, disjoint, with the
+    shapes and dtypes of the selection outputs; host-side byte counts of the end-to-end
+    path."""
+    st = dl.DecodeStep(Bq, 64, 64, 100, kq, device="cpu")
+    views = [st.idx, st.n_sel, st.tok_sel, st.conf_sel]
+    assert [v.shape for v in views] == [(Bq, kq), (Bq,), (Bq, kq), (Bq, kq)]
+    assert [v.dtype for v in views] == [torch.int32, torch.int32, torch.int32, torch.float32]
+    base = st.sel_buf.data_ptr()
+    spans = []
+    for v in views:
+        off = v.data_ptr() - base
+        assert off % 16 == 0
+        spans.append((off, off + v.numel() * 4))
+    spans.sort()
+    assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:]))          # disjoint
+    assert spans[-1][1] <= st.sel_buf.numel() * 4
+    # writing through the views lands in the one buffer the host copies back
+    st.sel_buf.zero_()
+    st.conf_sel.fill_(0.5)
+    assert int((st.sel_buf.view(torch.float32) == 0.5).sum()) == Bq * kq
+    assert st.d2h_bytes() == st.sel_buf.numel() * 4
+    # only the mask and the masked rows of H cross the bus
+    assert st.h2d_bytes_zero_copy(10) == Bq * 64 + 2 * 10 * 64
+
+
+def test_decode_step_validates_policy_and_shapes():
+    with pytest.raises(ValueError, match="policy"):
+        dl.DecodeStep(1, 64, 64, 100, 4, device="cpu", policy="random")
+    with pytest.raises(ValueError, match="k must be"):
+        dl.DecodeStep(1, 64, 64, 100, dl.MAX_K + 1, device="cpu")
+    with pytest.raises(ValueError, match="invalid shapes"):
+        dl.DecodeStep(1, 64, 100, 100, 4, device="cpu")              # d not a multiple of 64
