@@ -174,25 +174,43 @@ def prepare_rows(H, M, d, V, row_idx, seq_off, count, ws, stream=None, win_lo=No
     of the masked rows of H into ``ws``.  H and M may be page-locked CPU tensors (read over
     the bus: only the mask and the masked rows move)."""
     B, L = M.shape
-    _check(lib().dllm_prepare_rows(
-        _ptr(H, torch.bfloat16, "H", True, B * L * d), _ptr(M, torch.uint8, "M", True), B, L, d, V,
-        _ptr(win_lo, torch.int32, "win_lo", n=B), _ptr(win_hi, torch.int32, "win_hi", n=B),
-        _ptr(row_idx, torch.int32, "row_idx", n=B * L), _ptr(seq_off, torch.int32, "seq_off", n=B + 1),
-        _ptr(count, torch.int32, "count", n=1), _ptr(ws, None, "ws"), ws.numel() * ws.element_size(),
-        _stream(stream)), "dllm_prepare_rows")
+    _check(lib().dllm_prepare_rows(*_step_inputs(H, M, B, L, d), B, L, d, V,
+                                   *_prepare_tail(B, L, row_idx, seq_off, count, ws, win_lo, win_hi),
+                                   _stream(stream)), "dllm_prepare_rows")
+
+
+def _step_inputs(H, M, B: int, L: int, d: int) -> tuple:
+    """Pointers of a step's H [B*L, d] and M [B, L] (device or page-locked host memory)."""
+    if tuple(M.shape) != (B, L):
+        raise ValueError(f"M: expected shape ({B}, {L}), got {tuple(M.shape)}")
+    return _ptr(H, torch.bfloat16, "H", True, B * L * d), _ptr(M, torch.uint8, "M", True)
+
+
+def _prepare_tail(B, L, row_idx, seq_off, count, ws, win_lo, win_hi) -> tuple:
+    """Arguments of dllm_prepare_rows after (H, M, B, L, d, V), without the stream."""
+    return (_ptr(win_lo, torch.int32, "win_lo", n=B), _ptr(win_hi, torch.int32, "win_hi", n=B),
+            _ptr(row_idx, torch.int32, "row_idx", n=B * L),
+            _ptr(seq_off, torch.int32, "seq_off", n=B + 1), _ptr(count, torch.int32, "count", n=1),
+            _ptr(ws, None, "ws"), ws.numel() * ws.element_size())
 
 
 def masked_logits_prepared(W, B, L, stats, tok, conf, lse, entropy, margin, count, ws,
                            stream=None) -> None:
     """Second half of masked_logits: the GEMM and its statistics on rows prepared in ``ws``."""
+    _check(lib().dllm_masked_logits_prepared(
+        *_prepared_args(W, B, L, stats, tok, conf, lse, entropy, margin, count, ws),
+        _stream(stream)), "dllm_masked_logits_prepared")
+
+
+def _prepared_args(W, B, L, stats, tok, conf, lse, entropy, margin, count, ws) -> tuple:
+    """Arguments of dllm_masked_logits_prepared, without the stream."""
     V, d = W.shape
     n = B * L
-    _check(lib().dllm_masked_logits_prepared(
-        _ptr(W, torch.bfloat16, "W"), B, L, d, V, stats, _ptr(tok, torch.int32, "tok", n=n),
-        _ptr(conf, torch.float32, "conf", n=n), _ptr(lse, torch.float32, "lse", n=n),
-        _ptr(entropy, torch.float32, "entropy", n=n), _ptr(margin, torch.float32, "margin", n=n),
-        _ptr(count, torch.int32, "count", n=1), _ptr(ws, None, "ws"), ws.numel() * ws.element_size(),
-        _stream(stream)), "dllm_masked_logits_prepared")
+    return (_ptr(W, torch.bfloat16, "W"), B, L, d, V, stats, _ptr(tok, torch.int32, "tok", n=n),
+            _ptr(conf, torch.float32, "conf", n=n), _ptr(lse, torch.float32, "lse", n=n),
+            _ptr(entropy, torch.float32, "entropy", n=n),
+            _ptr(margin, torch.float32, "margin", n=n), _ptr(count, torch.int32, "count", n=1),
+            _ptr(ws, None, "ws"), ws.numel() * ws.element_size())
 
 
 def masked_partials(H, M, W_shard, v_offset, stats, part_m, part_s, part_a, part_t, part_m2,
@@ -237,34 +255,46 @@ def select_unmask_ex(score, row_idx, seq_off, B, L, k, threshold, min_sel, idx, 
                      score_sel=None, stream=None) -> None:
     """Threshold-based selection: per sequence min(k, max(min(min_sel, n), #qualifying))
     best candidates; qualifying = score >= threshold (<= with ascending=True)."""
-    # the per-row inputs are read below the device-side seq_off[B] only (callers may pass
-    # exactly that many entries), so only the [B+1], [B] and [B, k] buffers are checked
-    n, nk = 0, B * k
     _check(lib().dllm_select_unmask_ex(
-        _ptr(score, torch.float32, "score", n=n), _ptr(row_idx, torch.int32, "row_idx", n=n),
-        _ptr(seq_off, torch.int32, "seq_off", n=B + 1), B, L, k, float(threshold), min_sel,
-        1 if ascending else 0, _ptr(win_lo, torch.int32, "win_lo", n=B),
-        _ptr(win_hi, torch.int32, "win_hi", n=B), _ptr(tok, torch.int32, "tok", n=n),
-        _ptr(idx, torch.int32, "idx", n=nk), _ptr(n_sel, torch.int32, "n_sel", n=B),
-        _ptr(tok_sel, torch.int32, "tok_sel", n=nk),
-        _ptr(score_sel, torch.float32, "score_sel", n=nk),
+        *_select_ex_args(score, row_idx, seq_off, B, L, k, threshold, min_sel, idx, n_sel,
+                         ascending, win_lo, win_hi, tok, tok_sel, score_sel),
         _stream(stream)), "dllm_select_unmask_ex")
+
+
+def _select_ex_args(score, row_idx, seq_off, B, L, k, threshold, min_sel, idx, n_sel,
+                    ascending, win_lo, win_hi, tok, tok_sel, score_sel) -> tuple:
+    """Arguments of dllm_select_unmask_ex, without the stream.  The per-row inputs are read
+    below the device-side seq_off[B] only (callers may pass exactly that many entries), so
+    only the [B+1], [B] and [B, k] buffers are size-checked."""
+    nk = B * k
+    return (_ptr(score, torch.float32, "score"), _ptr(row_idx, torch.int32, "row_idx"),
+            _ptr(seq_off, torch.int32, "seq_off", n=B + 1), B, L, k, float(threshold), min_sel,
+            1 if ascending else 0, _ptr(win_lo, torch.int32, "win_lo", n=B),
+            _ptr(win_hi, torch.int32, "win_hi", n=B), _ptr(tok, torch.int32, "tok"),
+            _ptr(idx, torch.int32, "idx", n=nk), _ptr(n_sel, torch.int32, "n_sel", n=B),
+            _ptr(tok_sel, torch.int32, "tok_sel", n=nk),
+            _ptr(score_sel, torch.float32, "score_sel", n=nk))
 
 
 def select_unmask(conf, row_idx, seq_off, B, L, k, idx, n_sel, win_lo=None, win_hi=None,
                   tok=None, tok_sel=None, conf_sel=None, stream=None) -> None:
-    # the per-row inputs are read below the device-side seq_off[B] only (callers may pass
-    # exactly that many entries), so only the [B+1], [B] and [B, k] buffers are checked
-    n, nk = 0, B * k
     _check(lib().dllm_select_unmask(
-        _ptr(conf, torch.float32, "conf", n=n), _ptr(row_idx, torch.int32, "row_idx", n=n),
-        _ptr(seq_off, torch.int32, "seq_off", n=B + 1), B, L, k,
-        _ptr(win_lo, torch.int32, "win_lo", n=B), _ptr(win_hi, torch.int32, "win_hi", n=B),
-        _ptr(tok, torch.int32, "tok", n=n),
-        _ptr(idx, torch.int32, "idx", n=nk), _ptr(n_sel, torch.int32, "n_sel", n=B),
-        _ptr(tok_sel, torch.int32, "tok_sel", n=nk),
-        _ptr(conf_sel, torch.float32, "conf_sel", n=nk),
-        _stream(stream)), "dllm_select_unmask")
+        *_select_args(conf, row_idx, seq_off, B, L, k, idx, n_sel, win_lo, win_hi, tok, tok_sel,
+                      conf_sel), _stream(stream)), "dllm_select_unmask")
+
+
+def _select_args(conf, row_idx, seq_off, B, L, k, idx, n_sel, win_lo, win_hi, tok, tok_sel,
+                 conf_sel) -> tuple:
+    """Arguments of dllm_select_unmask, without the stream (sizes checked as in
+    _select_ex_args)."""
+    nk = B * k
+    return (_ptr(conf, torch.float32, "conf"), _ptr(row_idx, torch.int32, "row_idx"),
+            _ptr(seq_off, torch.int32, "seq_off", n=B + 1), B, L, k,
+            _ptr(win_lo, torch.int32, "win_lo", n=B), _ptr(win_hi, torch.int32, "win_hi", n=B),
+            _ptr(tok, torch.int32, "tok"),
+            _ptr(idx, torch.int32, "idx", n=nk), _ptr(n_sel, torch.int32, "n_sel", n=B),
+            _ptr(tok_sel, torch.int32, "tok_sel", n=nk),
+            _ptr(conf_sel, torch.float32, "conf_sel", n=nk))
 
 
 def decode_step(H, M, W, k, tok, conf, lse, row_idx, seq_off, count, idx, n_sel, ws,
@@ -404,21 +434,28 @@ class DecodeStep:
     def _plain(self) -> bool:
         return self.policy == "confidence" and self.threshold is None
 
-    def _select(self, row_idx, seq_off, win_lo, win_hi, stream) -> None:
-        """The selection of this step's policy on the scores the logits call left."""
+    def _select_call(self, row_idx, seq_off, win_lo, win_hi) -> tuple:
+        """(C entry point, its arguments without the stream, name) of the selection of this
+        step's policy on the scores the logits call leaves."""
         if self._plain():
-            select_unmask(self.conf, row_idx, seq_off, self.B, self.L, self.k, self.idx,
-                          self.n_sel, win_lo, win_hi, self.tok, self.tok_sel, self.conf_sel,
-                          stream)
-            return
+            return (lib().dllm_select_unmask,
+                    _select_args(self.conf, row_idx, seq_off, self.B, self.L, self.k, self.idx,
+                                 self.n_sel, win_lo, win_hi, self.tok, self.tok_sel,
+                                 self.conf_sel), "dllm_select_unmask")
         score = {"confidence": self.conf, "entropy": self.entropy, "margin": self.margin}[self.policy]
         ascending = self.policy == "entropy"
         tau = self.threshold
         if tau is None:                                  # plain top-k of this score
             tau = float("inf") if ascending else float("-inf")
-        select_unmask_ex(score, row_idx, seq_off, self.B, self.L, self.k, tau, self.min_sel,
-                         self.idx, self.n_sel, ascending, win_lo, win_hi, self.tok, self.tok_sel,
-                         self.conf_sel, stream)
+        return (lib().dllm_select_unmask_ex,
+                _select_ex_args(score, row_idx, seq_off, self.B, self.L, self.k, tau,
+                                self.min_sel, self.idx, self.n_sel, ascending, win_lo, win_hi,
+                                self.tok, self.tok_sel, self.conf_sel), "dllm_select_unmask_ex")
+
+    def _select(self, row_idx, seq_off, win_lo, win_hi, stream) -> None:
+        """The selection of this step's policy on the scores the logits call left."""
+        fn, args, name = self._select_call(row_idx, seq_off, win_lo, win_hi)
+        _check(fn(*args, _stream(stream)), name)
 
     def _outputs(self) -> dict:
         out = dict(tok=self.tok, conf=self.conf, lse=self.lse, row_idx=self.row_idx,
@@ -602,31 +639,42 @@ class DecodeStep:
         serving process whose inputs are already on the GPU.  sel_out, if given, is a list
         (one per batch) of int32 device buffers shaped like ``sel_buf`` that receive each
         step's packed selection; otherwise only the last step's outputs remain (this
-        object's buffers)."""
+        object's buffers).
+
+        Every argument but each batch's H and M is validated and turned into pointers once
+        per call, so a step costs the host three library calls and four event operations:
+        short steps stay bound by the device, not by Python."""
         B, L, d, V = self.B, self.L, self.d, self.V
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
         ps = prep_stream if prep_stream is not None else torch.cuda.Stream(self.device)
         ob = self._double()
+        lb = lib()
+        pw = (win_lo, win_hi) if block_only else (None, None)
+        prep = [_prepare_tail(B, L, ob["row_idx"][b], ob["seq_off"][b], ob["count"][b],
+                              ob["ws"][b], *pw) for b in range(2)]
+        gemm = [_prepared_args(W, B, L, self.stats, self.tok, self.conf, self.lse, self.entropy,
+                               self.margin, ob["count"][b], ob["ws"][b]) for b in range(2)]
+        sel = [self._select_call(ob["row_idx"][b], ob["seq_off"][b], win_lo, win_hi)
+               for b in range(2)]
+        s_h, ps_h = _stream(s), _stream(ps)
         prepped = [torch.cuda.Event() for _ in range(2)]
         used = [torch.cuda.Event() for _ in range(2)]
-        pw = (win_lo, win_hi) if block_only else (None, None)
         ps.wait_stream(s)                            # inputs written before the call are ready
         last = 0
         for i, (H, M) in enumerate(batches):
             b = i & 1
-            with torch.cuda.stream(ps):
-                if i >= 2:
-                    ps.wait_event(used[b])           # step i-2 no longer reads this workspace
-                prepare_rows(H, M, d, V, ob["row_idx"][b], ob["seq_off"][b], ob["count"][b],
-                             ob["ws"][b], ps, *pw)
-                prepped[b].record(ps)
-            with torch.cuda.stream(s):
-                s.wait_event(prepped[b])
-                masked_logits_prepared(W, B, L, self.stats, self.tok, self.conf, self.lse,
-                                       self.entropy, self.margin, ob["count"][b], ob["ws"][b], s)
-                self._select(ob["row_idx"][b], ob["seq_off"][b], win_lo, win_hi, s)
-                used[b].record(s)
-                if sel_out is not None:
+            if i >= 2:
+                ps.wait_event(used[b])               # step i-2 no longer reads this workspace
+            _check(lb.dllm_prepare_rows(*_step_inputs(H, M, B, L, d), B, L, d, V, *prep[b], ps_h),
+                   "dllm_prepare_rows")
+            prepped[b].record(ps)
+            s.wait_event(prepped[b])
+            _check(lb.dllm_masked_logits_prepared(*gemm[b], s_h), "dllm_masked_logits_prepared")
+            fn, args, name = sel[b]
+            _check(fn(*args, s_h), name)
+            used[b].record(s)
+            if sel_out is not None:
+                with torch.cuda.stream(s):
                     sel_out[i].copy_(self.sel_buf, non_blocking=True)
             last = b
         if last == 1:                                # leave the last step's compaction in place

@@ -24,6 +24,8 @@ class FakeLib:
 
         def call(*args):
             assert len(args) == len(_abi.PROTOTYPES[name][1]), (name, len(args))
+            if name == "dllm_workspace_bytes":             # sizing, not a library call to log
+                return 4096
             self.calls.append(name)
             return 0
         return call
@@ -204,3 +206,87 @@ def test_decode_step_validates_policy_and_shapes():
         dl.DecodeStep(1, 64, 64, 100, dl.MAX_K + 1, device="cpu")
     with pytest.raises(ValueError, match="invalid shapes"):
         dl.DecodeStep(1, 64, 100, 100, 4, device="cpu")              # d not a multiple of 64
+
+
+class _FakeStream:
+    def __init__(self, log, name):
+        self.log, self.name, self.cuda_stream = log, name, 0
+
+    def wait_stream(self, other):
+        self.log.append(("wait_stream", self.name, other.name))
+
+    def wait_event(self, ev):
+        self.log.append(("wait", self.name, ev.ident))
+
+
+class _FakeEvent:
+    count = 0
+
+    def __init__(self, log):
+        _FakeEvent.count += 1
+        self.log, self.ident = log, _FakeEvent.count
+
+    def record(self, stream):
+        self.log.append(("record", stream.name, self.ident))
+
+
+@pytest.mark.parametrize("policy,threshold", [("confidence", None), ("entropy", 7.0)])
+def test_overlapped_loop_call_order(fake, monkeypatch, policy, threshold):
+    """run_overlapped on fake streams and events: per step one staging call on the staging
+    stream, then the GEMM and the selection on the compute stream after the staging
+    event; from the third step on, the staging of step i waits for the event recorded
+    after step i-2's selection (the workspace it is about to overwrite)."""
+    import contextlib
+    log = []
+    fake.calls = log                                   # library calls go to the same log
+    comp, prep = _FakeStream(log, "s"), _FakeStream(log, "ps")
+    monkeypatch.setattr(torch.cuda, "Event", lambda *a, **k: _FakeEvent(log))
+    monkeypatch.setattr(torch.cuda, "stream", lambda st: contextlib.nullcontext())
+    st = dl.DecodeStep(B, L, d, V, k, device="cpu", policy=policy, threshold=threshold)
+    b = bufs()
+    n_steps = 5
+    sel_out = [torch.empty_like(st.sel_buf) for _ in range(n_steps)]
+    st.run_overlapped([(b["H"], b["M"])] * n_steps, b["W"], stream=comp, prep_stream=prep,
+                      sel_out=sel_out)
+    calls = [e for e in log if isinstance(e, str)]
+    sel_name = "dllm_select_unmask" if policy == "confidence" and threshold is None \
+        else "dllm_select_unmask_ex"
+    assert calls == ["dllm_prepare_rows", "dllm_masked_logits_prepared", sel_name] * n_steps
+    assert log[0] == ("wait_stream", "ps", "s")
+    # walk the log: per step, the events recorded and waited on
+    step = -1
+    used_ev, prepped_ev = {}, {}
+    pending_wait = []
+    for e in log[1:]:
+        if e == "dllm_prepare_rows":
+            step += 1
+            if step >= 2:                              # waited for step-2's used event
+                assert ("ps", used_ev[step - 2]) in pending_wait, step
+            pending_wait = []
+        elif isinstance(e, tuple) and e[0] == "wait":
+            pending_wait.append((e[1], e[2]))
+        elif isinstance(e, tuple) and e[0] == "record" and e[1] == "ps":
+            prepped_ev[step] = e[2]
+        elif e == "dllm_masked_logits_prepared":
+            assert ("s", prepped_ev[step]) in pending_wait       # GEMM after its staging
+        elif isinstance(e, tuple) and e[0] == "record" and e[1] == "s":
+            used_ev[step] = e[2]
+    assert step == n_steps - 1 and len(used_ev) == n_steps
+    # consecutive steps alternate workspaces: the staging events of steps i and i+2 are the
+    # same two events, re-recorded
+    assert prepped_ev[0] == prepped_ev[2] != prepped_ev[1] == prepped_ev[3]
+
+
+def test_overlapped_loop_checks_each_batch(fake, monkeypatch):
+    import contextlib
+    log = []
+    monkeypatch.setattr(torch.cuda, "Event", lambda *a, **k: _FakeEvent(log))
+    monkeypatch.setattr(torch.cuda, "stream", lambda st: contextlib.nullcontext())
+    st = dl.DecodeStep(B, L, d, V, k, device="cpu")
+    b = bufs()
+    comp, prep = _FakeStream(log, "s"), _FakeStream(log, "ps")
+    bad_M = torch.zeros(L, B, dtype=torch.uint8)                   # transposed
+    with pytest.raises(ValueError, match="M: expected shape"):
+        st.run_overlapped([(b["H"], b["M"]), (b["H"], bad_M)], b["W"], stream=comp, prep_stream=prep)
+    with pytest.raises(ValueError, match="H: needs at least"):
+        st.run_overlapped([(b["H"][:-1], b["M"])], b["W"], stream=comp, prep_stream=prep)
