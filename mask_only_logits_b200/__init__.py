@@ -580,29 +580,36 @@ class DecodeStep:
         selected = [torch.cuda.Event() for _ in range(2)]
         done = [torch.cuda.Event() for _ in range(2)]
         pw = (win_lo, win_hi) if block_only else (None, None)
+        # every argument but each batch's H and M, validated and marshalled once per call
+        lb = lib()
+        prep_tail = [_prepare_tail(B, L, pb["row_idx"][b], pb["seq_off"][b], pb["count"][b],
+                                   pb["ws"][b], *pw) for b in range(2)]
+        gemm = [_prepared_args(W, B, L, self.stats, self.tok, self.conf, self.lse, self.entropy,
+                               self.margin, pb["count"][b], pb["ws"][b]) for b in range(2)]
+        sel = [self._select_call(pb["row_idx"][b], pb["seq_off"][b], win_lo, win_hi)
+               for b in range(2)]
+        s_h, ps_h = _stream(s), _stream(ps)
 
         def prep(i, Hh, Mh):
             if not (Hh.is_pinned() and Mh.is_pinned()):
                 raise ValueError("host batches must be page-locked (pinned) CPU tensors")
             b = i & 1
-            with torch.cuda.stream(ps):
-                if i >= 2:
-                    ps.wait_event(used[b])           # step i-2 no longer reads this workspace
-                prepare_rows(Hh, Mh, d, V, pb["row_idx"][b], pb["seq_off"][b], pb["count"][b],
-                             pb["ws"][b], ps, *pw)
-                prepped[b].record(ps)
+            if i >= 2:
+                ps.wait_event(used[b])               # step i-2 no longer reads this workspace
+            _check(lb.dllm_prepare_rows(*_step_inputs(Hh, Mh, B, L, d), B, L, d, V,
+                                        *prep_tail[b], ps_h), "dllm_prepare_rows")
+            prepped[b].record(ps)
 
         def compute(i):
             b = i & 1
-            with torch.cuda.stream(s):
-                s.wait_event(prepped[b])
-                masked_logits_prepared(W, B, L, self.stats, self.tok, self.conf, self.lse,
-                                       self.entropy, self.margin, pb["count"][b], pb["ws"][b], s)
-                if i >= 1:
-                    s.wait_event(done[(i - 1) & 1])  # step i-1's selection has been copied out
-                self._select(pb["row_idx"][b], pb["seq_off"][b], win_lo, win_hi, s)
-                used[b].record(s)
-                selected[b].record(s)
+            s.wait_event(prepped[b])
+            _check(lb.dllm_masked_logits_prepared(*gemm[b], s_h), "dllm_masked_logits_prepared")
+            if i >= 1:
+                s.wait_event(done[(i - 1) & 1])      # step i-1's selection has been copied out
+            fn, args, name = sel[b]
+            _check(fn(*args, s_h), name)
+            used[b].record(s)
+            selected[b].record(s)
             # the selection goes back on the copy stream: the next step's GEMM does not wait
             with torch.cuda.stream(cs):
                 cs.wait_event(selected[b])
