@@ -170,8 +170,9 @@ dllm_status dllm_mask_compact_noalloc(const uint8_t* M, int32_t B, int32_t L,
  *     lse[i] = log sum_v exp(z_v)                        (natural log)
  *     conf[i]= exp(max_v z_v - lse[i])                   (largest softmax probability)
  * No logit is ever written to memory: the GEMM epilogue keeps a running max, sum of
- * exponentials and argmax per row over vocabulary tiles, and a merge kernel (lse_merge)
- * combines the per-split partials.
+ * exponentials and argmax per row over vocabulary tiles, and inside the same kernel the
+ * last work unit to finish a block of rows merges that block's per-split partials
+ * (lse_merge, in vocabulary order, so the lowest token wins a tie of maxima).
  *
  *   H        device, bf16 [B*L, d] row-major.
  *   M        device, uint8 [B, L] row-major.
