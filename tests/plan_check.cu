@@ -7,7 +7,10 @@
 //     part_entries(); the number of writers of an m-tile equals the unit count the
 //     epilogue's merge waits for;
 //   - without remainder holders, the streams of a group differ by at most one tile; with
-//     them, no holder runs more tiles than the busiest stream would without them.
+//     them, no holder runs more tiles than the busiest stream would without them;
+//   - part_entries() fits the partial region the workspace reserves: groups x holders x
+//     rows per m-tile, or (holders + gmax^2) x rows per m-tile when the problem fits one
+//     group (remainder holders), for any masked count up to the capacity.
 // Prints "ok <cases>" and exits 0, or prints the first failing case and exits 1.
 #include <algorithm>
 #include <cstdio>
@@ -36,6 +39,10 @@ bool check_case(int count, int V, int ctas, int cg) {
   std::vector<int> writers(pl.numM, 0);
   std::set<long long> slots_used;
   const long long entries = pl.part_entries();
+  const long long reserve = std::max(static_cast<long long>(pl.ngroups) * ctas * bm,
+                                     pl.ngroups == 1 ? (static_cast<long long>(ctas) + gmax * gmax) * bm
+                                                     : 0LL);
+  if (entries > reserve) return fail("partials exceed the workspace reserve", count, V, ctas, cg);
   for (int h = 0; h < ctas; ++h) {
     bool bad_tile = false;
     auto rec = [&](int m, int n) -> bool {
