@@ -171,7 +171,58 @@ def _window_mask_ignores_seq(M, win_lo, win_hi):
     return ((M != 0) & inside).astype(np.uint8)
 
 
+def _policy_entropy_no_mean(Z):
+    Z = np.asarray(Z, dtype=np.float64)
+    m = Z.max(axis=1, keepdims=True)
+    e = np.exp(Z - m)
+    tot = e.sum(axis=1)
+    ent = np.log(tot)                                  # dropped "- sum p (z - m)"
+    p = e / tot[:, None]
+    s = np.sort(p, axis=1)
+    return ent, s[:, -1] - (s[:, -2] if p.shape[1] > 1 else 0)
+
+
+def _threshold_no_floor(score, row_idx, seq_off, L, k, threshold, min_sel=1, win_lo=None,
+                        win_hi=None):
+    score = np.asarray(score)
+    row_idx = np.asarray(row_idx, dtype=np.int64)
+    seq_off = np.asarray(seq_off, dtype=np.int64)
+    B = seq_off.size - 1
+    idx = np.full((B, k), -1, dtype=np.int32)
+    n_sel = np.zeros(B, dtype=np.int32)
+    for b in range(B):
+        pos = row_idx[seq_off[b]:seq_off[b + 1]] - b * L
+        c = score[seq_off[b]:seq_off[b + 1]]
+        if win_lo is not None:
+            keep = (pos >= win_lo[b]) & (pos < win_hi[b])
+            pos, c = pos[keep], c[keep]
+        n_take = min(k, int((c >= threshold).sum()))             # min_sel floor ignored
+        order = np.lexsort((pos, -c))[:n_take]
+        n_sel[b] = n_take
+        idx[b, :n_take] = pos[order]
+    return idx, n_sel
+
+
+def _partial_local_argmax(Z, v0, v1):
+    Zs = Z[:, v0:v1]
+    m = Zs.max(axis=1)
+    return m, np.exp(Zs - m[:, None]).sum(axis=1), Zs.argmax(axis=1).astype(np.int32)  # no + v0
+
+
+def _mask_compact_not_flattened(M):
+    M = np.asarray(M)
+    B = M.shape[0]
+    bs, ls = np.nonzero(M != 0)
+    row_idx = ls.astype(np.int32)                                 # l instead of b * L + l
+    per_seq = (M != 0).sum(axis=1)
+    return row_idx, np.concatenate([[0], np.cumsum(per_seq)]).astype(np.int32), int(row_idx.size)
+
+
 MUTATIONS = {
+    "entropy_drops_mean_term": ("row_policy_stats", _policy_entropy_no_mean),
+    "threshold_ignores_min_sel": ("select_unmask_threshold", _threshold_no_floor),
+    "partial_argmax_not_global": ("partial_stats", _partial_local_argmax),
+    "compact_positions_not_flattened": ("mask_compact", _mask_compact_not_flattened),
     "block_window_closed": ("window_mask", _window_mask_closed),
     "block_window_first_seq_only": ("window_mask", _window_mask_ignores_seq),
     "entropy_log2": ("row_policy_stats", _policy_entropy_log2),
