@@ -290,3 +290,33 @@ def test_overlapped_loop_checks_each_batch(fake, monkeypatch):
         st.run_overlapped([(b["H"], b["M"]), (b["H"], bad_M)], b["W"], stream=comp, prep_stream=prep)
     with pytest.raises(ValueError, match="H: needs at least"):
         st.run_overlapped([(b["H"][:-1], b["M"])], b["W"], stream=comp, prep_stream=prep)
+
+
+@pytest.mark.parametrize("policy,threshold,block_only,expected", [
+    ("confidence", None, False, ["dllm_decode_step"]),
+    ("confidence", None, True, ["dllm_decode_block_step"]),
+    ("confidence", 0.5, False, ["dllm_masked_logits_ex", "dllm_select_unmask_ex"]),
+    ("entropy", None, False, ["dllm_masked_logits_ex", "dllm_select_unmask_ex"]),
+    ("margin", 0.1, True, ["dllm_masked_logits_window", "dllm_select_unmask_ex"]),
+])
+def test_decode_step_run_calls(fake, policy, threshold, block_only, expected):
+    """DecodeStep.run: the plain confidence top-k is one library call (the whole step);
+    every other policy is the extended logits call and the threshold selection; block-only
+    steps take the windowed entry points."""
+    st = dl.DecodeStep(B, L, d, V, k, device="cpu", policy=policy, threshold=threshold)
+    b = bufs()
+    st.run(b["H"], b["M"], b["W"], b["lo"], b["hi"], S, block_only=block_only)
+    assert fake.calls == expected
+
+
+def test_vocab_sharded_step_one_rank_calls(fake):
+    """One-rank vocabulary-parallel step: partials on the whole vocabulary, the merge (no
+    collective), the selection."""
+    from mask_only_logits_b200.sharded import VocabShardedStep
+    vs = VocabShardedStep(B, L, d, V, k, device="cpu")
+    b = bufs()
+    out = vs.run(b["H"], b["M"], b["W"], stream=S)
+    assert fake.calls == ["dllm_masked_partials", "dllm_lse_merge", "dllm_select_unmask"]
+    assert out["idx"].shape == (B, k)
+    with pytest.raises(ValueError, match="W_shard"):
+        vs.run(b["H"], b["M"], b["W"][:-1], stream=S)
