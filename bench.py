@@ -468,6 +468,9 @@ def main() -> None:
         run_reference(args, cfg)
         return
 
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: the library's arm needs a CUDA device (there is no CPU "
+                         "fallback); --impl reference times the oracle on the host")
     if args.shard == "vocab":
         run_vocab_sharded(args, cfg)
         return

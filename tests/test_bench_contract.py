@@ -120,3 +120,15 @@ def test_reference_arm_other_ranks_do_nothing():
                      dict(RANK="1", WORLD_SIZE="2"))
     assert res.returncode == 0, res.stderr
     assert res.stdout.strip() == ""
+
+
+def test_library_arm_refuses_to_run_without_a_gpu():
+    """The library's arm has no CPU fallback: on a machine without CUDA it exits non-zero
+    at once, naming the reason, and prints no result line."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present")
+    res = _run_bench(["--config", "cfg0", "--steps", "3", "--warmup", "3"])
+    assert res.returncode != 0
+    assert "needs a CUDA device" in res.stderr
+    assert res.stdout.strip() == ""
