@@ -320,3 +320,34 @@ def test_vocab_sharded_step_one_rank_calls(fake):
     assert out["idx"].shape == (B, k)
     with pytest.raises(ValueError, match="W_shard"):
         vs.run(b["H"], b["M"], b["W"][:-1], stream=S)
+
+
+@pytest.mark.parametrize("n_cap,extended,world", [(1, False, 1), (7, False, 3), (130, True, 4),
+                                                  (4096, True, 2)])
+def test_partial_layout_addresses(n_cap, extended, world):
+    """Packed partials: each rank's local fields, gathered in rank order, are found by the
+    merge at (field view start) + j * split_stride for rank j, with every field's start
+    16-byte aligned; the gathered views cover every entry read."""
+    lay = PartialLayout(n_cap, extended)
+    names = ("m", "s", "a", "t", "m2")[:lay.fields]
+    locals_ = []
+    for j in range(world):
+        loc = lay.empty(None, "cpu")
+        f = lay.fields_of(loc)
+        for q, name in enumerate(names):
+            vals = torch.arange(n_cap, dtype=torch.int32) + 1000 * q + 100000 * j
+            if name == "a":
+                f[name][:n_cap] = vals
+            else:
+                f[name][:n_cap] = vals.float()
+        locals_.append(loc)
+    gathered = torch.stack(locals_)                  # what the all-gather produces
+    gf = lay.fields_of(gathered)
+    for q, name in enumerate(names):
+        v = gf[name]
+        assert (v.data_ptr() - gathered.data_ptr()) % 16 == 0
+        assert v.numel() >= (world - 1) * lay.split_stride + n_cap
+        for j in range(world):
+            got = v[j * lay.split_stride: j * lay.split_stride + n_cap]
+            want = torch.arange(n_cap, dtype=torch.int32) + 1000 * q + 100000 * j
+            assert torch.equal(got if name == "a" else got.to(torch.int32), want)
