@@ -366,12 +366,17 @@ def test_overlapped_steps_match_single_steps(dl):
     what single steps select, batch by batch, and leave the last step's outputs."""
     for name in ("cfg0", "cfg1", "cfg4"):            # cfg1: the launch mode bench.py times
         cfg = WL.CONFIGS[name]
-        inps = [WL.make_inputs(cfg, seed=s) for s in (21, 22, 23, 24, 25)]
-        W = inps[0]["W"].cuda()
-        lo = None if inps[0]["win_lo"] is None else torch.from_numpy(inps[0]["win_lo"]).cuda()
-        hi = None if inps[0]["win_hi"] is None else torch.from_numpy(inps[0]["win_hi"]).cuda()
+        inp0 = WL.make_inputs(cfg, seed=21)
+        host = [(inp0["H"], inp0["M"])]
+        for sd in (22, 23, 24, 25):              # more batches: new H and mask, same W
+            g = torch.Generator().manual_seed(sd)
+            H = (torch.randn(cfg.B * cfg.L, cfg.d, generator=g) * cfg.h_std).to(torch.bfloat16)
+            host.append((H, WL.make_mask(cfg, g)))
+        W = inp0["W"].cuda()
+        lo = None if inp0["win_lo"] is None else torch.from_numpy(inp0["win_lo"]).cuda()
+        hi = None if inp0["win_hi"] is None else torch.from_numpy(inp0["win_hi"]).cuda()
         step = dl.DecodeStep(cfg.B, cfg.L, cfg.d, cfg.V, cfg.k)
-        dev = [(inp["H"].cuda(), inp["M"].cuda()) for inp in inps]
+        dev = [(H.cuda(), M.cuda()) for H, M in host]
         expected = []
         for H, M in dev:
             step.run(H, M, W, lo, hi)
@@ -384,5 +389,5 @@ def test_overlapped_steps_match_single_steps(dl):
             assert torch.equal(got, exp), name
         assert torch.equal(step.sel_buf, expected[-1])
         c = int(out["count"][0])
-        ref_rows, _, ref_c = O.mask_compact(inps[-1]["M"].numpy())
+        ref_rows, _, ref_c = O.mask_compact(host[-1][1].numpy())
         assert c == ref_c and np.array_equal(out["row_idx"][:c].cpu().numpy(), ref_rows)
