@@ -431,6 +431,12 @@ class DecodeStep:
                 buf[o[2]:o[2] + B * k].view(B, k),
                 buf[o[3]:o[3] + B * k].view(torch.float32).view(B, k))
 
+    def _check_W(self, W) -> None:
+        """W must be this step's [V, d] projection: the staging and the GEMM halves of a step
+        take their shapes from this object and from W respectively."""
+        if tuple(W.shape) != (self.V, self.d):
+            raise ValueError(f"W: expected shape ({self.V}, {self.d}), got {tuple(W.shape)}")
+
     def _plain(self) -> bool:
         return self.policy == "confidence" and self.threshold is None
 
@@ -470,6 +476,7 @@ class DecodeStep:
     def run(self, H, M, W, win_lo=None, win_hi=None, stream=None, block_only=False) -> dict:
         """One step on device tensors.  block_only=True (windows required): logits for the
         masked rows inside the windows only; tok/conf/lse/row_idx then cover those rows."""
+        self._check_W(W)
         if self._plain():
             decode_step(H, M, W, self.k, self.tok, self.conf, self.lse, self.row_idx,
                         self.seq_off, self.count, self.idx, self.n_sel, self.ws, win_lo, win_hi,
@@ -562,6 +569,7 @@ class DecodeStep:
         iteration).  Each batch's H_host and M_host must stay valid and unchanged until its
         step has been yielded.
         """
+        self._check_W(W)
         B, L, d, V = self.B, self.L, self.d, self.V
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
         ps = prep_stream if prep_stream is not None else torch.cuda.Stream(self.device)
@@ -651,6 +659,7 @@ class DecodeStep:
         Every argument but each batch's H and M is validated and turned into pointers once
         per call, so a step costs the host three library calls and four event operations:
         short steps stay bound by the device, not by Python."""
+        self._check_W(W)
         B, L, d, V = self.B, self.L, self.d, self.V
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
         ps = prep_stream if prep_stream is not None else torch.cuda.Stream(self.device)

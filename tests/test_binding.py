@@ -351,3 +351,19 @@ def test_partial_layout_addresses(n_cap, extended, world):
             got = v[j * lay.split_stride: j * lay.split_stride + n_cap]
             want = torch.arange(n_cap, dtype=torch.int32) + 1000 * q + 100000 * j
             assert torch.equal(got if name == "a" else got.to(torch.int32), want)
+
+
+def test_decode_step_refuses_a_w_of_another_shape(fake, monkeypatch):
+    import contextlib
+    log = []
+    monkeypatch.setattr(torch.cuda, "Event", lambda *a, **k: _FakeEvent(log))
+    monkeypatch.setattr(torch.cuda, "stream", lambda st: contextlib.nullcontext())
+    st = dl.DecodeStep(B, L, d, V, k, device="cpu")
+    b = bufs()
+    W_bad = torch.zeros(V + 1, d, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="W: expected shape"):
+        st.run(b["H"], b["M"], W_bad, stream=S)
+    with pytest.raises(ValueError, match="W: expected shape"):
+        st.run_overlapped([(b["H"], b["M"])], W_bad, stream=_FakeStream(log, "s"),
+                          prep_stream=_FakeStream(log, "ps"))
+    assert fake.calls == []
