@@ -59,6 +59,15 @@ def stats(z):
     return tok, m, lse, conf
 
 
+def top2_gap(z):
+    """Largest logit minus the second largest, by sorting the row (0 when the maximum occurs
+    twice; infinite for a one-entry row, which has no second logit)."""
+    if len(z) < 2:
+        return math.inf
+    zs = sorted(z, reverse=True)
+    return zs[0] - zs[1]
+
+
 def policy_stats(z):
     """(entropy, margin) of softmax(z) by definition: -sum p ln p and p_(1) - p_(2)."""
     m = max(z)

@@ -316,8 +316,79 @@ def check_block_step(o):
             assert np.array_equal(blk[key], np.asarray(full[key])[sel]), key
 
 
+def check_top2_gap(o):
+    """The near-tie exemption of the parity tests rests on top2_gap: pinned against a sorted
+    brute force, exactly 0 on a repeated maximum, infinite when a row has one logit."""
+    rng = np.random.default_rng(17)
+    for V in (1, 2, 3, 9, 64):
+        Z = rng.standard_normal((6, V)) * 2.0
+        if V >= 2:
+            Z[1, 0] = Z[1, V - 1] = Z[1].max() + 1.0  # the maximum twice: gap exactly 0
+            Z[2, :] = 0.5                            # every entry tied
+        if V >= 3:
+            top = Z[3].max() + 1.0
+            Z[3, 0] = top                            # unique maximum ...
+            Z[3, 1] = Z[3, 2] = top - 0.25           # ... over a repeated second: gap 0.25
+        got = o.top2_gap(Z)
+        want = [brute.top2_gap(row) for row in Z.tolist()]
+        assert got.shape == (Z.shape[0],)
+        assert got.tolist() == want, (V, got, want)
+        if V == 1:
+            assert np.all(np.isinf(got))
+        else:
+            assert got[1] == 0.0 and got[2] == 0.0
+        if V >= 3:
+            assert got[3] == 0.25
+
+
+def _onehot_case(V, d, targets, rng):
+    """Rows of H that are unit vectors e_r, so that row r's logits are column r of W; W's
+    column r gets its maximum at vocabulary entry targets[r].  Further rows are random."""
+    n_hot = len(targets)
+    H = np.zeros((n_hot + 3, d), np.float32)
+    H[:n_hot, :n_hot] = np.eye(n_hot)
+    H[n_hot:] = rng.standard_normal((3, d))
+    W = (rng.standard_normal((V, d)) * 0.25).astype(np.float32)
+    for r, t in enumerate(targets):
+        W[:, r] = np.clip(W[:, r], -1.0, 1.0)
+        W[t, r] = 4.0
+    return _bits(torch.tensor(H).bfloat16().float().numpy()), \
+        _bits(torch.tensor(W).bfloat16().float().numpy())
+
+
+def check_chunked_rows(o):
+    """rows_stats_chunked, the path of every full-vocabulary parity check, against the brute
+    force per row, with the maximum planted on the last and first columns of chunks: small
+    chunks (1, 5, 7) on V = 33 and the default chunk at V = 8193 and V = 16385."""
+    rng = np.random.default_rng(19)
+    cases = [(33, 1, [0, 32, 16]), (33, 5, [4, 5, 32, 29]), (33, 7, [6, 13, 7, 32]),
+             (33, 64, [32, 0]),
+             (8193, o.V_CHUNK, [8191, 8192, 0]), (16385, o.V_CHUNK, [8191, 8192, 16383, 16384])]
+    for V, chunk, targets in cases:
+        d = 8
+        Hb, Wb = _onehot_case(V, d, targets, rng)
+        tok, m, lse, conf, gap = o.rows_stats_chunked(Hb, Wb, chunk=chunk)
+        Hl, Wl = _bf16_list(Hb), _bf16_list(Wb)
+        for r in range(Hb.shape[0]):
+            z = brute.row_logits(Hl[r], Wl)
+            t, mm, ll, cc = brute.stats(z)
+            assert int(tok[r]) == t, (V, chunk, r, int(tok[r]), t)
+            if r < len(targets):
+                assert t == targets[r]
+            np.testing.assert_allclose(m[r], mm, rtol=1e-13)
+            np.testing.assert_allclose(lse[r], ll, rtol=1e-12)
+            np.testing.assert_allclose(conf[r], cc, rtol=1e-12)
+            np.testing.assert_allclose(gap[r], brute.top2_gap(z), rtol=1e-12, atol=1e-12 * abs(mm))
+        # the same rows unchunked: one matmul over the whole vocabulary
+        Z = o.logits_rows(o.bf16_bits_to_f64(Hb), o.bf16_bits_to_f64(Wb))
+        t2, m2, l2, c2 = o.row_stats(Z)
+        assert tok.tolist() == t2.tolist()
+        np.testing.assert_allclose(lse, l2, rtol=1e-13)
+        np.testing.assert_allclose(conf, c2, rtol=1e-13)
+
+
 ALL_CHECKS = [check_handworked, check_topk_ties, check_compact, check_brute_random,
               check_closed_forms, check_library_routines, check_invariants,
               check_mask_only_equals_full, check_merge_split_invariance,
               check_policy_closed_forms, check_policy_library_and_brute, check_threshold_select,
-              check_block_step]
+              check_block_step, check_top2_gap, check_chunked_rows]

@@ -218,7 +218,31 @@ def _mask_compact_not_flattened(M):
     return row_idx, np.concatenate([[0], np.cumsum(per_seq)]).astype(np.int32), int(row_idx.size)
 
 
+def _top2_gap_zero(Z):
+    return np.zeros(Z.shape[0])                                    # every near-tie excused
+
+
+def _make_chunked_drops_last_column(mod):
+    def rows_stats_chunked(H_rows_bits, W_bits, chunk=mod.V_CHUNK, with_policy=False, W64=None):
+        H64 = mod.bf16_bits_to_f64(H_rows_bits)
+        V = W_bits.shape[0]
+        Z = np.zeros((H64.shape[0], V), dtype=np.float64)
+        for v0 in range(0, V, chunk):
+            v1 = min(V, v0 + chunk)
+            Wc = mod.bf16_bits_to_f64(W_bits[v0:v1 - 1])             # last column of the chunk lost
+            Z[:, v0:v1 - 1] = mod.logits_rows(H64, Wc)
+        tok, m, lse, conf = mod.row_stats(Z)
+        gap = mod.top2_gap(Z)
+        if with_policy:
+            entropy, margin = mod.row_policy_stats(Z)
+            return tok, m, lse, conf, gap, entropy, margin
+        return tok, m, lse, conf, gap
+    return rows_stats_chunked
+
+
 MUTATIONS = {
+    "top2_gap_always_zero": ("top2_gap", _top2_gap_zero),
+    "chunk_drops_last_column": ("rows_stats_chunked", _make_chunked_drops_last_column),
     "entropy_drops_mean_term": ("row_policy_stats", _policy_entropy_no_mean),
     "threshold_ignores_min_sel": ("select_unmask_threshold", _threshold_no_floor),
     "partial_argmax_not_global": ("partial_stats", _partial_local_argmax),
@@ -244,11 +268,16 @@ MUTATIONS = {
 }
 
 
+FACTORY_MUTATIONS = {"chunk_drops_last_column"}
+
+
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
 def test_pins_catch_planted_mistake(name):
     attr, bad = MUTATIONS[name]
     mod = _fresh_copy()
     P.ALL_CHECKS[0](mod)            # the unmodified copy passes
+    if name in FACTORY_MUTATIONS:   # mutants that call back into the copy they replace
+        bad = bad(mod)
     setattr(mod, attr, bad)
     caught = []
     for check in P.ALL_CHECKS:
