@@ -4,12 +4,16 @@ One step = the whole hot path on one batch: mask compaction, masked-row gather, 
 tensor-core LM head with the fused softmax-statistics epilogue, lse_merge and the
 per-sequence top-k unmask selection (``dllm_decode_step``).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config cfg1] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config cfg3_r0.9] [--impl ours|reference]
 
-Prints ONE JSON line (rank 0).  ``value`` = masked rows per second over the whole job
-(device time, inputs resident in HBM); ``e2e`` = the same through ``DecodeStep.run_host``
-with the step's H and mask copied from pinned host memory and the selection copied back,
-every step.  Under torchrun each rank runs its own replica of the workload (weak scaling,
+The default workload is the largest one that fits one GPU: B1 L131072 d4096 V126464 with
+90% of the positions masked (the 128k-context, high-mask-ratio case of the Mosaic page,
+Fig. 3, where the logits are the memory peak).  Prints ONE JSON line (rank 0).  ``value``
+= masked rows per second over the whole job (device time, inputs resident in HBM);
+``e2e`` = the same through ``DecodeStep.run_host_pipeline`` with each step's mask and
+masked rows of H read from pinned host memory and the selection copied back, every step.
+``config`` names the workload only (identical in both arms); how the steps were launched
+is under ``run``.  Under torchrun each rank runs its own replica of the workload (weak scaling,
 no data-path collective): the decode steps of independent batches share nothing.
 ``--impl reference`` times the fp64 CPU oracle on the host cores instead.
 """
@@ -99,15 +103,25 @@ def gemm_paired(variant: int, count: int) -> bool:
     return variant == 2 or (variant == 0 and 128 < count <= 16384)
 
 
+# A timed region at least this long runs in the regime of the measured sustained bf16 rate
+# (a seconds-long GEMM loop under the 1 kW power cap); shorter ones in the burst regime.
+LONG_REGION_S = 1.0
+
+
 def gemm_roofline(cfg, count: int, peaks: dict, gemm_s: float, paired: bool, kernel: str,
-                  power_capped: bool = False) -> dict:
+                  region_s: float = 0.0, sm_mhz: float | None = None) -> dict:
     """Roofline of the dominant kernel (the masked LM-head GEMM with its fused epilogue):
     the tensor pipe when its flops take longer than its bytes at the measured peaks, else
     HBM.  Algorithmic work per launch: 2 * count * V * d flops; bytes = W once (2 V d) plus
-    the gathered masked rows once (2 count d).  The tensor peak is the measured sustained
-    bf16 GEMM rate when the clock record shows the 1 kW power cap acting during the timed
-    region (the GEMM then runs in the same regime as that measurement), else the burst
-    rate; both fractions are reported."""
+    the gathered masked rows once (2 count d).
+
+    The tensor peak follows the length of the timed region the GEMM ran in, fixed in
+    advance: the measured burst bf16 rate for a short region (the kernel in the burst
+    regime, before the power cap takes hold), the measured sustained rate when the region
+    lasts LONG_REGION_S or more (steps of a long loop, as that figure was measured).  Both
+    fractions are always reported.  With the median SM clock of the region, the GEMM's
+    duration in clock cycles and its rate per GHz are reported too, so that runs at
+    different capped clocks can be compared."""
     flops = 2.0 * count * cfg.V * cfg.d
     gemm_bytes = 2.0 * cfg.V * cfg.d + 2.0 * count * cfg.d
     tensor_bound = flops / (peaks["bf16_tflops"] * 1e12) >= gemm_bytes / (peaks["hbm_gbs"] * 1e9)
@@ -119,56 +133,159 @@ def gemm_roofline(cfg, count: int, peaks: dict, gemm_s: float, paired: bool, ker
     gbs = gemm_bytes / gemm_s / 1e9
     if tensor_bound:
         sustained = peaks.get("bf16_tflops_sustained")
-        use_sustained = power_capped and sustained is not None
+        use_sustained = region_s >= LONG_REGION_S and sustained is not None
         peak = sustained if use_sustained else peaks["bf16_tflops"]
         out.update(achieved=tflops, peak=peak, unit="TFLOP/s", frac=tflops / peak,
                    frac_of_burst=tflops / peaks["bf16_tflops"],
                    frac_of_sustained=tflops / sustained if sustained else None,
                    peak_source=peaks["source"] + (
-                       " sustained bf16 GEMM (sw_power_cap active during the timed region)"
-                       if use_sustained else " burst bf16 GEMM"),
+                       f" sustained bf16 GEMM (timed region of {region_s:.1f} s >= "
+                       f"{LONG_REGION_S:g} s)" if use_sustained else
+                       f" burst bf16 GEMM (timed region of {region_s:.3f} s)"),
                    achieved_gbs=gbs)
     else:
         out.update(achieved=gbs, peak=peaks["hbm_gbs"], unit="GB/s", frac=gbs / peaks["hbm_gbs"],
                    peak_source=peaks["source"] + " (HBM copy)", achieved_tflops=tflops)
     out.update(gemm_ms_avg=gemm_s * 1e3, algorithmic_bytes=gemm_bytes, algorithmic_flops=flops,
                traffic=measured_traffic(cfg.name, kernel))
+    if sm_mhz:
+        out.update(sm_mhz_median=sm_mhz, gemm_mcycles=gemm_s * sm_mhz,
+                   tflops_per_ghz=tflops / (sm_mhz / 1e3))
     return out
 
 
 # ------------------------------------------------------------------------------ clocks
+_REASON_NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+
+def _nvml_reason_bits(nv) -> dict:
+    """NVML's clock-event reason bits for the four reasons the record reports."""
+    g = lambda new, old: getattr(nv, new, getattr(nv, old, 0))
+    return {"hw_slowdown": g("nvmlClocksEventReasonHwSlowdown", "nvmlClocksThrottleReasonHwSlowdown"),
+            "hw_thermal_slowdown": g("nvmlClocksEventReasonHwThermalSlowdown",
+                                     "nvmlClocksThrottleReasonHwThermalSlowdown"),
+            "sw_thermal_slowdown": g("nvmlClocksEventReasonSwThermalSlowdown",
+                                     "nvmlClocksThrottleReasonSwThermalSlowdown"),
+            "sw_power_cap": g("nvmlClocksEventReasonSwPowerCap", "nvmlClocksThrottleReasonSwPowerCap")}
+
+
+def summarize_clock_samples(samples: list) -> dict:
+    """Median SM clock, the highest max clock, median power and every reason seen, over
+    samples of (sm_mhz, max_mhz, power_w, set of active reason names)."""
+    if not samples:
+        return dict(sm_mhz=None, sm_max_mhz=None, reasons=[], samples=0)
+    sm = [x[0] for x in samples]
+    pw = [x[2] for x in samples if x[2] is not None]
+    reasons = sorted(set().union(*[x[3] for x in samples]))
+    return dict(sm_mhz=statistics.median(sm), sm_max_mhz=max(x[1] for x in samples),
+                reasons=reasons, samples=len(samples),
+                power_w=statistics.median(pw) if pw else None)
+
+
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    """SM clock, power and throttle reasons of the GPU the bench runs on, sampled while the
+    timed region runs: read-only NVML queries from a thread every `period_ms`, plus one
+    sample as the region starts and one as it ends, so that even a region of a few
+    milliseconds carries its own record.  Falls back to an `nvidia-smi --query-gpu` loop
+    when NVML cannot be loaded."""
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int, period_ms: int = 50):
-        self.gpu = gpu_index
+    def __init__(self, device, period_ms: int = 20):
+        self.device = device
         self.period = period_ms
-        self.proc = None
-        self.lines: list[str] = []
+        self.samples: list = []
+        self.source = None
+        self._nv = self._handle = None
+        self._stop = threading.Event()
         self._t = None
+        self.proc = None
 
-    def __enter__(self):
+    # ---- NVML
+    def _open_nvml(self) -> bool:
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            props = torch.cuda.get_device_properties(self.device)
+            bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+            self._handle = nv.nvmlDeviceGetHandleByPciBusId(bus)
+            self._nv = nv
+            self._bits = _nvml_reason_bits(nv)
+            self._max = nv.nvmlDeviceGetMaxClockInfo(self._handle, nv.NVML_CLOCK_SM)
+            self._sample()
+            return True
+        except Exception:  # noqa: BLE001 - no NVML: fall back to nvidia-smi
+            self._nv = None
+            return False
+
+    def _sample(self):
+        nv, h = self._nv, self._handle
+        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+        try:
+            pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+        except Exception:  # noqa: BLE001
+            pw = None
+        get = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        bits = get(h)
+        active = {name for name, b in self._bits.items() if b and bits & b}
+        self.samples.append((float(sm), float(self._max), pw, active))
+
+    def _loop(self):
+        while not self._stop.wait(self.period / 1000.0):
+            try:
+                self._sample()
+            except Exception:  # noqa: BLE001
+                return
+
+    # ---- nvidia-smi fallback
+    def _open_smi(self):
+        idx = torch.device(self.device).index or 0
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                ["nvidia-smi", f"--id={idx}", f"--query-gpu={self.QUERY}",
                  "--format=csv,noheader,nounits", f"-lms={self.period}"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t = threading.Thread(target=self._read_smi, daemon=True)
             self._t.start()
         except OSError:
             self.proc = None
+
+    def _read_smi(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm, mx, pw = float(parts[1]), float(parts[2]), float(parts[3])
+            except ValueError:
+                continue
+            active = {n for n, f in zip(_REASON_NAMES, parts[5:9]) if f.lower() == "active"}
+            self.samples.append((sm, mx, pw, active))
+
+    def __enter__(self):
+        if self._open_nvml():
+            self.source = "nvml"
+            self._t = threading.Thread(target=self._loop, daemon=True)
+            self._t.start()
+        else:
+            self.source = "nvidia-smi"
+            self._open_smi()
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def __exit__(self, *exc):
-        if self.proc is not None:
+        if self._nv is not None:
+            self._stop.set()
+            if self._t is not None:
+                self._t.join(timeout=5)
+            try:
+                self._sample()
+                self._nv.nvmlShutdown()
+            except Exception:  # noqa: BLE001
+                pass
+        elif self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -178,25 +295,9 @@ class ClockSampler:
                 self._t.join(timeout=5)
 
     def summary(self) -> dict:
-        sm, mx, pw, reasons = [], [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
-                pw.append(float(parts[3]))
-            except ValueError:
-                continue
-            for name, flag in zip(names, parts[5:9]):
-                if flag.lower() == "active":
-                    reasons.add(name)
-        if not sm:
-            return dict(sm_mhz=None, sm_max_mhz=None, reasons=[], samples=0)
-        return dict(sm_mhz=statistics.median(sm), sm_max_mhz=max(mx), reasons=sorted(reasons),
-                    samples=len(sm), power_w=statistics.median(pw) if pw else None)
+        out = summarize_clock_samples(self.samples)
+        out["source"] = self.source
+        return out
 
 
 # ---------------------------------------------------------------------------- oracle leg
@@ -312,6 +413,23 @@ def run_reference(args, cfg) -> None:
     print(json.dumps(line), flush=True)
 
 
+DEFAULT_CONFIG = "cfg3_r0.9"
+
+
+def default_steps(cfg) -> int:
+    """Timed steps when none are given: about 10 s of steps at 70% of the step's roofline
+    (the expected masked count), at least 20 and at most 1000."""
+    peaks = load_peaks()
+    if cfg.mask == "bernoulli":
+        M = cfg.B * cfg.L * cfg.r
+    elif cfg.mask == "suffix":
+        M = cfg.B * cfg.n_suffix
+    else:
+        M = cfg.B * (cfg.block if cfg.block_only else cfg.L // 2)
+    est = roofline_s(cfg, int(M), peaks) / 0.7 + 20e-6
+    return int(min(1000, max(20, round(10.0 / est))))
+
+
 def rows_of_step(inp: dict) -> int:
     """Masked rows whose logits one step computes: all masked positions, or with
     current-block-only logits those inside each sequence's window."""
@@ -368,7 +486,7 @@ def run_vocab_sharded(args, cfg) -> None:
     if dl.get_status(stream) != 0 or int(step.count[0]) != count:
         raise RuntimeError("warm-up failed")
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+    with ClockSampler(dev) as clk:
         barrier()
         ev0.record(stream)
         for _ in range(args.steps):
@@ -407,15 +525,16 @@ def run_vocab_sharded(args, cfg) -> None:
         ms_step = t_ms / args.steps
         clk_summary = clk.summary()
         roof = gemm_roofline(shard_cfg, count, peaks, gemm_ms / max(1, gemm_launches) / 1e3,
-                             gemm_paired(args.gemm_variant, count),
-                             "vocabulary shard", "sw_power_cap" in clk_summary["reasons"])
+                             gemm_paired(args.gemm_variant, count), "vocabulary shard",
+                             region_s=t_ms / 1e3, sm_mhz=clk_summary["sm_mhz"])
         roof["traffic"] = None
         roof["shard"] = f"rows [{step.v0}, {step.v1}) of W on rank 0"
         line = dict(
             metric=METRIC, value=count * args.steps / (t_ms / 1e3), unit=UNIT, n_gpus=world,
             steps=args.steps, warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True,
             scaling="strong", vs_baseline=None, dtype="bf16", data="synthetic",
-            config=dict(workload_config(cfg, count), parallelism=f"vocabulary-parallel over {world} GPU(s)"),
+            config=workload_config(cfg, count),
+            run=dict(parallelism=f"vocabulary-parallel over {world} GPU(s)"),
             roofline=roof, gpu_launches=launches,
             e2e=dict(value=count * e2e_steps / (e2e_ms / 1e3), unit=UNIT,
                      h2d_bytes_per_step=cfg.B * cfg.L + 2 * cfg.d * count,
@@ -435,9 +554,11 @@ def run_vocab_sharded(args, cfg) -> None:
 def main() -> None:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: about 10 s of steps, 20 to 1000)")
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--config", default="cfg1")
+    ap.add_argument("--config", default=DEFAULT_CONFIG,
+                    help="workload (default: the largest single-GPU one, cfg3 at r_m = 0.9)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=120.0,
@@ -463,6 +584,8 @@ def main() -> None:
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     cfg = WL.CONFIGS[args.config]
+    if args.steps is None:
+        args.steps = default_steps(cfg)
 
     if args.impl == "reference":
         run_reference(args, cfg)
@@ -543,7 +666,7 @@ def main() -> None:
             step.run(H, M, W, win_lo, win_hi, stream, blk)
 
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+    with ClockSampler(dev) as clk:
         barrier()
         ev0.record(stream)
         if overlap:
@@ -560,11 +683,12 @@ def main() -> None:
     # (the dominant kernel's live duration) and its count of kernel launches; kept out of
     # the region above because an event between two kernels stops them from overlapping
     barrier()
-    dl.prof_begin()
-    for _ in range(args.steps):
-        step.run(H, M, W, win_lo, win_hi, stream, blk)
-    torch.cuda.synchronize(dev)
-    gemm_ms, gemm_launches, launches = dl.prof_end()
+    with ClockSampler(dev) as clk_gemm:
+        dl.prof_begin()
+        for _ in range(args.steps):
+            step.run(H, M, W, win_lo, win_hi, stream, blk)
+        torch.cuda.synchronize(dev)
+        gemm_ms, gemm_launches, launches = dl.prof_end()
     status = dl.get_status(stream)
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
@@ -574,6 +698,7 @@ def main() -> None:
     job_rows = int(round(D.sum_over_ranks([count], dev)[0]))
     full_base = (full_logits_baseline(H, M, W, cfg.k, win_lo, win_hi, blk, dev)
                  if world == 1 and not args.no_full_baseline else None)
+    torch.cuda.empty_cache()            # hand the baseline's logits back to the device
 
     # ---- end to end from pinned host memory ----
     # as many steps as the device-resident region, so that both settle into the same
@@ -590,7 +715,7 @@ def main() -> None:
                                     block_only=blk):
         pass
     torch.cuda.synchronize(dev)
-    with ClockSampler(dev.index if dev.index is not None else 0) as clk_e2e:
+    with ClockSampler(dev) as clk_e2e:
         barrier()
         t0 = time.perf_counter()
         n_out = 0
@@ -606,6 +731,7 @@ def main() -> None:
     if rank == 0:
         peaks = load_peaks()
         clk_summary = clk.summary()
+        clk_gemm_summary = clk_gemm.summary()
         a = algorithmic(cfg, count)
         ms_step = t_ms / args.steps
         rows_s = job_rows * args.steps / (t_ms / 1e3)
@@ -622,16 +748,17 @@ def main() -> None:
             metric=METRIC, value=rows_s, unit=UNIT, n_gpus=world, steps=args.steps,
             warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True, scaling="weak",
             vs_baseline=None, dtype="bf16", data="synthetic",
-            config=dict(workload_config(cfg, count), masked_rows_all_ranks=job_rows,
-                        policy=args.policy, threshold=args.threshold,
-                        launch=("CUDA graph replay" if args.graph else
-                                "one stream, steps in sequence" if args.serial else
-                                "two streams: staging of step i+1 overlaps step i")),
+            config=workload_config(cfg, count),
+            run=dict(masked_rows_all_ranks=job_rows, policy=args.policy,
+                     threshold=args.threshold,
+                     launch=("CUDA graph replay" if args.graph else
+                             "one stream, steps in sequence" if args.serial else
+                             "two streams: staging of step i+1 overlaps step i")),
             tflops=step_tflops, gbs=step_gbs,
             roofline_frac_step=roof / (ms_step / 1e3),
             roofline_ms=roof * 1e3,
             roofline=gemm_roofline(cfg, count, peaks, gemm_avg_s, paired, gemm_kernel_name,
-                                   "sw_power_cap" in clk_summary["reasons"]),
+                                   region_s=t_ms / 1e3, sm_mhz=clk_gemm_summary["sm_mhz"]),
             gpu_launches=launches,
             memory=dict(peak_step_bytes=int(step_peak),
                         full_logits_fp32_bytes=int(full_logits),
@@ -651,6 +778,7 @@ def main() -> None:
                           "copied back to pinned memory; wall clock, device synchronised at "
                           "both ends"),
             clocks=clk_summary,
+            clocks_gemm_pass=clk_gemm_summary,
         )
         if cpu is not None:
             line["cpu_baseline"] = cpu

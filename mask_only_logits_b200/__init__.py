@@ -658,7 +658,14 @@ class DecodeStep:
 
         Every argument but each batch's H and M is validated and turned into pointers once
         per call, so a step costs the host three library calls and four event operations:
-        short steps stay bound by the device, not by Python."""
+        short steps stay bound by the device, not by Python.
+
+        Readiness of the inputs: a list or tuple of batches must be written before the call,
+        on ``stream`` or on the current stream (the staging stream waits for both once).
+        Any other iterable is taken as produced lazily: each batch is waited for on the
+        current stream at the moment it is yielded, so a generator may write a batch on the
+        current stream just before yielding it.  When that stream is ``stream`` itself, each
+        staging then also waits for the previous step's GEMM (correct, without overlap)."""
         self._check_W(W)
         B, L, d, V = self.B, self.L, self.d, self.V
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
@@ -675,10 +682,18 @@ class DecodeStep:
         s_h, ps_h = _stream(s), _stream(ps)
         prepped = [torch.cuda.Event() for _ in range(2)]
         used = [torch.cuda.Event() for _ in range(2)]
+        cur = torch.cuda.current_stream(self.device)
         ps.wait_stream(s)                            # inputs written before the call are ready
+        if cur != s:
+            ps.wait_stream(cur)
+        lazy = not isinstance(batches, (list, tuple))
         last = 0
         for i, (H, M) in enumerate(batches):
             b = i & 1
+            if lazy:                                 # written on the current stream as yielded
+                ready = torch.cuda.Event()
+                ready.record(torch.cuda.current_stream(self.device))
+                ps.wait_event(ready)
             if i >= 2:
                 ps.wait_event(used[b])               # step i-2 no longer reads this workspace
             _check(lb.dllm_prepare_rows(*_step_inputs(H, M, B, L, d), B, L, d, V, *prep[b], ps_h),

@@ -28,18 +28,42 @@ def test_algorithmic_work_of_a_step():
                           + 4 * (2 * 32 + 1))
 
 
-def test_gemm_roofline_tensor_bound_and_power_cap():
+def test_gemm_roofline_peak_follows_the_region_length():
+    """Burst peak for a short timed region, sustained peak from LONG_REGION_S on, fixed by
+    the region's length (not by a throttle flag); both fractions always reported."""
     cfg = WL.CONFIGS["cfg1"]
     M = 1024
     t = 2.0 * M * cfg.V * cfg.d / 1000e12            # a launch running at 1000 TFLOP/s
-    r = bench.gemm_roofline(cfg, M, PEAKS, t, True, "lmhead_auto_kernel<0>")
+    r = bench.gemm_roofline(cfg, M, PEAKS, t, True, "lmhead_auto_kernel<0>", region_s=0.014)
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     assert r["achieved"] == pytest.approx(1000.0)
     assert r["peak"] == 1500.0 and r["frac"] == pytest.approx(1000 / 1500)
-    capped = bench.gemm_roofline(cfg, M, PEAKS, t, True, "lmhead_auto_kernel<0>", power_capped=True)
-    assert capped["peak"] == 1200.0 and capped["frac"] == pytest.approx(1000 / 1200)
-    assert capped["frac_of_burst"] == pytest.approx(1000 / 1500)
-    assert capped["frac_of_sustained"] == pytest.approx(1000 / 1200)
+    long_ = bench.gemm_roofline(cfg, M, PEAKS, t, True, "lmhead_auto_kernel<0>",
+                                region_s=bench.LONG_REGION_S, sm_mhz=1250.0)
+    assert long_["peak"] == 1200.0 and long_["frac"] == pytest.approx(1000 / 1200)
+    assert long_["frac_of_burst"] == pytest.approx(1000 / 1500)
+    assert long_["frac_of_sustained"] == pytest.approx(1000 / 1200)
+    assert long_["tflops_per_ghz"] == pytest.approx(800.0)
+    assert long_["gemm_mcycles"] == pytest.approx(t * 1250.0)
+
+
+def test_clock_summary():
+    s = bench.summarize_clock_samples([(1965.0, 1965.0, 400.0, set()),
+                                       (1400.0, 1965.0, 990.0, {"sw_power_cap"}),
+                                       (1300.0, 1965.0, 1000.0, {"sw_power_cap"})])
+    assert s["samples"] == 3 and s["sm_mhz"] == 1400.0 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"] and s["power_w"] == 990.0
+    assert bench.summarize_clock_samples([])["samples"] == 0
+
+
+def test_default_workload_is_the_largest_single_gpu_config():
+    cfg = WL.CONFIGS[bench.DEFAULT_CONFIG]
+    assert (cfg.B, cfg.L, cfg.d, cfg.V, cfg.r) == (1, 131072, 4096, 126464, 0.9)
+    assert max(c.B * c.L * c.r if c.mask == "bernoulli" else 0 for c in WL.CONFIGS.values()) \
+        == cfg.B * cfg.L * cfg.r
+    assert 50 <= bench.default_steps(cfg) <= 200                 # ~10 s of ~0.1 s steps
+    assert bench.default_steps(WL.CONFIGS["cfg1"]) == 1000
+    assert bench.default_steps(WL.CONFIGS["cfg0"]) == 1000
 
 
 def test_gemm_roofline_hbm_bound():
@@ -108,6 +132,8 @@ def test_reference_arm_json_line():
     assert d["value"] > 0 and d["steps"] == 3 and d["warmup"] == 3 and d["higher_is_better"]
     assert d["vs_baseline"] is None and d["data"] == "synthetic" and d["dtype"] == "f64"
     assert d["config"]["workload"].startswith("cfg0")
+    # the config names the workload only, exactly as the library's arm reports it
+    assert d["config"] == bench.workload_config(WL.CONFIGS["cfg0"], d["config"]["masked_rows"])
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1
     assert cb["host_cpus"] >= 1 and cb["blas"] and cb["sample"]

@@ -242,6 +242,7 @@ def test_overlapped_loop_call_order(fake, monkeypatch, policy, threshold):
     comp, prep = _FakeStream(log, "s"), _FakeStream(log, "ps")
     monkeypatch.setattr(torch.cuda, "Event", lambda *a, **k: _FakeEvent(log))
     monkeypatch.setattr(torch.cuda, "stream", lambda st: contextlib.nullcontext())
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda *a, **k: comp)
     st = dl.DecodeStep(B, L, d, V, k, device="cpu", policy=policy, threshold=threshold)
     b = bufs()
     n_steps = 5
@@ -277,6 +278,41 @@ def test_overlapped_loop_call_order(fake, monkeypatch, policy, threshold):
     assert prepped_ev[0] == prepped_ev[2] != prepped_ev[1] == prepped_ev[3]
 
 
+def test_overlapped_loop_waits_for_each_lazy_batch(fake, monkeypatch):
+    """Batches from a generator: the current stream when the call starts is waited for once,
+    and each batch's staging waits for an event recorded on the current stream at the moment
+    that batch was yielded (a list's batches are taken as ready at the call)."""
+    import contextlib
+    log = []
+    fake.calls = log
+    comp, prep, cur = _FakeStream(log, "s"), _FakeStream(log, "ps"), _FakeStream(log, "cur")
+    monkeypatch.setattr(torch.cuda, "Event", lambda *a, **k: _FakeEvent(log))
+    monkeypatch.setattr(torch.cuda, "stream", lambda st: contextlib.nullcontext())
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda *a, **k: cur)
+    st = dl.DecodeStep(B, L, d, V, k, device="cpu")
+    b = bufs()
+    n_steps = 4
+
+    def gen():
+        for i in range(n_steps):
+            log.append(("yield", i))
+            yield b["H"], b["M"]
+
+    st.run_overlapped(gen(), b["W"], stream=comp, prep_stream=prep)
+    assert log[:2] == [("wait_stream", "ps", "s"), ("wait_stream", "ps", "cur")]
+    for i in range(n_steps):
+        y = log.index(("yield", i))
+        p = [j for j, e in enumerate(log) if e == "dllm_prepare_rows"][i]
+        between = log[y:p]
+        rec = [e for e in between if isinstance(e, tuple) and e[0] == "record" and e[1] == "cur"]
+        assert len(rec) == 1, (i, between)
+        assert ("wait", "ps", rec[0][2]) in between, (i, between)
+    # a list: no per-batch event on the current stream
+    log.clear()
+    st.run_overlapped([(b["H"], b["M"])] * n_steps, b["W"], stream=comp, prep_stream=prep)
+    assert not [e for e in log if isinstance(e, tuple) and e[0] == "record" and e[1] == "cur"]
+
+
 def test_overlapped_loop_checks_each_batch(fake, monkeypatch):
     import contextlib
     log = []
@@ -285,6 +321,7 @@ def test_overlapped_loop_checks_each_batch(fake, monkeypatch):
     st = dl.DecodeStep(B, L, d, V, k, device="cpu")
     b = bufs()
     comp, prep = _FakeStream(log, "s"), _FakeStream(log, "ps")
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda *a, **k: comp)
     bad_M = torch.zeros(L, B, dtype=torch.uint8)                   # transposed
     with pytest.raises(ValueError, match="M: expected shape"):
         st.run_overlapped([(b["H"], b["M"]), (b["H"], bad_M)], b["W"], stream=comp, prep_stream=prep)

@@ -391,3 +391,52 @@ def test_overlapped_steps_match_single_steps(dl):
         c = int(out["count"][0])
         ref_rows, _, ref_c = O.mask_compact(host[-1][1].numpy())
         assert c == ref_c and np.array_equal(out["row_idx"][:c].cpu().numpy(), ref_rows)
+
+
+def test_overlapped_steps_from_a_generator(dl):
+    """Batches yielded by a generator that writes each one (on the current stream) just
+    before yielding it: the staging of every step waits for that write, so the selections
+    equal single steps on the same inputs.  Run with a producer stream as the current
+    stream, and with the compute stream itself as the current stream."""
+    cfg = WL.CONFIGS["cfg1"]
+    inp0 = WL.make_inputs(cfg, seed=31)
+    host = []
+    for sd in (32, 33, 34, 35):
+        g = torch.Generator().manual_seed(sd)
+        H = (torch.randn(cfg.B * cfg.L, cfg.d, generator=g) * cfg.h_std).to(torch.bfloat16)
+        M = WL.make_mask(cfg, g) if sd % 2 else torch.roll(WL.make_mask(cfg, g), 7 * sd, 1)
+        host.append((H.pin_memory(), M.pin_memory()))
+    W = inp0["W"].cuda()
+    step = dl.DecodeStep(cfg.B, cfg.L, cfg.d, cfg.V, cfg.k)
+    expected = []
+    for H, M in host:
+        step.run(H.cuda(), M.cuda(), W)
+        expected.append(step.sel_buf.clone())
+    torch.cuda.synchronize()
+    compute = torch.cuda.Stream()
+    for producer in (torch.cuda.Stream(), compute):
+        # two pairs of buffers, each overwritten every other batch: a staging that read too
+        # early would see an older batch (or a half-written one)
+        bufs = [(torch.zeros(cfg.B * cfg.L, cfg.d, dtype=torch.bfloat16, device="cuda"),
+                 torch.zeros(cfg.B, cfg.L, dtype=torch.uint8, device="cuda")) for _ in range(2)]
+        used = [None, None]
+
+        def batches():
+            for i, (H, M) in enumerate(host):
+                Hd, Md = bufs[i & 1]
+                if used[i & 1] is not None:
+                    torch.cuda.current_stream().wait_event(used[i & 1])
+                Hd.copy_(H, non_blocking=True)
+                Md.copy_(M, non_blocking=True)
+                ev = torch.cuda.Event()
+                used[i & 1] = ev
+                yield Hd, Md
+                ev.record(compute)               # the step reading this pair is enqueued
+
+        sel_out = [torch.empty_like(step.sel_buf) for _ in host]
+        with torch.cuda.stream(producer):
+            step.run_overlapped(batches(), W, stream=compute, sel_out=sel_out)
+        torch.cuda.synchronize()
+        assert dl.get_status() == 0
+        for got, exp in zip(sel_out, expected):
+            assert torch.equal(got, exp)
