@@ -581,6 +581,10 @@ def main() -> None:
                     help="threshold-based parallel unmasking on the policy's score (default: top-k)")
     ap.add_argument("--gemm-variant", type=int, default=0, choices=[0, 1, 2],
                     help="0 = library default, 1 = single-SM GEMM, 2 = paired-SM GEMM")
+    ap.add_argument("--arena", action="store_true",
+                    help="the step's workspace in a virtual-memory arena mapped for the step's "
+                         "own masked count (steps run one at a time); reports the mapped bytes "
+                         "against the count's need and the fixed worst-case workspace")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     cfg = WL.CONFIGS[args.config]
@@ -625,11 +629,32 @@ def main() -> None:
     base_mem = torch.cuda.memory_allocated(dev)
     dl.debug_set_gemm_variant(args.gemm_variant)
     step = dl.DecodeStep(cfg.B, cfg.L, cfg.d, cfg.V, cfg.k, device=dev, policy=args.policy,
-                         threshold=args.threshold)
+                         threshold=args.threshold, arena=args.arena)
     stream = torch.cuda.current_stream(dev)
+    arena_rec = None
+    if args.arena:
+        # the host knows the step's masked count (it built the mask): map just that much
+        torch.cuda.synchronize(dev)
+        free0, _ = torch.cuda.mem_get_info(dev)
+        need = step.size_for_rows(count)
+        torch.cuda.synchronize(dev)
+        free1, _ = torch.cuda.mem_get_info(dev)
+        arena_rec = dict(workspace_need_bytes=int(need), mapped_bytes=step.arena.mapped,
+                         device_bytes_taken=int(free0 - free1),
+                         reserved_va_bytes=step.arena.reserved, chunk_bytes=step.arena.chunk,
+                         fixed_workspace_bytes=dl.workspace_bytes(cfg.B, cfg.L, cfg.d, cfg.V),
+                         note="workspace in a dllm_arena mapped for this step's masked count "
+                              "(dllm_workspace_bytes_rows) against the fixed workspace sized "
+                              "for every position masked; device_bytes_taken = drop of "
+                              "cudaMemGetInfo's free bytes when the arena was mapped")
+
+    def run_step(H_, M_):
+        if args.arena:
+            return step.run(H_, M_, W, win_lo, win_hi, stream, blk, max_rows=count)
+        return step.run(H_, M_, W, win_lo, win_hi, stream, blk)
 
     for _ in range(args.warmup):
-        step.run(H, M, W, win_lo, win_hi, stream, blk)
+        run_step(H, M)
     torch.cuda.synchronize(dev)
     status = dl.get_status(stream)
     if status != 0:
@@ -650,7 +675,7 @@ def main() -> None:
             step.replay(stream)
         torch.cuda.synchronize(dev)
 
-    overlap = not (args.graph or args.serial)
+    overlap = not (args.graph or args.serial or args.arena)
     if overlap:
         # the staging of step i+1 (compaction of the mask, gather of the masked rows) runs
         # on a second stream while step i's GEMM and selection run on this one
@@ -663,7 +688,7 @@ def main() -> None:
         if args.graph:
             step.replay(stream)
         else:
-            step.run(H, M, W, win_lo, win_hi, stream, blk)
+            run_step(H, M)
 
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev) as clk:
@@ -686,7 +711,7 @@ def main() -> None:
     with ClockSampler(dev) as clk_gemm:
         dl.prof_begin()
         for _ in range(args.steps):
-            step.run(H, M, W, win_lo, win_hi, stream, blk)
+            run_step(H, M)
         torch.cuda.synchronize(dev)
         gemm_ms, gemm_launches, launches = dl.prof_end()
     status = dl.get_status(stream)
@@ -709,18 +734,26 @@ def main() -> None:
     for _ in range(3):
         step.run_host(H_host, M_host, W, win_lo, win_hi, stream, blk)
     barrier()
-    # the decode loop a serving process runs: each step's inputs copied in from pinned host
-    # memory (overlapping the previous step) and its selection copied back
-    for _ in step.run_host_pipeline([(H_host, M_host)] * 3, W, win_lo, win_hi, stream,
-                                    block_only=blk):
+
+    def host_steps(n):
+        # the decode loop a serving process runs: each step's inputs copied in from pinned
+        # host memory (overlapping the previous step) and its selection copied back; in
+        # arena mode one step at a time (the mapping follows each step's mask)
+        if args.arena:
+            for _ in range(n):
+                yield step.run_host(H_host, M_host, W, win_lo, win_hi, stream, blk)
+        else:
+            yield from step.run_host_pipeline([(H_host, M_host)] * n, W, win_lo, win_hi, stream,
+                                              block_only=blk)
+
+    for _ in host_steps(3):
         pass
     torch.cuda.synchronize(dev)
     with ClockSampler(dev) as clk_e2e:
         barrier()
         t0 = time.perf_counter()
         n_out = 0
-        for _ in step.run_host_pipeline([(H_host, M_host)] * e2e_steps, W, win_lo, win_hi,
-                                        stream, block_only=blk):
+        for _ in host_steps(e2e_steps):
             n_out += 1
         torch.cuda.synchronize(dev)
         e2e_s = time.perf_counter() - t0
@@ -752,7 +785,8 @@ def main() -> None:
             run=dict(masked_rows_all_ranks=job_rows, policy=args.policy,
                      threshold=args.threshold,
                      launch=("CUDA graph replay" if args.graph else
-                             "one stream, steps in sequence" if args.serial else
+                             "one stream, steps in sequence, workspace in an arena" if args.arena
+                             else "one stream, steps in sequence" if args.serial else
                              "two streams: staging of step i+1 overlaps step i")),
             tflops=step_tflops, gbs=step_gbs,
             roofline_frac_step=roof / (ms_step / 1e3),
@@ -760,14 +794,15 @@ def main() -> None:
             roofline=gemm_roofline(cfg, count, peaks, gemm_avg_s, paired, gemm_kernel_name,
                                    region_s=t_ms / 1e3, sm_mhz=clk_gemm_summary["sm_mhz"]),
             gpu_launches=launches,
-            memory=dict(peak_step_bytes=int(step_peak),
+            memory=dict(peak_step_bytes=int(step_peak) if not args.arena else None,
                         full_logits_fp32_bytes=int(full_logits),
                         workspaces=1 if not overlap else 2,
                         note="peak = torch allocations of the step (outputs + workspace; two "
                              "workspaces when staging overlaps the previous step) over the "
                              "resident inputs; full_logits_fp32_bytes = B*L*V fp32 logits"),
             e2e=dict(value=job_rows * e2e_steps / (e2e_ms / 1e3), unit=UNIT,
-                     h2d_bytes_per_step=step.h2d_bytes_zero_copy(count),
+                     h2d_bytes_per_step=(step.h2d_bytes() if args.arena else
+                                         step.h2d_bytes_zero_copy(count)),
                      d2h_bytes_per_step=step.d2h_bytes(),
                      ms_per_step=e2e_ms / e2e_steps, steps=e2e_steps,
                      clocks=clk_e2e.summary(),
@@ -784,6 +819,8 @@ def main() -> None:
             line["cpu_baseline"] = cpu
         if full_base is not None:
             line["full_logits_baseline"] = full_base
+        if arena_rec is not None:
+            line["memory"]["arena"] = arena_rec
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()

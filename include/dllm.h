@@ -29,8 +29,10 @@
  *
  * Conventions for every call:
  *   - Pointers marked "device" must point to memory of the current CUDA device; the caller
- *     owns every buffer.  The library never allocates device memory: scratch space is the
- *     caller's workspace, sized by dllm_workspace_bytes().
+ *     owns every buffer.  The library never allocates device memory on its own: scratch
+ *     space is the caller's workspace, sized by dllm_workspace_bytes() (or, for a known
+ *     masked count, dllm_workspace_bytes_rows()); a dllm_arena maps device memory only
+ *     when the caller asks it to.
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  All
  *     work is enqueued asynchronously on it; no call synchronises the host except
  *     dllm_get_status() and dllm_prof_end().  Kernels are launched with programmatic
@@ -66,13 +68,14 @@ typedef int32_t dllm_status;
 #define DLLM_ERR_NULL       -1   /* a required pointer is NULL                              */
 #define DLLM_ERR_ALIGN      -2   /* a device pointer is not 16-byte aligned                 */
 #define DLLM_ERR_SHAPE      -3   /* B, L, d, V or k out of range (see each call)            */
-#define DLLM_ERR_WORKSPACE  -4   /* workspace smaller than dllm_workspace_bytes()           */
+#define DLLM_ERR_WORKSPACE  -4   /* workspace too small (see dllm_workspace_bytes_rows)      */
 #define DLLM_ERR_CUDA       -5   /* a CUDA runtime/driver call failed                       */
 #define DLLM_ERR_TIMEOUT    -6   /* a device-side wait exceeded its limit (kernel returned) */
 #define DLLM_ERR_DEVICE     -7   /* the current device is not an sm_100 GPU                 */
 #define DLLM_ERR_BOUNDS     -8   /* a device-side bound check failed (access skipped)       */
 #define DLLM_ERR_SCRATCH    -9   /* B*L exceeds the fixed scratch of dllm_mask_compact_noalloc */
 #define DLLM_ERR_MEMORY     -10  /* an input is neither device memory nor page-locked host memory */
+#define DLLM_ERR_CAPACITY   -11  /* more masked rows than the workspace was sized for (device) */
 
 /* Limits. */
 #define DLLM_MAX_K          1024 /* largest k accepted by dllm_select_unmask                */
@@ -92,6 +95,75 @@ const char* dllm_status_string(dllm_status s);
  * Needs no GPU.
  */
 size_t dllm_workspace_bytes(int32_t B, int32_t L, int32_t d, int32_t V);
+
+/*
+ * Workspace sized for steps with at most max_rows masked rows (a step's gathered rows and
+ * partials grow with its masked count; the Mosaic page, Fig. 3, shows how that count sets
+ * the step's memory peak as the mask ratio changes).  A caller that knows its masked count
+ * -- a decoding loop does: it built the mask -- can hold a workspace of this size instead of
+ * the upper bound, e.g. mapped on demand in a dllm_arena.  max_rows >= B*L gives
+ * dllm_workspace_bytes().  Returns 0 for invalid shapes or max_rows < 1.  Needs no GPU.
+ *
+ * Every call that takes a workspace (ws, ws_bytes) accepts one smaller than
+ * dllm_workspace_bytes(): its masked-row capacity is then the largest max_rows whose size
+ * fits in ws_bytes (dllm_workspace_rows).  DLLM_ERR_WORKSPACE is returned only when not even
+ * one row fits.  A step whose mask has more masked rows than the capacity computes the
+ * first `capacity` rows, leaves the rest of tok/conf/lse untouched, touches no workspace
+ * byte past ws_bytes, and records DLLM_ERR_CAPACITY for dllm_get_status(): its selection is
+ * then not valid.
+ */
+size_t dllm_workspace_bytes_rows(int32_t B, int32_t L, int32_t d, int32_t V, int64_t max_rows);
+
+/* Masked-row capacity of a workspace of ws_bytes for these shapes (B*L when it holds the
+ * upper bound; 0 when too small for one row or for invalid shapes).  Needs no GPU. */
+int64_t dllm_workspace_rows(int32_t B, int32_t L, int32_t d, int32_t V, size_t ws_bytes);
+
+/*
+ * dllm_arena - device memory behind one fixed virtual address range, backed by physical
+ * memory on demand: the "global memory manager with virtual memory mapping" of the Mosaic
+ * page (TL;DR and Abstract; Fig. 4 compares the memory it reserves with the theoretical
+ * peak).  The whole range is reserved once (cuMemAddressReserve) and never moves, so its
+ * address can be kept in a workspace argument, a tensor map or a CUDA graph; only the
+ * prefix [0, mapped) is backed by physical memory (cuMemCreate + cuMemMap, in chunks).
+ * Growing or shrinking the mapped prefix to what the next step needs
+ * (dllm_workspace_bytes_rows of its masked count) keeps the memory held close to the
+ * step's own requirement instead of the worst case over all masks.
+ *
+ * The arena is the one object of this library that allocates device memory, and only when
+ * the caller asks it to (dllm_arena_create, dllm_arena_map).  It is not thread-safe: one
+ * thread at a time per arena.
+ *
+ * dllm_arena_create: reserve `reserve_bytes` (rounded up to the chunk size) of virtual
+ * address space on the current device, with nothing mapped.  chunk_bytes = the unit in
+ * which physical memory is created, mapped and released (rounded up to the device's
+ * allocation granularity; 0 = that granularity, 2 MiB on B200).  *out receives the arena.
+ * Errors: DLLM_ERR_NULL (out), DLLM_ERR_SHAPE (reserve_bytes == 0), DLLM_ERR_CUDA (the
+ * reservation or a driver query failed), DLLM_ERR_DEVICE.
+ *
+ * dllm_arena_map: make [0, bytes) usable, in whole chunks: chunks are created and mapped
+ * (read-write for the current device) up to round_up(bytes, chunk); chunks wholly past that
+ * point are unmapped and released.  Before it releases anything it synchronises the device
+ * (cudaDeviceSynchronize), so no kernel still running can touch memory being released;
+ * growing does not synchronise.  On a failed grow every chunk created by this call is
+ * released again and the arena keeps its previous mapping.  Errors: DLLM_ERR_NULL,
+ * DLLM_ERR_SHAPE (bytes > the reserved size), DLLM_ERR_CUDA (out of device memory or a
+ * driver call failed).
+ *
+ * dllm_arena_ptr: base device address of the range (16-byte aligned; fixed for the arena's
+ * life).  dllm_arena_reserved / dllm_arena_mapped / dllm_arena_chunk: the reserved size,
+ * the bytes currently backed by physical memory, the chunk size.
+ *
+ * dllm_arena_destroy: synchronise the device, unmap and release every chunk, free the
+ * reservation and the arena object.  NULL is accepted (no-op).
+ */
+typedef struct dllm_arena dllm_arena;
+dllm_status dllm_arena_create(size_t reserve_bytes, size_t chunk_bytes, dllm_arena** out);
+dllm_status dllm_arena_map(dllm_arena* arena, size_t bytes);
+void* dllm_arena_ptr(const dllm_arena* arena);
+size_t dllm_arena_reserved(const dllm_arena* arena);
+size_t dllm_arena_mapped(const dllm_arena* arena);
+size_t dllm_arena_chunk(const dllm_arena* arena);
+dllm_status dllm_arena_destroy(dllm_arena* arena);
 
 /*
  * dllm_mask_compact - prefix-sum compaction of the mask (Mosaic page, Abstract: logits are
@@ -384,8 +456,9 @@ dllm_status dllm_decode_block_step(const uint16_t* H, const uint8_t* M, const ui
 
 /*
  * dllm_get_status - synchronise `stream`, then return (and clear) the device-side status
- * word of the current device: DLLM_OK, DLLM_ERR_TIMEOUT or DLLM_ERR_BOUNDS; DLLM_ERR_CUDA
- * if the synchronisation itself failed.
+ * word of the current device: DLLM_OK, DLLM_ERR_TIMEOUT, DLLM_ERR_BOUNDS or
+ * DLLM_ERR_CAPACITY (in that order of precedence when several were recorded);
+ * DLLM_ERR_CUDA if the synchronisation itself failed.
  */
 dllm_status dllm_get_status(void* stream);
 

@@ -21,7 +21,8 @@ import torch
 from . import _abi
 
 __all__ = [
-    "DllmError", "lib", "version", "workspace_bytes", "mask_compact", "mask_compact_noalloc",
+    "DllmError", "lib", "version", "workspace_bytes", "workspace_bytes_rows", "workspace_rows",
+    "Arena", "mask_compact", "mask_compact_noalloc",
     "masked_logits", "masked_logits_ex", "select_unmask_ex", "STAT_ENTROPY", "STAT_MARGIN",
     "masked_partials", "lse_merge", "prepare_rows", "masked_logits_prepared",
     "select_unmask", "decode_step", "get_status", "debug_lmhead_logits", "debug_lse_merge",
@@ -36,7 +37,7 @@ STAT_MARGIN = 2
 STATUS = {0: "DLLM_OK", -1: "DLLM_ERR_NULL", -2: "DLLM_ERR_ALIGN", -3: "DLLM_ERR_SHAPE",
           -4: "DLLM_ERR_WORKSPACE", -5: "DLLM_ERR_CUDA", -6: "DLLM_ERR_TIMEOUT",
           -7: "DLLM_ERR_DEVICE", -8: "DLLM_ERR_BOUNDS", -9: "DLLM_ERR_SCRATCH",
-          -10: "DLLM_ERR_MEMORY"}
+          -10: "DLLM_ERR_MEMORY", -11: "DLLM_ERR_CAPACITY"}
 
 
 class DllmError(RuntimeError):
@@ -93,6 +94,89 @@ def version() -> int:
 
 def workspace_bytes(B: int, L: int, d: int, V: int) -> int:
     return int(lib().dllm_workspace_bytes(B, L, d, V))
+
+
+def workspace_bytes_rows(B: int, L: int, d: int, V: int, max_rows: int) -> int:
+    """Workspace bytes for steps with at most max_rows masked rows (0 if invalid)."""
+    return int(lib().dllm_workspace_bytes_rows(B, L, d, V, max_rows))
+
+
+def workspace_rows(B: int, L: int, d: int, V: int, ws_bytes: int) -> int:
+    """Masked-row capacity of a workspace of ws_bytes (B*L for the full size, 0 if too small)."""
+    return int(lib().dllm_workspace_rows(B, L, d, V, ws_bytes))
+
+
+class _DeviceBytes:
+    """A device byte range exposed through __cuda_array_interface__, so that torch can view
+    it as a uint8 tensor without copying or allocating."""
+
+    def __init__(self, ptr: int, nbytes: int):
+        self.__cuda_array_interface__ = dict(shape=(nbytes,), typestr="|u1", data=(ptr, False),
+                                             version=3, strides=None)
+
+
+class Arena:
+    """Device memory behind one fixed virtual address range, backed on demand (the C ABI's
+    dllm_arena: the Mosaic page's memory manager with virtual memory mapping).
+
+    ``map(nbytes)`` backs [0, nbytes) (whole chunks) with physical memory and releases the
+    chunks past it; the address never moves.  ``tensor()`` is a uint8 view of the mapped
+    prefix, usable as a step's workspace.  Shrinking synchronises the device first."""
+
+    def __init__(self, reserve_bytes: int, chunk_bytes: int = 0, device=None):
+        if device is not None:
+            torch.cuda.set_device(device)
+        self.device = torch.device("cuda", torch.cuda.current_device())
+        h = ctypes.c_void_p()
+        _check(lib().dllm_arena_create(reserve_bytes, chunk_bytes, ctypes.byref(h)),
+               "dllm_arena_create")
+        self._h = h
+        self._view = None
+
+    @property
+    def ptr(self) -> int:
+        return int(lib().dllm_arena_ptr(self._h) or 0)
+
+    @property
+    def reserved(self) -> int:
+        return int(lib().dllm_arena_reserved(self._h))
+
+    @property
+    def mapped(self) -> int:
+        return int(lib().dllm_arena_mapped(self._h))
+
+    @property
+    def chunk(self) -> int:
+        return int(lib().dllm_arena_chunk(self._h))
+
+    def map(self, nbytes: int) -> int:
+        """Back [0, nbytes) with physical memory (whole chunks); returns the mapped size."""
+        if self._h is None:
+            raise RuntimeError("arena closed")
+        self._view = None
+        _check(lib().dllm_arena_map(self._h, nbytes), "dllm_arena_map")
+        return self.mapped
+
+    def tensor(self) -> torch.Tensor:
+        """uint8 view of the mapped prefix (valid until the next map() or close())."""
+        if self._view is None:
+            n = self.mapped
+            if n == 0:
+                raise RuntimeError("nothing is mapped")
+            self._view = torch.as_tensor(_DeviceBytes(self.ptr, n), device=self.device)
+        return self._view
+
+    def close(self) -> None:
+        if self._h is not None:
+            self._view = None
+            _check(lib().dllm_arena_destroy(self._h), "dllm_arena_destroy")
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:  # noqa: BLE001 - interpreter shutdown
+            pass
 
 
 def mask_compact(M, row_idx, seq_off, count, ws, stream=None, win_lo=None, win_hi=None) -> None:
@@ -387,7 +471,8 @@ class DecodeStep:
     """
 
     def __init__(self, B: int, L: int, d: int, V: int, k: int, device="cuda",
-                 policy: str = "confidence", threshold: float | None = None, min_sel: int = 1):
+                 policy: str = "confidence", threshold: float | None = None, min_sel: int = 1,
+                 arena: bool = False, arena_chunk: int = 0):
         if k < 1 or k > MAX_K:
             raise ValueError(f"k must be in [1, {MAX_K}]")
         if policy not in POLICIES:
@@ -419,8 +504,30 @@ class DecodeStep:
         nbytes = workspace_bytes(B, L, d, V)
         if nbytes == 0:
             raise ValueError("invalid shapes (d must be a positive multiple of 64)")
-        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        # arena=True: the workspace lives in an Arena whose mapping follows each step's
+        # masked count (``run(..., max_rows=...)``) instead of the worst case over all masks
+        self.arena = Arena(nbytes, arena_chunk, self.device) if arena else None
+        self.ws = None if arena else torch.empty(nbytes, dtype=torch.uint8, device=self.device)
         self._host = None
+
+    def size_for_rows(self, max_rows: int) -> int:
+        """Arena mode: map the workspace a step with at most max_rows masked rows needs
+        (growing or shrinking the arena's backing); returns the bytes that step needs."""
+        if self.arena is None:
+            raise RuntimeError("size_for_rows needs DecodeStep(..., arena=True)")
+        need = workspace_bytes_rows(self.B, self.L, self.d, self.V, max(1, int(max_rows)))
+        if self.ws is None or self.arena.mapped != -(-need // self.arena.chunk) * self.arena.chunk:
+            self.arena.map(need)
+        self.ws = self.arena.tensor()
+        return need
+
+    def _rows_of(self, M, win_lo, win_hi, block_only) -> int:
+        """Masked rows a step on M computes (a device mask is read back: a synchronisation)."""
+        m = M != 0
+        if block_only:
+            pos = torch.arange(self.L, device=M.device)[None, :]
+            m = m & (pos >= win_lo.to(M.device)[:, None]) & (pos < win_hi.to(M.device)[:, None])
+        return int(m.sum())
 
     def _sel_views(self, buf):
         """idx [B, k], n_sel [B], tok_sel [B, k] (int32) and conf_sel [B, k] (float32) views
@@ -473,10 +580,16 @@ class DecodeStep:
             out["margin"] = self.margin
         return out
 
-    def run(self, H, M, W, win_lo=None, win_hi=None, stream=None, block_only=False) -> dict:
+    def run(self, H, M, W, win_lo=None, win_hi=None, stream=None, block_only=False,
+            max_rows: int | None = None) -> dict:
         """One step on device tensors.  block_only=True (windows required): logits for the
-        masked rows inside the windows only; tok/conf/lse/row_idx then cover those rows."""
+        masked rows inside the windows only; tok/conf/lse/row_idx then cover those rows.
+        Arena mode: the workspace is mapped for max_rows masked rows first (a decoding loop
+        knows its masked count; if max_rows is None it is counted from M)."""
         self._check_W(W)
+        if self.arena is not None:
+            self.size_for_rows(self._rows_of(M, win_lo, win_hi, block_only)
+                               if max_rows is None else max_rows)
         if self._plain():
             decode_step(H, M, W, self.k, self.tok, self.conf, self.lse, self.row_idx,
                         self.seq_off, self.count, self.idx, self.n_sel, self.ws, win_lo, win_hi,
@@ -495,6 +608,10 @@ class DecodeStep:
         on whatever those tensors hold at replay time, for one launch of CPU work; the
         outputs are this object's buffers as after ``run``.  Tensors must keep their
         addresses while the graph is used."""
+        if self.arena is not None:
+            # a graph would keep the workspace size of capture time while the arena's mapping
+            # follows later masks
+            raise RuntimeError("capture() needs a fixed workspace: use arena=False")
         side = torch.cuda.Stream(self.device)
         side.wait_stream(torch.cuda.current_stream(self.device))
         with torch.cuda.stream(side):
@@ -536,10 +653,12 @@ class DecodeStep:
         """
         hb = self._host_buffers()
         s = stream if stream is not None else torch.cuda.current_stream()
+        rows = (self._rows_of(M_host, win_lo, win_hi, block_only)   # counted on the host
+                if self.arena is not None else None)
         with torch.cuda.stream(s):
             hb["H"].copy_(H_host, non_blocking=True)
             hb["M"].copy_(M_host, non_blocking=True)
-            self.run(hb["H"], hb["M"], W, win_lo, win_hi, s, block_only)
+            self.run(hb["H"], hb["M"], W, win_lo, win_hi, s, block_only, max_rows=rows)
             hb["sel"].copy_(self.sel_buf, non_blocking=True)
         s.synchronize()
         return dict(zip(("idx", "n_sel", "tok_sel", "conf_sel"), self._sel_views(hb["sel"])))
@@ -547,6 +666,9 @@ class DecodeStep:
     def _double(self) -> dict:
         """Two sets of (workspace, row_idx, seq_off, count): this object's own and a second
         one, so that staging of one step can run while the previous step computes."""
+        if self.arena is not None:
+            raise RuntimeError("the overlapped loops keep two fixed workspaces; with arena=True "
+                               "run steps one at a time (run, run_host)")
         if getattr(self, "_dbl", None) is None:
             i32 = dict(dtype=torch.int32, device=self.device)
             self._dbl = dict(ws=[self.ws, torch.empty_like(self.ws)],

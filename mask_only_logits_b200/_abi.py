@@ -17,6 +17,15 @@ PROTOTYPES = {
     "dllm_version": (_i32, []),
     "dllm_status_string": (ctypes.c_char_p, [_st]),
     "dllm_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32]),
+    "dllm_workspace_bytes_rows": (_sz, [_i32, _i32, _i32, _i32, ctypes.c_int64]),
+    "dllm_workspace_rows": (ctypes.c_int64, [_i32, _i32, _i32, _i32, _sz]),
+    "dllm_arena_create": (_st, [_sz, _sz, ctypes.POINTER(_p)]),
+    "dllm_arena_map": (_st, [_p, _sz]),
+    "dllm_arena_ptr": (_p, [_p]),
+    "dllm_arena_reserved": (_sz, [_p]),
+    "dllm_arena_mapped": (_sz, [_p]),
+    "dllm_arena_chunk": (_sz, [_p]),
+    "dllm_arena_destroy": (_st, [_p]),
     "dllm_mask_compact": (_st, [_p, _i32, _i32, _p, _p, _p, _p, _sz, _p]),
     "dllm_mask_compact_window": (_st, [_p, _i32, _i32, _p, _p, _p, _p, _p, _p, _sz, _p]),
     "dllm_mask_compact_noalloc": (_st, [_p, _i32, _i32, _p, _p, _p, _p]),

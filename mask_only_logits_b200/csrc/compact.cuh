@@ -7,11 +7,14 @@
 // Optional per-sequence windows [lo_b, hi_b) restrict the compaction to the masked positions
 // of each sequence's current block.
 //
-// Two launches, both over tiles of kCompactTile positions (one 16-byte vector per thread):
+// Launches over tiles of kCompactTile positions (one 16-byte vector per thread):
 //   compact_count_kernel    tile t -> number of nonzero mask bytes in the tile
-//   compact_scatter_kernel  tile t -> its offset (sum of earlier tiles' counts, reduced by
-//                           the whole CTA), a block-wide exclusive scan of per-thread
-//                           counts, then the ascending positions, seq_off and count.
+//   compact_scan_kernel     (more than kCompactDirectTiles tiles only) one CTA turns the
+//                           counts into exclusive offsets, in place
+//   compact_scatter_kernel  tile t -> its offset (read, or for at most kCompactDirectTiles
+//                           tiles the sum of earlier tiles' counts reduced by the whole
+//                           CTA), a block-wide exclusive scan of per-thread counts, then the
+//                           ascending positions, seq_off and count.
 #pragma once
 #include "ptx.cuh"
 
@@ -20,6 +23,11 @@ namespace dllm {
 constexpr int kCompactThreads = 512;
 constexpr int kCompactVec = 16;                                   // bytes per thread
 constexpr int kCompactTile = kCompactThreads * kCompactVec;       // 8192 positions
+// Up to this many tiles each scatter CTA sums the earlier tiles' counts itself (at most 63
+// loads); beyond it a scan launch computes every tile's offset once, so the total work stays
+// linear in the number of tiles.
+constexpr int kCompactDirectTiles = 64;
+constexpr int kScanThreads = 1024;
 
 // 0x80 in every byte of w that is nonzero, 0 elsewhere (no carries cross bytes because
 // (b & 0x7F) + 0x7F <= 0xFE).
@@ -104,21 +112,65 @@ compact_count_kernel(const uint8_t* __restrict__ M, long long n, int L, const in
   if (threadIdx.x == 0) tile_count[blockIdx.x] = total;
 }
 
+// Exclusive prefix sum of the n tile counts, in place (one CTA): thread i sums a contiguous
+// chunk, the chunk sums are scanned across the CTA, then each thread writes its chunk's
+// offsets.
+__global__ void __launch_bounds__(kScanThreads)
+compact_scan_kernel(int* __restrict__ tile_count, int n) {
+  __shared__ int warp_tot[kScanThreads / 32];
+  pdl_wait();
+  pdl_launch_dependents();
+  const int per = (n + kScanThreads - 1) / kScanThreads;
+  const int i0 = threadIdx.x * per;
+  const int i1 = i0 + per < n ? i0 + per : n;
+  int sum = 0;
+  for (int i = i0; i < i1; ++i) sum += tile_count[i];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = sum;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int w = warp_tot[lane];               // kScanThreads / 32 == 32 warps
+    int wi = w;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += y;
+    }
+    warp_tot[lane] = wi - w;
+  }
+  __syncthreads();
+  int run = warp_tot[warp] + incl - sum;        // exclusive offset of this thread's chunk
+  for (int i = i0; i < i1; ++i) {
+    const int c = tile_count[i];
+    tile_count[i] = run;
+    run += c;
+  }
+}
+
 __global__ void __launch_bounds__(kCompactThreads)
 compact_scatter_kernel(const uint8_t* __restrict__ M, int B, int L, const int* __restrict__ win_lo,
                        const int* __restrict__ win_hi, const int* __restrict__ tile_count,
-                       int* __restrict__ row_idx, int* __restrict__ seq_off, int* __restrict__ count,
-                       int* __restrict__ status) {
+                       bool offsets, int* __restrict__ row_idx, int* __restrict__ seq_off,
+                       int* __restrict__ count, int* __restrict__ status) {
   __shared__ int red[33];
   __shared__ int warp_excl[kCompactThreads / 32];
   pdl_wait();
   pdl_launch_dependents();
   const long long n = static_cast<long long>(B) * L;
   const int t = blockIdx.x;
-  // offset of this tile = sum of the counts of tiles 0..t-1
-  int part = 0;
-  for (int i = threadIdx.x; i < t; i += kCompactThreads) part += tile_count[i];
-  const int tile_base = block_sum(part, red);
+  // offset of this tile = sum of the counts of tiles 0..t-1 (already scanned when `offsets`)
+  int tile_base;
+  if (offsets) {
+    tile_base = tile_count[t];
+  } else {
+    int part = 0;
+    for (int i = threadIdx.x; i < t; i += kCompactThreads) part += tile_count[i];
+    tile_base = block_sum(part, red);
+  }
 
   const long long p0 = (static_cast<long long>(t) * kCompactThreads + threadIdx.x) * kCompactVec;
   const uint32_t bits = window_filter(load_mask16(M, p0, n), p0, L, win_lo, win_hi);
@@ -171,13 +223,16 @@ compact_scatter_kernel(const uint8_t* __restrict__ M, int B, int L, const int* _
 }
 
 // Copy the masked rows H[row_idx[r]] (d bf16 each) into the dense matrix Hm[r] for
-// r < count (one warp per row, 16-byte vectors), and zero n_zero ints at `zero`.
+// r < count (one warp per row, 16-byte vectors), and zero n_zero ints at `zero`.  Hm holds
+// n_cap rows: a larger count records kStatusCapacity and only the first n_cap rows are
+// copied.
 constexpr int kGatherThreads = 256;
 
 __global__ void __launch_bounds__(kGatherThreads)
 gather_rows_kernel(const uint16_t* __restrict__ H, const int* __restrict__ row_idx,
-                   const int* __restrict__ count, long long n_pos, int d, uint16_t* __restrict__ Hm,
-                   int* __restrict__ zero, int n_zero, int* __restrict__ status) {
+                   const int* __restrict__ count, long long n_pos, long long n_cap, int d,
+                   uint16_t* __restrict__ Hm, int* __restrict__ zero, int n_zero,
+                   int* __restrict__ status) {
   pdl_wait();
   pdl_launch_dependents();
   // also clear the GEMM's per-m-tile unit counters for this step
@@ -187,6 +242,9 @@ gather_rows_kernel(const uint16_t* __restrict__ H, const int* __restrict__ row_i
   if (n < 0 || n > n_pos) {                          // cannot happen: bad compaction
     if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(status, kStatusBounds);
     n = 0;
+  } else if (n > n_cap) {                            // workspace sized for fewer rows
+    if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(status, kStatusCapacity);
+    n = static_cast<int>(n_cap);
   }
   const int lane = threadIdx.x & 31;
   const int warps = gridDim.x * (kGatherThreads / 32);

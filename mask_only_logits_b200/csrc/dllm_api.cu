@@ -20,6 +20,7 @@
 #include "lmhead.cuh"
 #include "merge.cuh"
 #include "select.cuh"
+#include "arena.cuh"
 
 namespace dllm {
 
@@ -33,7 +34,7 @@ struct NvtxRange {
   NvtxRange& operator=(const NvtxRange&) = delete;
 };
 
-// Device-side error bits (kStatusTimeout, kStatusBounds); one word per device.
+// Device-side error bits (kStatusTimeout, kStatusBounds, kStatusCapacity); one word per device.
 __device__ int g_status;
 
 namespace {
@@ -170,23 +171,27 @@ dllm_status device_state(DeviceState** out) {
   return DLLM_OK;
 }
 
-// Workspace layout:
+// Workspace layout for at most `rows` masked rows (rows = B*L: any mask):
 // [tile counts | unit counters | gathered rows Hm | part_m | part_s | part_a | part_t | part_m2].
 struct WsLayout {
   size_t tiles_off, ctr_off, hm_off, pm_off, ps_off, pa_off, pt_off, pm2_off, total;
   long long part_cap;
+  long long rows;          // masked-row capacity: rows of Hm, and the GEMM's row bound
   int n_ctr;
 };
 
-WsLayout ws_layout(int B, int L, int d, int V) {
+WsLayout ws_layout(int B, int L, int d, int V, long long rows) {
   WsLayout w{};
   const long long n = static_cast<long long>(B) * L;
   const long long ntiles = (n + kCompactTile - 1) / kCompactTile;
-  // partial entries: worst case over the masked count (all positions masked), the largest
-  // number of work holders and either GEMM variant; fewer masked rows never need more.
-  const lm::Plan w1 = lm::Plan::make(static_cast<int>(n), V, lm::kMaxCtas, lm::Cfg<1>::kGroupM,
+  if (rows > n) rows = n;
+  if (rows < 1) rows = 1;
+  w.rows = rows;
+  // partial entries: worst case over the masked count (up to `rows`), the largest number of
+  // work holders and either GEMM variant; fewer masked rows never need more.
+  const lm::Plan w1 = lm::Plan::make(static_cast<int>(rows), V, lm::kMaxCtas, lm::Cfg<1>::kGroupM,
                                      lm::Cfg<1>::BM);
-  const lm::Plan w2 = lm::Plan::make(static_cast<int>(n), V, lm::kMaxCtas / 2, lm::Cfg<2>::kGroupM,
+  const lm::Plan w2 = lm::Plan::make(static_cast<int>(rows), V, lm::kMaxCtas / 2, lm::Cfg<2>::kGroupM,
                                      lm::Cfg<2>::BM);
   const long long cap1 = w1.ngroups * static_cast<long long>(lm::kMaxCtas) * lm::Cfg<1>::BM;
   const long long cap2 = w2.ngroups * static_cast<long long>(lm::kMaxCtas / 2) * lm::Cfg<2>::BM;
@@ -201,12 +206,12 @@ WsLayout ws_layout(int B, int L, int d, int V) {
   if (r2 > cap) cap = r2;
   if (cap < 1) cap = 1;
   w.part_cap = cap;
-  // one counter per (m-tile, CTA of the pair): ceil(n / 128) + 2 covers both variants
-  w.n_ctr = static_cast<int>((n + 127) / 128 + 2);
+  // one counter per (m-tile, CTA of the pair): ceil(rows / 128) + 2 covers both variants
+  w.n_ctr = static_cast<int>((rows + 127) / 128 + 2);
   size_t off = 0;
   w.tiles_off = off; off = round_up(off + sizeof(int) * ntiles, 256);
   w.ctr_off = off;   off = round_up(off + sizeof(int) * static_cast<size_t>(w.n_ctr), 256);
-  w.hm_off = off;    off = round_up(off + static_cast<size_t>(n) * d * 2, 256);
+  w.hm_off = off;    off = round_up(off + static_cast<size_t>(rows) * d * 2, 256);
   w.pm_off = off;    off = round_up(off + sizeof(float) * cap, 256);
   w.ps_off = off;    off = round_up(off + sizeof(float) * cap, 256);
   w.pa_off = off;    off = round_up(off + sizeof(int) * cap, 256);
@@ -214,6 +219,27 @@ WsLayout ws_layout(int B, int L, int d, int V) {
   w.pm2_off = off;   off = round_up(off + sizeof(float) * cap, 256);
   w.total = off;
   return w;
+}
+
+// The layout a workspace of ws_bytes can hold: all B*L rows when it is at least the full
+// layout, else the largest masked-row capacity whose layout fits (the total grows with the
+// capacity), or rows = 0 when not even one row fits.
+WsLayout ws_layout_for(int B, int L, int d, int V, size_t ws_bytes) {
+  const long long n = static_cast<long long>(B) * L;
+  WsLayout full = ws_layout(B, L, d, V, n);
+  if (ws_bytes >= full.total) return full;
+  WsLayout one = ws_layout(B, L, d, V, 1);
+  if (ws_bytes < one.total) {
+    one.rows = 0;
+    return one;
+  }
+  long long lo = 1, hi = n;                   // layout(lo) fits, layout(hi) does not
+  while (hi - lo > 1) {
+    const long long mid = lo + (hi - lo) / 2;
+    if (ws_layout(B, L, d, V, mid).total <= ws_bytes) lo = mid;
+    else hi = mid;
+  }
+  return ws_layout(B, L, d, V, lo);
 }
 
 // A step input (H or M) may live in device memory or in page-locked host memory that the
@@ -253,8 +279,15 @@ dllm_status launch_compact(const uint8_t* M, int B, int L, const int* win_lo, co
       return DLLM_ERR_CUDA;
     count_launch();
   }
+  const bool offsets = ntiles > static_cast<unsigned>(kCompactDirectTiles);
+  if (offsets) {
+    if (launch_pdl(compact_scan_kernel, dim3(1), dim3(kScanThreads), 0, s, tiles,
+                   static_cast<int>(ntiles)) != cudaSuccess)
+      return DLLM_ERR_CUDA;
+    count_launch();
+  }
   if (launch_pdl(compact_scatter_kernel, dim3(ntiles), dim3(kCompactThreads), 0, s, M, B, L, win_lo,
-                 win_hi, (const int*)tiles, row_idx, seq_off, count, status) != cudaSuccess)
+                 win_hi, (const int*)tiles, offsets, row_idx, seq_off, count, status) != cudaSuccess)
     return DLLM_ERR_CUDA;
   count_launch();
   return DLLM_OK;
@@ -308,7 +341,7 @@ dllm_status validate_logits(const LogitsArgs& a, bool debug, bool prepared = fal
                         a.raw.a, a.raw.t, a.raw.m2};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return DLLM_ERR_ALIGN;
-  if (a.ws_bytes < ws_layout(a.B, a.L, a.d, a.V).total) return DLLM_ERR_WORKSPACE;
+  if (ws_layout_for(a.B, a.L, a.d, a.V, a.ws_bytes).rows < 1) return DLLM_ERR_WORKSPACE;
   return DLLM_OK;
 }
 
@@ -330,7 +363,7 @@ dllm_status prepare_rows(const LogitsArgs& a, const DeviceState& ds, const WsLay
     return st;
   if (launch_pdl(gather_rows_kernel, dim3(ds.sms * 4), dim3(kGatherThreads), 0, a.s,
                  static_cast<const uint16_t*>(Hd), (const int*)a.row_idx, (const int*)a.count, n,
-                 a.d, Hm, ctr, w.n_ctr, ds.status) != cudaSuccess)
+                 w.rows, a.d, Hm, ctr, w.n_ctr, ds.status) != cudaSuccess)
     return DLLM_ERR_CUDA;
   count_launch();
   return DLLM_OK;
@@ -343,7 +376,7 @@ dllm_status run_logits(const LogitsArgs& a, bool debug, bool skip_prepare = fals
   if (st != DLLM_OK) return st;
   DeviceState* ds = nullptr;
   if ((st = device_state(&ds)) != DLLM_OK) return st;
-  const WsLayout w = ws_layout(a.B, a.L, a.d, a.V);
+  const WsLayout w = ws_layout_for(a.B, a.L, a.d, a.V, a.ws_bytes);
   uint8_t* ws = static_cast<uint8_t*>(a.ws);
   uint16_t* Hm = reinterpret_cast<uint16_t*>(ws + w.hm_off);
   float* pm = reinterpret_cast<float*>(ws + w.pm_off);
@@ -354,7 +387,7 @@ dllm_status run_logits(const LogitsArgs& a, bool debug, bool skip_prepare = fals
   int* ctr = reinterpret_cast<int*>(ws + w.ctr_off);
   const lm::Partials part{pm, ps, pa, pt, pm2};
   const lm::Outputs outs{a.tok, a.conf, a.lse, a.entropy, a.margin, a.raw, a.a_offset};
-  const long long n = static_cast<long long>(a.B) * a.L;
+  const long long n = w.rows;        // masked-row capacity of this workspace (B*L when full)
 
   // GEMM variant: 0 = chosen on the device from the masked count (lm::auto_variant, one
   // launch in clusters of two CTAs), 1 / 2 = forced single CTAs / CTA pairs (test hook)
@@ -524,7 +557,7 @@ dllm_status dllm_mask_compact_noalloc(const uint8_t* M, int32_t B, int32_t L, in
                         static_cast<cudaStream_t>(stream));
 }
 
-int32_t dllm_version(void) { return 10100; }
+int32_t dllm_version(void) { return 10200; }
 
 const char* dllm_status_string(dllm_status s) {
   switch (s) {
@@ -539,13 +572,25 @@ const char* dllm_status_string(dllm_status s) {
     case DLLM_ERR_BOUNDS: return "a device-side bound check failed";
     case DLLM_ERR_SCRATCH: return "B*L exceeds the fixed scratch of the allocation-free entry point";
     case DLLM_ERR_MEMORY: return "an input is neither device memory nor page-locked host memory";
+    case DLLM_ERR_CAPACITY: return "more masked rows than the workspace was sized for";
     default: return "unknown status";
   }
 }
 
 size_t dllm_workspace_bytes(int32_t B, int32_t L, int32_t d, int32_t V) {
   if (!shapes_ok(B, L) || V < 1 || d < DLLM_D_MULTIPLE || d % DLLM_D_MULTIPLE != 0) return 0;
-  return ws_layout(B, L, d, V).total;
+  return ws_layout(B, L, d, V, static_cast<long long>(B) * L).total;
+}
+
+size_t dllm_workspace_bytes_rows(int32_t B, int32_t L, int32_t d, int32_t V, int64_t max_rows) {
+  if (!shapes_ok(B, L) || V < 1 || d < DLLM_D_MULTIPLE || d % DLLM_D_MULTIPLE != 0 || max_rows < 1)
+    return 0;
+  return ws_layout(B, L, d, V, max_rows).total;
+}
+
+int64_t dllm_workspace_rows(int32_t B, int32_t L, int32_t d, int32_t V, size_t ws_bytes) {
+  if (!shapes_ok(B, L) || V < 1 || d < DLLM_D_MULTIPLE || d % DLLM_D_MULTIPLE != 0) return 0;
+  return ws_layout_for(B, L, d, V, ws_bytes).rows;
 }
 
 dllm_status dllm_mask_compact_window(const uint8_t* M, int32_t B, int32_t L, const int32_t* win_lo,
@@ -673,8 +718,8 @@ dllm_status dllm_prepare_rows(const uint16_t* H, const uint8_t* M, int32_t B, in
   const void* ptrs[] = {H, M, row_idx, seq_off, count, ws, win_lo, win_hi};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return DLLM_ERR_ALIGN;
-  const WsLayout w = ws_layout(B, L, d, V);
-  if (ws_bytes < w.total) return DLLM_ERR_WORKSPACE;
+  const WsLayout w = ws_layout_for(B, L, d, V, ws_bytes);
+  if (w.rows < 1) return DLLM_ERR_WORKSPACE;
   DeviceState* ds = nullptr;
   dllm_status st = device_state(&ds);
   if (st != DLLM_OK) return st;
@@ -831,6 +876,7 @@ dllm_status dllm_get_status(void* stream) {
   if (v != 0 && cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return DLLM_ERR_CUDA;
   if (v & kStatusTimeout) return DLLM_ERR_TIMEOUT;
   if (v & kStatusBounds) return DLLM_ERR_BOUNDS;
+  if (v & kStatusCapacity) return DLLM_ERR_CAPACITY;
   return DLLM_OK;
 }
 

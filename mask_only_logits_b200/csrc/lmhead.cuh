@@ -36,8 +36,10 @@
 // combine in order); with P = 1 the unit's statistics are the result.
 //
 // Every wait is bounded (ptx.cuh).  On a timeout the CTA raises its abort flag, every role
-// unwinds, the MMA issuer waits (bounded) for its issued MMAs, the CTA lingers 2 ms so that
-// TMA loads already in flight land, and TMEM is released before the kernel returns.
+// unwinds, the MMA issuer waits (bounded) for its issued MMAs, the producer of the CTA that
+// arms the stages waits (bounded) for the full barrier of the last phase it armed on every
+// stage, so that no TMA load is still writing shared memory, and TMEM is released before
+// the kernel returns.
 #pragma once
 #include "ptx.cuh"
 
@@ -540,6 +542,9 @@ __device__ __forceinline__ void lmhead_run(uint8_t* smem_raw, const CUtensorMap*
                              static_cast<int>(gridDim.x) / CG, gmax, C::BM);
   const int holder = static_cast<int>(blockIdx.x) / CG;
   const int KB = d / BK;
+  // producer thread of the arming CTA: stages armed so far (bit s), and the phase parity of
+  // the last arming of each stage (bit s), for the abort path's wait on loads in flight
+  uint32_t armed_mask = 0, armed_parity = 0;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -561,6 +566,8 @@ __device__ __forceinline__ void lmhead_run(uint8_t* smem_raw, const CUtensorMap*
           if (it == DLLM_FAULT_SKIP_STAGE) continue;
 #endif
           const uint32_t fb = smem_u32(&sm.full[s]);
+          armed_mask |= 1u << s;
+          armed_parity = (armed_parity & ~(1u << s)) | (ph << s);
           if constexpr (CG == 1) {
             mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
             tma_load_2d(smem_u32(sm.a + s * C::A_BYTES), tmA, fb, kb * BK, a_row);
@@ -825,10 +832,26 @@ __device__ __forceinline__ void lmhead_run(uint8_t* smem_raw, const CUtensorMap*
   tc_fence_before();
   if constexpr (CG == 1) __syncthreads();
   else cluster_sync();          // neither CTA leaves while its peer may still touch its smem
-  if (*abort_flag) {
-    // aborted: give TMA loads already in flight time to land before shared memory is freed
-    const unsigned long long t0 = globaltimer_ns();
-    while (globaltimer_ns() - t0 < 2000000ull) { }
+  // Every role has left its loop, so the abort flags no longer change; both CTAs of a pair
+  // read both flags and take the same decision.
+  bool aborted = *abort_flag != 0;
+  if constexpr (CG == 2)
+    aborted = aborted || ld_shared_cluster_s32(smem_u32(sm.abort_flag), rank ^ 1u) != 0;
+  if (aborted) {
+    // Loads already issued must land before shared memory is released: wait for the last
+    // armed phase of every stage (the arming CTA's barrier counts the loads of both CTAs of a
+    // pair).  A phase that was armed but whose loads were never all issued (a CTA that
+    // stopped first) holds the wait to the shared deadline, by which the issued loads have
+    // long landed.
+    if (warp == 0 && lane == 0 && (CG == 1 || leader)) {
+      const unsigned long long deadline = globaltimer_ns() + kWaitLimitNs;
+      for (int s = 0; s < C::kStages; ++s)
+        if (armed_mask & (1u << s))
+          if (!mbar_wait_until(smem_u32(&sm.full[s]), (armed_parity >> s) & 1u, deadline, status))
+            break;
+    }
+    if constexpr (CG == 1) __syncthreads();
+    else cluster_sync();
   }
   if (warp == 1) {
     __syncwarp();

@@ -14,6 +14,7 @@ namespace dllm {
 // Device status word bits (reported by dllm_get_status).
 constexpr int kStatusTimeout = 1;
 constexpr int kStatusBounds = 2;
+constexpr int kStatusCapacity = 4;   // more masked rows than the workspace holds
 
 // One second: every wait in these kernels is for one pipeline event (a tile landing, an
 // accumulator draining), which takes microseconds.
@@ -121,6 +122,20 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, i
   return true;
 }
 
+// Wait used on the abort path for loads already issued: completes when the phase with the
+// given parity completes, or returns false at the absolute `deadline` (globaltimer ns)
+// shared by all such waits of one unwind; ignores the abort flag.
+__device__ __forceinline__ bool mbar_wait_until(uint32_t bar, uint32_t parity,
+                                                unsigned long long deadline, int* status) {
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() > deadline) {
+      atomicOr(status, kStatusTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
 // ---------------------------------------------------------------------------------------
 // Clusters of two CTAs (the CTA pair of a cta_group::2 MMA)
 // ---------------------------------------------------------------------------------------
@@ -134,6 +149,19 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
 // co-scheduled and every wait in the kernels before it is bounded, so it always completes.
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
+// 32-bit load from the shared-memory word at the same offset in CTA `cta` of the cluster.
+__device__ __forceinline__ int ld_shared_cluster_s32(uint32_t addr, uint32_t cta) {
+  int v;
+  asm volatile(
+      "{\n\t.reg .b32 ra;\n\t"
+      "mapa.shared::cluster.u32 ra, %1, %2;\n\t"
+      "ld.shared::cluster.s32 %0, [ra];\n\t}"
+      : "=r"(v)
+      : "r"(addr), "r"(cta)
+      : "memory");
+  return v;
 }
 
 // A shared::cta address with the CTA-rank bit cleared names the same offset in rank 0 of

@@ -38,8 +38,8 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.dllm_version() == 10100
-    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8):
+    assert lib.dllm_version() == 10200
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8, -9, -10, -11):
         assert lib.dllm_status_string(code)
     assert lib.dllm_status_string(-99) == b"unknown status"
 
@@ -57,6 +57,50 @@ def test_workspace_bytes(lib):
     assert ws(1, 10, 100, 10) == 0           # d not a multiple of 64
     assert ws(1, 10, 64, 0) == 0
     assert ws(1 << 16, 1 << 15, 64, 10) == 0  # B*L >= 2^31
+
+
+def test_workspace_rows_arithmetic(lib):
+    """A workspace sized for max_rows masked rows: at least the gathered rows, growing with
+    max_rows, equal to the upper bound at B*L; the capacity of a workspace is the largest
+    row count whose size fits, so sizing for r rows gives a capacity of at least r."""
+    rows_b, cap = lib.dllm_workspace_bytes_rows, lib.dllm_workspace_rows
+    for B, L, d, V in [(1, 131072, 4096, 126464), (8, 8192, 2048, 151936), (1, 256, 256, 4096),
+                       (3, 97, 192, 777)]:
+        n = B * L
+        full = lib.dllm_workspace_bytes(B, L, d, V)
+        assert rows_b(B, L, d, V, n) == full and rows_b(B, L, d, V, 10 * n) == full
+        prev = 0
+        for r in sorted({1, 2, 127, 128, 129, 4096, n // 10, n // 2, (9 * n) // 10, n - 1, n}):
+            if r < 1 or r > n:
+                continue
+            b = rows_b(B, L, d, V, r)
+            assert b >= 2 * d * r and b >= prev and b <= full, (B, L, d, V, r)
+            prev = b
+            c = cap(B, L, d, V, b)
+            assert r <= c <= n and rows_b(B, L, d, V, c) <= b, (r, c)
+            if c < n:
+                assert rows_b(B, L, d, V, c + 1) > b                     # the largest that fits
+            assert cap(B, L, d, V, b - 1) < r or rows_b(B, L, d, V, r) <= b - 1
+        assert cap(B, L, d, V, full) == n and cap(B, L, d, V, 1 << 62) == n
+        assert cap(B, L, d, V, rows_b(B, L, d, V, 1) - 1) == 0
+    # the cfg3 sweep: the workspace of a step follows its masked count
+    B, L, d, V = 1, 131072, 4096, 126464
+    for r_m in (0.1, 0.5, 0.9):
+        m = int(r_m * L)
+        assert rows_b(B, L, d, V, m) < lib.dllm_workspace_bytes(B, L, d, V) * (r_m + 0.02)
+    assert rows_b(B, L, d, V, 0) == 0 and rows_b(0, L, d, V, 5) == 0
+    assert cap(B, L, 100, V, 1 << 30) == 0
+
+
+def test_arena_validates_on_host(lib):
+    out = ctypes.c_void_p()
+    assert lib.dllm_arena_create(1 << 20, 0, None) == -1
+    assert lib.dllm_arena_create(0, 0, ctypes.byref(out)) == -3
+    assert lib.dllm_arena_map(None, 10) == -1
+    assert lib.dllm_arena_ptr(None) is None
+    assert lib.dllm_arena_mapped(None) == 0 and lib.dllm_arena_reserved(None) == 0
+    assert lib.dllm_arena_chunk(None) == 0
+    assert lib.dllm_arena_destroy(None) == 0
 
 
 def _p(x):

@@ -43,7 +43,11 @@ def _compact_case(dl, M_np):
                                    (2, 8191, 0.3), (1, 8193, 0.99), (4, 17, 0.0), (4, 17, 1.0),
                                    (1, 16, 1.0), (1, 15, 1.0), (37, 1111, 0.5),
                                    # 16 tiles (one launch) / 17 and 19 tiles (count + scatter)
-                                   (16, 8192, 0.5), (1, 131073, 0.5), (3, 50000, 0.4)])
+                                   (16, 8192, 0.5), (1, 131073, 0.5), (3, 50000, 0.4),
+                                   # 64 tiles (offsets summed per CTA) / 65, 129 and 184 tiles
+                                   # (offsets from the scan launch)
+                                   (64, 8192, 0.5), (65, 8192, 0.5), (1, 1048577, 0.5),
+                                   (3, 500000, 0.6)])
 def test_compact_bit_exact(dl, B, L, p):
     rng = np.random.default_rng(B * 1000 + L)
     M = (rng.random((B, L)) < p).astype(np.uint8)
@@ -81,7 +85,8 @@ def _compact_window_case(dl, M_np, lo, hi):
 
 @pytest.mark.parametrize("B,L,p", [(1, 256, 0.5), (8, 8192, 1.0), (3, 1000, 0.5), (7, 3, 0.6),
                                    (5, 1, 1.0), (2, 8191, 0.3), (37, 1111, 0.5), (1, 131072, 0.9),
-                                   (64, 17, 0.8), (16, 8192, 0.7), (20, 8192, 0.7), (1, 131073, 0.5)])
+                                   (64, 17, 0.8), (16, 8192, 0.7), (20, 8192, 0.7), (1, 131073, 0.5),
+                                   (80, 8192, 0.7), (2, 300001, 0.5)])
 def test_compact_windows_bit_exact(dl, B, L, p):
     """Current-block-only compaction: windows of random placement and width, including
     empty, inverted, negative and past-the-end ones, and sequences shorter than a vector."""
