@@ -835,8 +835,10 @@ __device__ __forceinline__ void lmhead_run(uint8_t* smem_raw, const CUtensorMap*
   // Every role has left its loop, so the abort flags no longer change; both CTAs of a pair
   // read both flags and take the same decision.
   bool aborted = *abort_flag != 0;
-  if constexpr (CG == 2)
+  if constexpr (CG == 2) {
     aborted = aborted || ld_shared_cluster_s32(smem_u32(sm.abort_flag), rank ^ 1u) != 0;
+    cluster_sync();             // the peer's shared memory stays alive until both have read
+  }
   if (aborted) {
     // Loads already issued must land before shared memory is released: wait for the last
     // armed phase of every stage (the arming CTA's barrier counts the loads of both CTAs of a
