@@ -37,6 +37,10 @@ constexpr int kSelThreads = 1024;
 constexpr int kSelMaxK = 1024;
 constexpr int kSelStage = 4096;     // up to this many candidates: keys staged in shared memory
 constexpr int kSelRankMax = 256;    // up to this many: output place by rank, no select or sort
+// Passes over candidates read kSelUnroll keys per thread (rows base + j * kSelThreads + tid)
+// before using any, so that a pass over a long sequence (e.g. 117961 candidates: 15 chunks
+// instead of 116 dependent loads per thread) is not bound by one L2 round trip per key.
+constexpr int kSelUnroll = 8;
 static_assert(kSelRankMax <= kSelThreads && kSelRankMax <= kSelStage, "one staged key per thread");
 
 // Float -> unsigned with the same order (for non-NaN values).
@@ -50,7 +54,7 @@ __device__ __forceinline__ unsigned long long sel_key(uint32_t okey, int r) {
          static_cast<unsigned long long>(~static_cast<uint32_t>(r));
 }
 
-__global__ void __launch_bounds__(kSelThreads)
+__global__ void __launch_bounds__(kSelThreads, 1)
 select_unmask_kernel(const float* __restrict__ conf, const int* __restrict__ row_idx,
                      const int* __restrict__ seq_off, int n_pos, int L, int k,
                      bool use_threshold, float threshold, int min_sel, bool ascending,
@@ -109,6 +113,7 @@ select_unmask_kernel(const float* __restrict__ conf, const int* __restrict__ row
     __syncthreads();
     const uint32_t tq = okey(threshold);
     int mine = 0;
+#pragma unroll 8
     for (int r = c0 + tid; r < c1; r += kSelThreads) mine += key_of(r) >= tq ? 1 : 0;
     for (int o = 16; o > 0; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
     if (lane == 0 && mine) atomicAdd(&sh_q, mine);
@@ -160,15 +165,21 @@ select_unmask_kernel(const float* __restrict__ conf, const int* __restrict__ row
       __syncthreads();
       // warp-aggregated histogram: confidences crowd into few bins (most share their top
       // bits), so lanes with the same bin add their count once
-      for (int base = c0; base < c1; base += kSelThreads) {
-        const int r = base + tid;
-        uint32_t bin = 0xFFFFFFFFu;
-        if (r < c1) {
-          const uint32_t u = key_of(r);
-          if ((u & pmask) == prefix) bin = (u >> shift) & 255u;
+      for (int base = c0; base < c1; base += kSelThreads * kSelUnroll) {
+        uint32_t u[kSelUnroll];
+#pragma unroll
+        for (int j = 0; j < kSelUnroll; ++j) {
+          const int r = base + j * kSelThreads + tid;
+          u[j] = r < c1 ? key_of(r) : 0u;
         }
-        const unsigned peers = __match_any_sync(0xffffffffu, bin);
-        if (bin != 0xFFFFFFFFu && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+#pragma unroll
+        for (int j = 0; j < kSelUnroll; ++j) {
+          const int r = base + j * kSelThreads + tid;
+          uint32_t bin = 0xFFFFFFFFu;
+          if (r < c1 && (u[j] & pmask) == prefix) bin = (u[j] >> shift) & 255u;
+          const unsigned peers = __match_any_sync(0xffffffffu, bin);
+          if (bin != 0xFFFFFFFFu && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+        }
       }
       __syncthreads();
       if (warp == 0) {
@@ -201,27 +212,35 @@ select_unmask_kernel(const float* __restrict__ conf, const int* __restrict__ row
     const uint32_t T = prefix;
     if (tid == 0) sh_taken = 0;
     __syncthreads();
-    for (int base = c0; base < c1; base += kSelThreads) {
-      const int r = base + tid;
-      uint32_t u = 0;
-      if (r < c1) u = key_of(r);
-      const bool gt = r < c1 && u > T;
-      const bool eq = r < c1 && u == T;
-      if (gt) keys[atomicAdd(&sh_n, 1)] = sel_key(u, r);
-      const unsigned bal = __ballot_sync(0xffffffffu, eq);
-      if (lane == 0) warp_cnt[warp] = __popc(bal);
-      __syncthreads();
-      int before = sh_taken;
-      for (int w = 0; w < warp; ++w) before += warp_cnt[w];
-      before += __popc(bal & ((1u << lane) - 1u));
-      if (eq && before < krem) keys[atomicAdd(&sh_n, 1)] = sel_key(u, r);
-      __syncthreads();
-      if (tid == 0) {
-        int tot = 0;
-        for (int w = 0; w < kSelThreads / 32; ++w) tot += warp_cnt[w];
-        sh_taken += tot;
+    for (int base = c0; base < c1; base += kSelThreads * kSelUnroll) {
+      uint32_t uu[kSelUnroll];
+#pragma unroll
+      for (int j = 0; j < kSelUnroll; ++j) {
+        const int r = base + j * kSelThreads + tid;
+        uu[j] = r < c1 ? key_of(r) : 0u;
       }
-      __syncthreads();
+      // blocks of kSelThreads rows in ascending order, so "first in row order" holds
+      for (int j = 0; j < kSelUnroll && base + j * kSelThreads < c1; ++j) {
+        const int r = base + j * kSelThreads + tid;
+        const uint32_t u = uu[j];
+        const bool gt = r < c1 && u > T;
+        const bool eq = r < c1 && u == T;
+        if (gt) keys[atomicAdd(&sh_n, 1)] = sel_key(u, r);
+        const unsigned bal = __ballot_sync(0xffffffffu, eq);
+        if (lane == 0) warp_cnt[warp] = __popc(bal);
+        __syncthreads();
+        int before = sh_taken;
+        for (int w = 0; w < warp; ++w) before += warp_cnt[w];
+        before += __popc(bal & ((1u << lane) - 1u));
+        if (eq && before < krem) keys[atomicAdd(&sh_n, 1)] = sel_key(u, r);
+        __syncthreads();
+        if (tid == 0) {
+          int tot = 0;
+          for (int w = 0; w < kSelThreads / 32; ++w) tot += warp_cnt[w];
+          sh_taken += tot;
+        }
+        __syncthreads();
+      }
     }
   }
   __syncthreads();
