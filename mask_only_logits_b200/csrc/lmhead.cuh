@@ -62,6 +62,9 @@
 #ifndef DLLM_A_EVICT_LAST
 #define DLLM_A_EVICT_LAST 0       // single-CTA body: load Hm tiles with the L2 evict_last hint
 #endif
+#ifndef DLLM_PACE_TILES
+#define DLLM_PACE_TILES 0         // single-CTA body, full groups: lead over the stream's slowest
+#endif                            // holder, in tiles (0 = no pacing)
 
 namespace dllm {
 namespace lm {
@@ -578,7 +581,39 @@ __device__ __forceinline__ void lmhead_run(uint8_t* smem_raw, const CUtensorMap*
       // cleared), which the leader arms for the bytes of both CTAs.
       uint32_t it = 0;
       const uint64_t a_policy = DLLM_A_EVICT_LAST ? policy_evict_last() : 0ull;
+      // Pacing (single CTAs, groups of gmax m-tiles): the holders of one stream read the
+      // same W tiles, so W comes from HBM once per group only while they stay close.  Each
+      // holder publishes how many tiles it has started (holders of one stream start the same
+      // number per full group) and, before a tile, waits until every stream-mate has
+      // started at least DLLM_PACE_TILES fewer.  The slowest holder never waits, so every
+      // wait ends; it is bounded all the same.
+      int* const progress = unit_ctr + ((n_cap + 127) / 128 + 2);
+      int started = 0;
+      auto pace = [&](int m_tile) -> bool {
+        if (DLLM_PACE_TILES <= 0 || CG != 1 || pl.ngroups < 2 || pl.rem) return true;
+        const int g = m_tile / pl.gmax;
+        if (pl.group_size(g) != pl.gmax) return true;            // the last, smaller group
+        st_relaxed_gpu(progress + holder, started);
+        const int need = started - DLLM_PACE_TILES;
+        if (need <= 0) return true;
+        const int first = (holder / pl.gmax) * pl.gmax;          // the stream's first holder
+        const unsigned long long t0 = globaltimer_ns();
+        for (;;) {
+          bool behind = false;
+          for (int j = 0; j < pl.gmax; ++j) behind |= ld_relaxed_gpu(progress + first + j) < need;
+          if (!behind) return true;
+          if (*abort_flag) return false;
+          if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(status, kStatusTimeout);
+            *abort_flag = 1;
+            return false;
+          }
+          __nanosleep(256);
+        }
+      };
       auto load_tile = [&](int m_tile, int n) -> bool {
+        if (!pace(m_tile)) return false;
+        ++started;
         const int a_row = m_tile * C::BM + static_cast<int>(rank) * C::BM_CTA;
         const int b_row = n * C::kBN + static_cast<int>(rank) * C::B_ROWS;
         for (int kb = 0; kb < KB; ++kb, ++it) {
