@@ -62,6 +62,9 @@
 #ifndef DLLM_A_EVICT_LAST
 #define DLLM_A_EVICT_LAST 0       // single-CTA body: load Hm tiles with the L2 evict_last hint
 #endif
+#ifndef DLLM_EPI_PACKED
+#define DLLM_EPI_PACKED 0         // epilogue: 3-input max and packed fp32x2 fma / add
+#endif
 #ifndef DLLM_PACE_TILES
 #define DLLM_PACE_TILES 0         // single-CTA body, full groups: lead over the stream's slowest
 #endif                            // holder, in tiles (0 = no pacing)
@@ -327,9 +330,21 @@ __device__ __forceinline__ void fold_chunk(float (&v)[32], int col0, int V, RowS
     for (int j = 0; j < 32; ++j)
       if (col0 + j >= V) v[j] = -INFINITY;
   }
-  float mx = v[0];
+  float mx;
+  if constexpr (DLLM_EPI_PACKED) {
+    // 32 -> 11 -> 4 -> 1 with three-input maxima (17 instructions instead of 31)
+    float t[11];
 #pragma unroll
-  for (int j = 1; j < 32; ++j) mx = fmaxf(mx, v[j]);
+    for (int i = 0; i < 10; ++i) t[i] = max3f(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+    t[10] = fmaxf(v[30], v[31]);
+    const float u0 = max3f(t[0], t[1], t[2]), u1 = max3f(t[3], t[4], t[5]);
+    const float u2 = max3f(t[6], t[7], t[8]), u3 = fmaxf(t[9], t[10]);
+    mx = fmaxf(max3f(u0, u1, u2), u3);
+  } else {
+    mx = v[0];
+#pragma unroll
+    for (int j = 1; j < 32; ++j) mx = fmaxf(mx, v[j]);
+  }
   if (mx == -INFINITY) return;                 // the whole chunk is past the vocabulary
   float c2 = -INFINITY;                        // chunk's second largest (= mx on a tie)
   if constexpr (kExt) {
@@ -373,6 +388,21 @@ __device__ __forceinline__ void fold_chunk(float (&v)[32], int col0, int V, RowS
       t1 += e1 > 0.f ? e1 * (v[j + 1] - st.m) : 0.f;
     }
     st.t += t0 + t1;
+  } else if constexpr (DLLM_EPI_PACKED) {
+    // the same arithmetic as the scalar loop below (same four accumulators, same order and
+    // roundings), with fma and add two lanes per instruction
+    const uint64_t scale = pack2f(kLog2e, kLog2e), shift = pack2f(-mb, -mb);
+    uint64_t acc01 = pack2f(0.f, 0.f), acc23 = pack2f(0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+      float a0, a1, a2, a3;
+      unpack2f(fma2f(pack2f(v[j + 0], v[j + 1]), scale, shift), a0, a1);
+      unpack2f(fma2f(pack2f(v[j + 2], v[j + 3]), scale, shift), a2, a3);
+      acc01 = add2f(acc01, pack2f(ex2_approx(a0), ex2_approx(a1)));
+      acc23 = add2f(acc23, pack2f(ex2_approx(a2), ex2_approx(a3)));
+    }
+    unpack2f(acc01, s0, s1);
+    unpack2f(acc23, s2, s3);
   } else {
 #pragma unroll
     for (int j = 0; j < 32; j += 4) {
