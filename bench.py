@@ -98,9 +98,9 @@ def roofline_s(cfg, M: int, peaks: dict) -> float:
 
 
 def gemm_paired(variant: int, count: int) -> bool:
-    """Whether the GEMM runs on CTA pairs: forced (1, 3 single; 2, 4 pairs), or the library's
-    choice from the masked count (pairs for 129..16384 rows)."""
-    return variant in (2, 4) or (variant == 0 and 128 < count <= 16384)
+    """Whether the GEMM runs on CTA pairs: forced (1, 2), or the library's choice from the
+    masked count (pairs for 129..16384 rows)."""
+    return variant == 2 or (variant == 0 and 128 < count <= 16384)
 
 
 # A timed region at least this long runs in the regime of the measured sustained bf16 rate
@@ -579,9 +579,8 @@ def main() -> None:
                          "GEMM's extended epilogue)")
     ap.add_argument("--threshold", type=float, default=None,
                     help="threshold-based parallel unmasking on the policy's score (default: top-k)")
-    ap.add_argument("--gemm-variant", type=int, default=0, choices=[0, 1, 2, 3, 4],
-                    help="0 = library default, 1 = single-SM GEMM, 2 = paired-SM GEMM, 3 / 4 = "
-                         "the same with 128-column vocabulary tiles")
+    ap.add_argument("--gemm-variant", type=int, default=0, choices=[0, 1, 2],
+                    help="0 = library default, 1 = single-SM GEMM, 2 = paired-SM GEMM")
     ap.add_argument("--arena", action="store_true",
                     help="the step's workspace in a virtual-memory arena mapped for the step's "
                          "own masked count (steps run one at a time); reports the mapped bytes "
@@ -777,8 +776,7 @@ def main() -> None:
         paired = gemm_paired(args.gemm_variant, count)
         mode = 1 if step.stats else 0
         gemm_kernel_name = (f"lmhead_auto_kernel<{mode}>" if args.gemm_variant == 0 else
-                            f"lmhead_kernel<{1 if args.gemm_variant in (1, 3) else 2}, "
-                            f"{256 if args.gemm_variant <= 2 else 128}, {mode}>")
+                            f"lmhead_kernel<{args.gemm_variant}, {mode}>")
         line = dict(
             metric=METRIC, value=rows_s, unit=UNIT, n_gpus=world, steps=args.steps,
             warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True, scaling="weak",

@@ -487,14 +487,12 @@ dllm_status dllm_debug_lse_merge(const float* part_m, const float* part_s,
 /*
  * Test hook: choose the tensor-core GEMM variant used by later calls in this process:
  * 2 = CTA pairs (tcgen05 cta_group::2, 256x256 tiles over two SMs), 1 = single CTAs
- * (cta_group::1, 128x256 tiles), 4 / 3 = pairs / single CTAs with 128-column vocabulary
- * tiles, 0 = the default: one launch that picks on the device, from the masked count,
- * pairs for 129..16384 rows and single CTAs otherwise, and 128-column tiles when the
- * masked rows fit one group of m-tiles whose vocabulary tiles spread more evenly over the
- * SMs that way.  Results agree to fp32 rounding; the variants differ in speed.  Returns
- * DLLM_ERR_SHAPE for other values.
+ * (cta_group::1, 128x256 tiles), 0 = the default: one launch that picks on the device,
+ * from the masked count, pairs for 129..16384 rows and single CTAs otherwise.  Results
+ * agree to fp32 rounding; the variants differ in speed.  Returns DLLM_ERR_SHAPE for other
+ * values.
  */
-dllm_status dllm_debug_set_gemm_variant(int32_t variant);
+dllm_status dllm_debug_set_gemm_variant(int32_t cta_group);
 
 /*
  * Kernel-time accounting for benchmarks.  dllm_prof_begin() starts recording a CUDA event

@@ -125,7 +125,8 @@ class Arena:
 
     def __init__(self, reserve_bytes: int, chunk_bytes: int = 0, device=None):
         if device is not None:
-            torch.cuda.set_device(device)
+            d = torch.device(device)
+            torch.cuda.set_device(d.index if d.index is not None else torch.cuda.current_device())
         self.device = torch.device("cuda", torch.cuda.current_device())
         h = ctypes.c_void_p()
         _check(lib().dllm_arena_create(reserve_bytes, chunk_bytes, ctypes.byref(h)),
@@ -434,12 +435,10 @@ def debug_lse_merge(part_m, part_s, part_a, tok, conf, lse, stream=None) -> None
         "dllm_debug_lse_merge")
 
 
-def debug_set_gemm_variant(variant: int) -> None:
-    """Test hook: 2 = paired-SM GEMM, 1 = single-SM GEMM (256-column vocabulary tiles), 4 / 3
-    = the same with 128-column tiles, 0 = default (chosen on the device from the masked
-    count: pairs for 129..16384 rows, single SMs otherwise; narrow tiles when one group of
-    m-tiles divides into them more evenly)."""
-    _check(lib().dllm_debug_set_gemm_variant(variant), "dllm_debug_set_gemm_variant")
+def debug_set_gemm_variant(cta_group: int) -> None:
+    """Test hook: 2 = paired-SM GEMM, 1 = single-SM GEMM, 0 = default (chosen on the device
+    from the masked count: pairs for 129..16384 rows, single SMs otherwise)."""
+    _check(lib().dllm_debug_set_gemm_variant(cta_group), "dllm_debug_set_gemm_variant")
 
 
 def prof_begin() -> None:

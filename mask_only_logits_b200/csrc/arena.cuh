@@ -136,26 +136,29 @@ dllm_status dllm_arena_map(dllm_arena* a, size_t bytes) {
   const size_t have = a->handles.size();
   if (want > have) {
     const CUmemAllocationProp prop = device_prop(a->device);
+    CUmemAccessDesc acc = {};
+    acc.location.type = CU_MEM_LOCATION_TYPE_DEVICE;
+    acc.location.id = a->device;
+    acc.flags = CU_MEM_ACCESS_FLAGS_PROT_READWRITE;
     for (size_t i = have; i < want; ++i) {
       CUmemGenericAllocationHandle h;
       if (d.create(&h, a->chunk, &prop, 0) != CUDA_SUCCESS) {
         trim(a, have);
         return DLLM_ERR_CUDA;
       }
-      if (d.map(a->base + i * a->chunk, a->chunk, 0, h, 0) != CUDA_SUCCESS) {
+      const CUdeviceptr at = a->base + i * a->chunk;
+      if (d.map(at, a->chunk, 0, h, 0) != CUDA_SUCCESS) {
         d.release(h);
         trim(a, have);
         return DLLM_ERR_CUDA;
       }
       a->handles.push_back(h);
-    }
-    CUmemAccessDesc acc = {};
-    acc.location.type = CU_MEM_LOCATION_TYPE_DEVICE;
-    acc.location.id = a->device;
-    acc.flags = CU_MEM_ACCESS_FLAGS_PROT_READWRITE;
-    if (d.set_access(a->base + have * a->chunk, (want - have) * a->chunk, &acc, 1) != CUDA_SUCCESS) {
-      trim(a, have);
-      return DLLM_ERR_CUDA;
+      // access per chunk: a chunk unmapped later is then referenced by nothing else (an
+      // access range spanning several chunks kept released chunks allocated)
+      if (d.set_access(at, a->chunk, &acc, 1) != CUDA_SUCCESS) {
+        trim(a, have);
+        return DLLM_ERR_CUDA;
+      }
     }
   } else if (want < have) {
     // no kernel still running may touch a chunk that is about to be released

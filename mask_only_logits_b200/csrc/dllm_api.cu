@@ -50,13 +50,11 @@ struct DeviceState {
 };
 
 // GEMM variant: 2 = CTA pairs (cta_group::2, 256x256 tiles), 1 = single CTAs
-// (cta_group::1, 128x256 tiles), 4 / 3 = the same with 128-column vocabulary tiles, all
-// forced (test hook).  0 = default: chosen on the device from the masked count
-// (lm::auto_choice): pairs for 129..16384 rows (the larger tile does more work per clock),
-// single CTAs for one m-tile (a pair would compute 128 empty rows) and for long GEMMs
-// (measured under the 1 kW power cap, the single-CTA kernel does more work per joule and
-// sustains a higher clock); narrow vocabulary tiles when one group of m-tiles divides
-// into them more evenly.
+// (cta_group::1, 128x256 tiles), both forced (test hook).  0 = default: chosen on the
+// device from the masked count (lm::auto_variant): pairs for 129..16384 rows (the larger
+// tile does more work per clock), single CTAs for one m-tile (a pair would compute 128
+// empty rows) and for long GEMMs (measured under the 1 kW power cap, the single-CTA kernel
+// does more work per joule and sustains a higher clock).
 std::atomic<int> g_gemm_variant{0};
 
 std::mutex g_mu;
@@ -105,20 +103,6 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-constexpr auto kSmemAttr = cudaFuncAttributeMaxDynamicSharedMemorySize;
-
-// Raise the shared-memory limit of the three epilogue modes of one fixed GEMM body.
-template <int CG, int TBN>
-cudaError_t set_smem() {
-  constexpr int bytes = lm::Cfg<CG, TBN>::SMEM_BYTES;
-  cudaError_t e = cudaFuncSetAttribute(lm::lmhead_kernel<CG, TBN, lm::kModeStats>, kSmemAttr, bytes);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(lm::lmhead_kernel<CG, TBN, lm::kModeStatsExt>, kSmemAttr, bytes);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(lm::lmhead_kernel<CG, TBN, lm::kModeDebugStore>, kSmemAttr, bytes);
-  return e;
-}
-
 // Per-device setup, once: check the architecture, find g_status, raise the GEMM's shared
 // memory limit, resolve the tensor-map encoder.
 dllm_status device_state(DeviceState** out) {
@@ -139,12 +123,17 @@ dllm_status device_state(DeviceState** out) {
       void* p = nullptr;
       if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) st.err = DLLM_ERR_CUDA;
       st.status = static_cast<int*>(p);
+      const auto smem_attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
       if (st.err == DLLM_OK &&
-          (set_smem<1, lm::BN>() || set_smem<2, lm::BN>() || set_smem<1, lm::BN_NARROW>() ||
-           set_smem<2, lm::BN_NARROW>() ||
-           cudaFuncSetAttribute(lm::lmhead_auto_kernel<lm::kModeStats>, kSmemAttr, lm::kAutoSmemBytes) ||
-           cudaFuncSetAttribute(lm::lmhead_auto_kernel<lm::kModeStatsExt>, kSmemAttr, lm::kAutoSmemBytes) ||
-           cudaFuncSetAttribute(lm::lmhead_auto_kernel<lm::kModeDebugStore>, kSmemAttr, lm::kAutoSmemBytes)))
+          (cudaFuncSetAttribute(lm::lmhead_kernel<1, lm::kModeStats>, smem_attr, lm::Cfg<1>::SMEM_BYTES) ||
+           cudaFuncSetAttribute(lm::lmhead_kernel<1, lm::kModeStatsExt>, smem_attr, lm::Cfg<1>::SMEM_BYTES) ||
+           cudaFuncSetAttribute(lm::lmhead_kernel<1, lm::kModeDebugStore>, smem_attr, lm::Cfg<1>::SMEM_BYTES) ||
+           cudaFuncSetAttribute(lm::lmhead_kernel<2, lm::kModeStats>, smem_attr, lm::Cfg<2>::SMEM_BYTES) ||
+           cudaFuncSetAttribute(lm::lmhead_kernel<2, lm::kModeStatsExt>, smem_attr, lm::Cfg<2>::SMEM_BYTES) ||
+           cudaFuncSetAttribute(lm::lmhead_kernel<2, lm::kModeDebugStore>, smem_attr, lm::Cfg<2>::SMEM_BYTES) ||
+           cudaFuncSetAttribute(lm::lmhead_auto_kernel<lm::kModeStats>, smem_attr, lm::kAutoSmemBytes) ||
+           cudaFuncSetAttribute(lm::lmhead_auto_kernel<lm::kModeStatsExt>, smem_attr, lm::kAutoSmemBytes) ||
+           cudaFuncSetAttribute(lm::lmhead_auto_kernel<lm::kModeDebugStore>, smem_attr, lm::kAutoSmemBytes)))
         st.err = DLLM_ERR_CUDA;
       if (st.err == DLLM_OK) {
         // how many CTA pairs of the paired GEMM can be resident at once (a persistent grid
@@ -161,7 +150,7 @@ dllm_status device_state(DeviceState** out) {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int clusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&clusters, lm::lmhead_kernel<2, lm::BN, lm::kModeStats>, &cfg) != cudaSuccess)
+        if (cudaOccupancyMaxActiveClusters(&clusters, lm::lmhead_kernel<2, lm::kModeStats>, &cfg) != cudaSuccess)
           clusters = 0;
         st.pairs = clusters < lm::kMaxCtas / 2 ? clusters : lm::kMaxCtas / 2;
       }
@@ -200,7 +189,6 @@ WsLayout ws_layout(int B, int L, int d, int V, long long rows) {
   w.rows = rows;
   // partial entries: worst case over the masked count (up to `rows`), the largest number of
   // work holders and either GEMM variant; fewer masked rows never need more.
-  // (the number of groups does not depend on the vocabulary tile width)
   const lm::Plan w1 = lm::Plan::make(static_cast<int>(rows), V, lm::kMaxCtas, lm::Cfg<1>::kGroupM,
                                      lm::Cfg<1>::BM);
   const lm::Plan w2 = lm::Plan::make(static_cast<int>(rows), V, lm::kMaxCtas / 2, lm::Cfg<2>::kGroupM,
@@ -218,9 +206,8 @@ WsLayout ws_layout(int B, int L, int d, int V, long long rows) {
   if (r2 > cap) cap = r2;
   if (cap < 1) cap = 1;
   w.part_cap = cap;
-  // one counter per (m-tile, CTA of the pair): ceil(rows / 128) + 2 covers both variants;
-  // then one progress word per work holder (the GEMM's optional pacing)
-  w.n_ctr = static_cast<int>((rows + 127) / 128 + 2 + lm::kMaxCtas);
+  // one counter per (m-tile, CTA of the pair): ceil(rows / 128) + 2 covers both variants
+  w.n_ctr = static_cast<int>((rows + 127) / 128 + 2);
   size_t off = 0;
   w.tiles_off = off; off = round_up(off + sizeof(int) * ntiles, 256);
   w.ctr_off = off;   off = round_up(off + sizeof(int) * static_cast<size_t>(w.n_ctr), 256);
@@ -404,52 +391,37 @@ dllm_status run_logits(const LogitsArgs& a, bool debug, bool skip_prepare = fals
 
   // GEMM variant: 0 = chosen on the device from the masked count (lm::auto_variant, one
   // launch in clusters of two CTAs), 1 / 2 = forced single CTAs / CTA pairs (test hook)
-  int variant = g_gemm_variant.load();
-  if (ds->pairs < 1) variant = variant == 4 ? 3 : (variant == 2 ? 1 : variant);   // no CTA pairs
-  if (ds->pairs < 1 && variant == 0) variant = 1;
-  const int cg = variant == 0 ? 0 : (variant == 2 || variant == 4 ? 2 : 1);
-  const int fixed_bn = variant >= 3 ? lm::BN_NARROW : lm::BN;
+  int cg = g_gemm_variant.load();
+  if (ds->pairs < 1) cg = 1;                                   // no CTA pairs on this device
   const int single_holders = cg == 0 ? 2 * ds->pairs : (ds->sms < lm::kMaxCtas ? ds->sms : lm::kMaxCtas);
   for (int v = 1; v <= 2; ++v) {
     if (cg != 0 && cg != v) continue;
-    for (int bn : {lm::BN, lm::BN_NARROW}) {
-      if (cg != 0 && bn != fixed_bn) continue;
-      // largest partial footprint over every masked count this body may run: all positions
-      // masked, or any count that fits one group of m-tiles (remainder holders)
-      const int holders = v == 2 ? ds->pairs : single_holders;
-      const int bm = v == 2 ? lm::Cfg<2>::BM : lm::Cfg<1>::BM;
-      const int gmax = v == 2 ? lm::Cfg<2>::kGroupM : lm::Cfg<1>::kGroupM;
-      long long need = lm::Plan::make(static_cast<int>(n), a.V, holders, gmax, bm, bn).part_entries();
-      const long long mt = (n + bm - 1) / bm;
-      for (long long m = 1; m <= mt && m <= gmax; ++m) {
-        const long long c = m * bm < n ? m * bm : n;
-        const long long e =
-            lm::Plan::make(static_cast<int>(c), a.V, holders, gmax, bm, bn).part_entries();
-        if (e > need) need = e;
-      }
-      if (need > w.part_cap) return DLLM_ERR_WORKSPACE;                // cannot happen on B200
+    // largest partial footprint over every masked count this variant may run: all
+    // positions masked, or any count that fits one group of m-tiles (remainder holders)
+    const int holders = v == 2 ? ds->pairs : single_holders;
+    const int bm = v == 2 ? lm::Cfg<2>::BM : lm::Cfg<1>::BM;
+    const int gmax = v == 2 ? lm::Cfg<2>::kGroupM : lm::Cfg<1>::kGroupM;
+    long long need = lm::Plan::make(static_cast<int>(n), a.V, holders, gmax, bm).part_entries();
+    const long long mt = (n + bm - 1) / bm;
+    for (long long m = 1; m <= mt && m <= gmax; ++m) {
+      const long long c = m * bm < n ? m * bm : n;
+      const long long e = lm::Plan::make(static_cast<int>(c), a.V, holders, gmax, bm).part_entries();
+      if (e > need) need = e;
     }
+    if (need > w.part_cap) return DLLM_ERR_WORKSPACE;                  // cannot happen on B200
   }
 
   if (!skip_prepare) {
     if ((st = prepare_rows(a, *ds, w)) != DLLM_OK) return st;
   }
 
-  // W is staged tile-width / CTA-group rows per CTA: 256 (single, wide), 128 (pairs wide,
-  // single narrow) or 64 (pairs narrow)
-  const int b_rows = cg == 0 ? 0 : fixed_bn / cg;
-  CUtensorMap tmA, tmB256, tmB128, tmB64;
+  // W is staged 256 rows per CTA by single CTAs and 128 rows per CTA by pairs
+  CUtensorMap tmA, tmB1, tmB2;
   if (make_tmap(&tmA, Hm, static_cast<uint64_t>(n), a.d, 128) != DLLM_OK) return DLLM_ERR_CUDA;
-  if ((cg == 0 || b_rows == 256) &&
-      make_tmap(&tmB256, a.W, static_cast<uint64_t>(a.V), a.d, 256) != DLLM_OK)
+  if (cg != 2 && make_tmap(&tmB1, a.W, static_cast<uint64_t>(a.V), a.d, lm::BN) != DLLM_OK)
     return DLLM_ERR_CUDA;
-  if ((cg == 0 || b_rows == 128) &&
-      make_tmap(&tmB128, a.W, static_cast<uint64_t>(a.V), a.d, 128) != DLLM_OK)
+  if (cg != 1 && make_tmap(&tmB2, a.W, static_cast<uint64_t>(a.V), a.d, lm::BN / 2) != DLLM_OK)
     return DLLM_ERR_CUDA;
-  if ((cg == 0 || b_rows == 64) &&
-      make_tmap(&tmB64, a.W, static_cast<uint64_t>(a.V), a.d, 64) != DLLM_OK)
-    return DLLM_ERR_CUDA;
-  const CUtensorMap& tmB = b_rows == 256 ? tmB256 : (b_rows == 128 ? tmB128 : tmB64);
 
   cudaEvent_t e0 = nullptr, e1 = nullptr;
   if (g_prof.on) {
@@ -481,39 +453,35 @@ dllm_status run_logits(const LogitsArgs& a, bool debug, bool skip_prepare = fals
       attr[1].val.clusterDim.z = 1;
       cfg.numAttrs = 2;
       cfg.gridDim = dim3(2 * ds->pairs, 1, 1);
-      cfg.dynamicSmemBytes = cg == 0 ? lm::kAutoSmemBytes
-                           : fixed_bn == lm::BN ? lm::Cfg<2, lm::BN>::SMEM_BYTES
-                                                : lm::Cfg<2, lm::BN_NARROW>::SMEM_BYTES;
+      cfg.dynamicSmemBytes = cg == 0 ? lm::kAutoSmemBytes : lm::Cfg<2>::SMEM_BYTES;
     } else {
       cfg.gridDim = dim3(single_holders, 1, 1);
-      cfg.dynamicSmemBytes = fixed_bn == lm::BN ? lm::Cfg<1, lm::BN>::SMEM_BYTES
-                                                : lm::Cfg<1, lm::BN_NARROW>::SMEM_BYTES;
+      cfg.dynamicSmemBytes = lm::Cfg<1>::SMEM_BYTES;
     }
     const int n_cap = static_cast<int>(n);
     float* dbg = debug ? a.dbg : nullptr;
     const int mode = debug ? lm::kModeDebugStore : (a.stats ? lm::kModeStatsExt : lm::kModeStats);
     const int* cnt = a.count;
     cudaError_t e;
-#define DLLM_LAUNCH_GEMM(CGV, TBN, MODE)                                                      \
-  cudaLaunchKernelEx(&cfg, lm::lmhead_kernel<CGV, TBN, MODE>, tmA, tmB, cnt, n_cap, a.V, a.d, \
+#define DLLM_LAUNCH_GEMM(CGV, MODE, TMB)                                                      \
+  cudaLaunchKernelEx(&cfg, lm::lmhead_kernel<CGV, MODE>, tmA, TMB, cnt, n_cap, a.V, a.d,      \
                      lm::Cfg<CGV>::kGroupM, part, w.part_cap, ctr, outs, dbg, ds->status)
-#define DLLM_LAUNCH_FIXED(CGV, TBN)                                                            \
-  (mode == lm::kModeStats ? DLLM_LAUNCH_GEMM(CGV, TBN, lm::kModeStats)                         \
-   : mode == lm::kModeStatsExt ? DLLM_LAUNCH_GEMM(CGV, TBN, lm::kModeStatsExt)                 \
-   : DLLM_LAUNCH_GEMM(CGV, TBN, lm::kModeDebugStore))
 #define DLLM_LAUNCH_AUTO(MODE)                                                                 \
-  cudaLaunchKernelEx(&cfg, lm::lmhead_auto_kernel<MODE>, tmA, tmB256, tmB128, tmB64, cnt,     \
-                     n_cap, a.V, a.d, part, w.part_cap, ctr, outs, dbg, ds->status)
+  cudaLaunchKernelEx(&cfg, lm::lmhead_auto_kernel<MODE>, tmA, tmB1, tmB2, cnt, n_cap, a.V, a.d, \
+                     part, w.part_cap, ctr, outs, dbg, ds->status)
     if (cg == 0)
       e = mode == lm::kModeStats ? DLLM_LAUNCH_AUTO(lm::kModeStats)
         : mode == lm::kModeStatsExt ? DLLM_LAUNCH_AUTO(lm::kModeStatsExt)
         : DLLM_LAUNCH_AUTO(lm::kModeDebugStore);
     else if (cg == 2)
-      e = fixed_bn == lm::BN ? DLLM_LAUNCH_FIXED(2, lm::BN) : DLLM_LAUNCH_FIXED(2, lm::BN_NARROW);
+      e = mode == lm::kModeStats ? DLLM_LAUNCH_GEMM(2, lm::kModeStats, tmB2)
+        : mode == lm::kModeStatsExt ? DLLM_LAUNCH_GEMM(2, lm::kModeStatsExt, tmB2)
+        : DLLM_LAUNCH_GEMM(2, lm::kModeDebugStore, tmB2);
     else
-      e = fixed_bn == lm::BN ? DLLM_LAUNCH_FIXED(1, lm::BN) : DLLM_LAUNCH_FIXED(1, lm::BN_NARROW);
+      e = mode == lm::kModeStats ? DLLM_LAUNCH_GEMM(1, lm::kModeStats, tmB1)
+        : mode == lm::kModeStatsExt ? DLLM_LAUNCH_GEMM(1, lm::kModeStatsExt, tmB1)
+        : DLLM_LAUNCH_GEMM(1, lm::kModeDebugStore, tmB1);
 #undef DLLM_LAUNCH_GEMM
-#undef DLLM_LAUNCH_FIXED
 #undef DLLM_LAUNCH_AUTO
     if (e != cudaSuccess) return DLLM_ERR_CUDA;
   }
@@ -891,9 +859,9 @@ dllm_status dllm_debug_lse_merge(const float* part_m, const float* part_s, const
   return cudaPeekAtLastError() == cudaSuccess ? DLLM_OK : DLLM_ERR_CUDA;
 }
 
-dllm_status dllm_debug_set_gemm_variant(int32_t variant) {
-  if (variant < 0 || variant > 4) return DLLM_ERR_SHAPE;
-  g_gemm_variant.store(variant);
+dllm_status dllm_debug_set_gemm_variant(int32_t cta_group) {
+  if (cta_group != 0 && cta_group != 1 && cta_group != 2) return DLLM_ERR_SHAPE;
+  g_gemm_variant.store(cta_group);
   return DLLM_OK;
 }
 

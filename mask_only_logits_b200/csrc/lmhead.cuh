@@ -62,40 +62,38 @@
 #ifndef DLLM_A_EVICT_LAST
 #define DLLM_A_EVICT_LAST 0       // single-CTA body: load Hm tiles with the L2 evict_last hint
 #endif
+#ifndef DLLM_PAIR_A_HINT
+#define DLLM_PAIR_A_HINT 0        // CTA-pair body: L2 hint of the Hm loads (0 none, 1 evict_last)
+#endif
+#ifndef DLLM_PAIR_W_HINT
+#define DLLM_PAIR_W_HINT 0        // CTA-pair body: L2 hint of the W loads (0 none, 2 evict_first)
+#endif
 #ifndef DLLM_EPI_PACKED
 #define DLLM_EPI_PACKED 0         // epilogue: 3-input max and packed fp32x2 fma / add
 #endif
-#ifndef DLLM_PACE_TILES
-#define DLLM_PACE_TILES 0         // single-CTA body, full groups: lead over the stream's slowest
-#endif                            // holder, in tiles (0 = no pacing)
 
 namespace dllm {
 namespace lm {
 
-constexpr int BN = 256;                 // vocabulary entries per tile (UMMA N), the wide tile
-constexpr int BN_NARROW = 128;          // the narrow tile, for one group of few m-tiles
+constexpr int BN = 256;                 // vocabulary entries per tile (UMMA N)
 constexpr int BK = 64;                  // K per stage: one 128-byte swizzle atom of bf16
 constexpr int UK = 16;                  // K per tcgen05.mma (kind::f16)
 constexpr int kThreads = 192;
 constexpr int kEpiWarps = 4;
-constexpr int kTmemCols = 2 * BN;       // two accumulators, BN columns apart whatever the tile
+constexpr int kTmemCols = 2 * BN;       // two accumulators
 constexpr int kMaxCtas = 160;           // partial-buffer sizing bound (B200: 148 SMs)
 constexpr float kLog2e = 1.4426950408889634f;
 
-// One GEMM body: CTA group size CG and vocabulary tile width TBN (UMMA N).  The narrow
-// tile stages fewer bytes per stage, so its ring holds more stages in the same space.
-template <int CG, int TBN = BN>
+template <int CG>
 struct Cfg {
   static_assert(CG == 1 || CG == 2, "CTA group of 1 or 2");
-  static_assert(TBN == BN || TBN == BN_NARROW, "vocabulary tile of 256 or 128 columns");
-  static constexpr int kBN = TBN;                    // vocabulary columns per tile
   static constexpr int BM_CTA = 128;                 // rows per CTA (TMEM lanes)
   static constexpr int BM = BM_CTA * CG;             // rows per m-tile
-  static constexpr int B_ROWS = TBN / CG;            // W rows staged per CTA per stage
+  static constexpr int B_ROWS = BN / CG;             // W rows staged per CTA per stage
   static constexpr int A_BYTES = BM_CTA * BK * 2;
   static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int kStages = TBN == BN ? (CG == 1 ? 4 : DLLM_STAGES2) : (CG == 1 ? 6 : 8);
+  static constexpr int kStages = CG == 1 ? 4 : DLLM_STAGES2;
   // ring, barriers and flags, and the merge's combine buffer (4 x 128 row states)
   static constexpr int kCombBytes = 4 * BM_CTA * 20;
   static constexpr int SMEM_BYTES = 1024 + kStages * STAGE_BYTES + 256 + kCombBytes;
@@ -105,7 +103,7 @@ struct Cfg {
   // (bits 7-9 = 1, bits 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bits 17-22,
   // M >> 4 at bits 24-28.
   static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
-                                     (static_cast<uint32_t>(TBN >> 3) << 17) |
+                                     (static_cast<uint32_t>(BN >> 3) << 17) |
                                      (static_cast<uint32_t>(BM >> 4) << 24);
 };
 
@@ -122,19 +120,18 @@ struct Cfg {
 // R = ctas - G * P holders the streams leave idle.  Every holder then runs at most
 // max(rb, ceil(G * rr / R)) tiles instead of ceil(numN / P).
 struct Plan {
-  int count, bm, bn, numM, numN, ctas, gmax, ngroups, P_full;
+  int count, bm, numM, numN, ctas, gmax, ngroups, P_full;
   bool rem;        // remainder holders in use (implies ngroups == 1)
   int R, rb, rr;
 
   // ctas = number of work holders (CTAs for CG = 1, CTA pairs for CG = 2);
-  // bm = rows per m-tile; bn = vocabulary columns per tile.
-  __host__ __device__ static Plan make(int count, int V, int ctas, int gmax, int bm, int bn = BN) {
+  // bm = rows per m-tile.
+  __host__ __device__ static Plan make(int count, int V, int ctas, int gmax, int bm) {
     Plan p;
     p.count = count;
     p.bm = bm;
-    p.bn = bn;
     p.numM = (count + bm - 1) / bm;
-    p.numN = (V + bn - 1) / bn;
+    p.numN = (V + BN - 1) / BN;
     p.ctas = ctas;
     p.gmax = gmax < ctas ? gmax : ctas;
     p.ngroups = (p.numM + p.gmax - 1) / p.gmax;
@@ -162,21 +159,6 @@ struct Plan {
   }
   __host__ __device__ int group_size(int g) const {
     return g == ngroups - 1 ? numM - g * gmax : gmax;
-  }
-  // Tiles of the busiest holder: exact for one group of m-tiles; for several, the sum of
-  // every group's busiest stream (an upper bound).
-  __host__ __device__ int busiest() const {
-    int t = 0;
-    for (int g = 0; g < ngroups; ++g) {
-      const int G = group_size(g), P = streams(G, ctas, numN);
-      if (rem) {
-        const int r = (G * rr + R - 1) / R;
-        t += rb > r ? rb : r;
-      } else {
-        t += (numN + P - 1) / P;
-      }
-    }
-    return t;
   }
   // Partial-buffer index of (group g of size G, slot, row r within the group).  Slots:
   // streams 0..P-1, then remainder holders P..P+R-1.
@@ -265,7 +247,7 @@ __host__ __device__ __forceinline__ bool for_each_tile(const Plan& pl, int holde
   return true;
 }
 
-template <int CG, int TBN>
+template <int CG>
 struct Smem {
   uint8_t* a;          // kStages x A_BYTES
   uint8_t* b;          // kStages x B_BYTES
@@ -282,7 +264,7 @@ struct Smem {
   RowStateRaw* comb;         // merge: per warp quarter, the merged state of each of 128 rows
 
   __device__ __forceinline__ explicit Smem(uint8_t* raw) {
-    using C = Cfg<CG, TBN>;
+    using C = Cfg<CG>;
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
     a = base;
     b = base + C::kStages * C::A_BYTES;
@@ -539,17 +521,17 @@ struct Outputs {
 // point at the kernel's own __grid_constant__ tensor-map parameters (TMA needs their
 // parameter-space address, never a copy).  waited: the kernel already passed
 // griddepcontrol.wait (then the set-up below no longer overlaps the previous kernel).
-template <int CG, int TBN, int kMode>
+template <int CG, int kMode>
 __device__ __forceinline__ void lmhead_run(uint8_t* smem_raw, const CUtensorMap* tmA,
                                            const CUtensorMap* tmB, const int* __restrict__ count_ptr,
                                            bool waited, int n_cap, int V, int d, int gmax,
                                            const Partials& part, long long part_cap,
                                            int* __restrict__ unit_ctr, const Outputs& out,
                                            float* __restrict__ dbg_logits, int* __restrict__ status) {
-  using C = Cfg<CG, TBN>;
+  using C = Cfg<CG>;
   constexpr bool kDebugStore = kMode == kModeDebugStore;
   constexpr bool kExt = kMode == kModeStatsExt;
-  Smem<CG, TBN> sm(smem_raw);
+  Smem<CG> sm(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = CG == 1 ? 0u : cluster_ctarank();   // rank inside the CTA pair
   const bool leader = rank == 0;
@@ -596,7 +578,7 @@ __device__ __forceinline__ void lmhead_run(uint8_t* smem_raw, const CUtensorMap*
   }
   const int count = *count_ptr;
   const Plan pl = Plan::make(count < 0 ? 0 : (count > n_cap ? n_cap : count), V,
-                             static_cast<int>(gridDim.x) / CG, gmax, C::BM, C::kBN);
+                             static_cast<int>(gridDim.x) / CG, gmax, C::BM);
   const int holder = static_cast<int>(blockIdx.x) / CG;
   const int KB = d / BK;
   // producer thread of the arming CTA: stages armed so far (bit s), and the phase parity of
@@ -610,42 +592,12 @@ __device__ __forceinline__ void lmhead_run(uint8_t* smem_raw, const CUtensorMap*
       // completion is counted on the leader's full barrier (the address with the peer bit
       // cleared), which the leader arms for the bytes of both CTAs.
       uint32_t it = 0;
-      const uint64_t a_policy = DLLM_A_EVICT_LAST ? policy_evict_last() : 0ull;
-      // Pacing (single CTAs, groups of gmax m-tiles): the holders of one stream read the
-      // same W tiles, so W comes from HBM once per group only while they stay close.  Each
-      // holder publishes how many tiles it has started (holders of one stream start the same
-      // number per full group) and, before a tile, waits until every stream-mate has
-      // started at least DLLM_PACE_TILES fewer.  The slowest holder never waits, so every
-      // wait ends; it is bounded all the same.
-      int* const progress = unit_ctr + ((n_cap + 127) / 128 + 2);
-      int started = 0;
-      auto pace = [&](int m_tile) -> bool {
-        if (DLLM_PACE_TILES <= 0 || CG != 1 || pl.ngroups < 2 || pl.rem) return true;
-        const int g = m_tile / pl.gmax;
-        if (pl.group_size(g) != pl.gmax) return true;            // the last, smaller group
-        st_relaxed_gpu(progress + holder, started);
-        const int need = started - DLLM_PACE_TILES;
-        if (need <= 0) return true;
-        const int first = (holder / pl.gmax) * pl.gmax;          // the stream's first holder
-        const unsigned long long t0 = globaltimer_ns();
-        for (;;) {
-          bool behind = false;
-          for (int j = 0; j < pl.gmax; ++j) behind |= ld_relaxed_gpu(progress + first + j) < need;
-          if (!behind) return true;
-          if (*abort_flag) return false;
-          if (globaltimer_ns() - t0 > kWaitLimitNs) {
-            atomicOr(status, kStatusTimeout);
-            *abort_flag = 1;
-            return false;
-          }
-          __nanosleep(256);
-        }
-      };
+      const uint64_t a_policy =
+          (CG == 1 ? DLLM_A_EVICT_LAST : DLLM_PAIR_A_HINT) ? policy_evict_last() : 0ull;
+      const uint64_t w_policy = DLLM_PAIR_W_HINT ? policy_evict_first() : 0ull;
       auto load_tile = [&](int m_tile, int n) -> bool {
-        if (!pace(m_tile)) return false;
-        ++started;
         const int a_row = m_tile * C::BM + static_cast<int>(rank) * C::BM_CTA;
-        const int b_row = n * C::kBN + static_cast<int>(rank) * C::B_ROWS;
+        const int b_row = n * BN + static_cast<int>(rank) * C::B_ROWS;
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % C::kStages;
           const uint32_t ph = (it / C::kStages) & 1u;
@@ -668,8 +620,16 @@ __device__ __forceinline__ void lmhead_run(uint8_t* smem_raw, const CUtensorMap*
           } else {
             if (leader) mbar_arrive_expect_tx(fb, CG * C::STAGE_BYTES);
             const uint32_t fb_leader = fb & kPeerBitMask;
-            tma_load_2d_pair(smem_u32(sm.a + s * C::A_BYTES), tmA, fb_leader, kb * BK, a_row);
-            tma_load_2d_pair(smem_u32(sm.b + s * C::B_BYTES), tmB, fb_leader, kb * BK, b_row);
+            if (DLLM_PAIR_A_HINT)
+              tma_load_2d_pair_hint(smem_u32(sm.a + s * C::A_BYTES), tmA, fb_leader, kb * BK, a_row,
+                                    a_policy);
+            else
+              tma_load_2d_pair(smem_u32(sm.a + s * C::A_BYTES), tmA, fb_leader, kb * BK, a_row);
+            if (DLLM_PAIR_W_HINT)
+              tma_load_2d_pair_hint(smem_u32(sm.b + s * C::B_BYTES), tmB, fb_leader, kb * BK, b_row,
+                                    w_policy);
+            else
+              tma_load_2d_pair(smem_u32(sm.b + s * C::B_BYTES), tmB, fb_leader, kb * BK, b_row);
           }
         }
         return true;
@@ -738,11 +698,11 @@ __device__ __forceinline__ void lmhead_run(uint8_t* smem_raw, const CUtensorMap*
       const uint32_t taddr = lane_base + buf * BN;
       const int row = m_tile * C::BM + row_in_tile;
 #pragma unroll 1
-      for (int c = 0; c < C::kBN / 32; ++c) {
+      for (int c = 0; c < BN / 32; ++c) {
         float v[32];
         tmem_ld32(taddr + c * 32, v);
         tmem_ld_wait();
-        const int col0 = n * C::kBN + c * 32;
+        const int col0 = n * BN + c * 32;
         if constexpr (kDebugStore) {
           if (row < pl.count) {
             for (int j = 0; j < 32; ++j)
@@ -958,92 +918,49 @@ __device__ __forceinline__ void lmhead_run(uint8_t* smem_raw, const CUtensorMap*
 
 // One GEMM variant, fixed at launch (CG = 2 needs a launch in clusters of two CTAs).  Its
 // set-up (barriers, TMEM, tensor-map prefetch) runs before griddepcontrol.wait, overlapping
-// the previous kernel on the stream.  tmB stages TBN / CG rows of W per CTA.
-template <int CG, int TBN, int kMode>
+// the previous kernel on the stream.
+template <int CG, int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
 lmhead_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const int* __restrict__ count_ptr, int n_cap, int V, int d, int gmax,
               const Partials part, long long part_cap, int* __restrict__ unit_ctr,
               const Outputs out, float* __restrict__ dbg_logits, int* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
-  lmhead_run<CG, TBN, kMode>(smem_raw, &tmA, &tmB, count_ptr, false, n_cap, V, d, gmax, part,
-                             part_cap, unit_ctr, out, dbg_logits, status);
+  lmhead_run<CG, kMode>(smem_raw, &tmA, &tmB, count_ptr, false, n_cap, V, d, gmax, part, part_cap,
+                        unit_ctr, out, dbg_logits, status);
 }
 
 // The variant chosen on the device from the masked count, which the host does not know:
 // one m-tile of 128 rows or fewer runs on single CTAs (a pair would compute 128 empty
 // rows), up to kPairMaxRows rows on CTA pairs (per SM half the W bytes staged per flop),
 // more on single CTAs (longer GEMMs, where the pairs' higher power draw costs clock under
-// the power cap).
+// the power cap).  Launched in clusters of two CTAs with the shared memory of the larger
+// variant; the count is read first, so the set-up follows griddepcontrol.wait.
 constexpr int kSingleMaxRows = 128;
 constexpr int kPairMaxRows = 16384;
 __host__ __device__ inline int auto_variant(int count) {
   return count > kSingleMaxRows && count <= kPairMaxRows ? 2 : 1;
 }
+constexpr int kAutoSmemBytes = Cfg<1>::SMEM_BYTES > Cfg<2>::SMEM_BYTES ? Cfg<1>::SMEM_BYTES
+                                                                        : Cfg<2>::SMEM_BYTES;
 
-// The vocabulary tile width, chosen with the variant.  A problem of one group of m-tiles
-// spreads each m-tile's vocabulary tiles over many holders, and whole tiles rarely divide
-// evenly (B8 L8192 block step: 594 tiles on 74 pairs, so some pairs run 9 tiles while the
-// average is 8.03): narrow tiles halve that granularity.  The busiest holder's tiles times
-// the tile width, plus a small per-tile cost, estimates each schedule's critical path; the
-// narrow tile is taken when it is shorter.  Several groups always use the wide tile (their
-// streams are long, so one tile of imbalance matters little).
-constexpr int kTileCostCols = 8;
-struct Choice {
-  int cg, bn;
-};
-__host__ __device__ inline Choice auto_choice(int count, int V, int grid_ctas) {
-  const int cg = auto_variant(count);
-  const int holders = grid_ctas / cg;
-  const int bm = 128 * cg, gmax = cg == 2 ? Cfg<2>::kGroupM : Cfg<1>::kGroupM;
-  const Plan wide = Plan::make(count, V, holders, gmax, bm, BN);
-  if (wide.ngroups != 1) return Choice{cg, BN};
-  const Plan narrow = Plan::make(count, V, holders, gmax, bm, BN_NARROW);
-  const long long c_wide = static_cast<long long>(wide.busiest()) * (BN + kTileCostCols);
-  const long long c_narrow = static_cast<long long>(narrow.busiest()) * (BN_NARROW + kTileCostCols);
-  return Choice{cg, c_narrow < c_wide ? BN_NARROW : BN};
-}
-
-template <int A, int B>
-struct MaxOf {
-  static constexpr int value = A > B ? A : B;
-};
-constexpr int kAutoSmemBytes =
-    MaxOf<MaxOf<Cfg<1, BN>::SMEM_BYTES, Cfg<2, BN>::SMEM_BYTES>::value,
-          MaxOf<Cfg<1, BN_NARROW>::SMEM_BYTES, Cfg<2, BN_NARROW>::SMEM_BYTES>::value>::value;
-
-// Launched in clusters of two CTAs with the shared memory of the largest body; the count is
-// read first, so the set-up follows griddepcontrol.wait.  Tensor maps of W by rows staged
-// per CTA: tmB256 (single CTAs, wide tile), tmB128 (pairs wide, single CTAs narrow), tmB64
-// (pairs narrow).
 template <int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
-lmhead_auto_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB256,
-                   const __grid_constant__ CUtensorMap tmB128,
-                   const __grid_constant__ CUtensorMap tmB64, const int* __restrict__ count_ptr,
+lmhead_auto_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB1,
+                   const __grid_constant__ CUtensorMap tmB2, const int* __restrict__ count_ptr,
                    int n_cap, int V, int d, const Partials part, long long part_cap,
                    int* __restrict__ unit_ctr, const Outputs out, float* __restrict__ dbg_logits,
                    int* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
   pdl_wait();
   pdl_launch_dependents();
-  int c = *count_ptr;
-  c = c < 0 ? 0 : (c > n_cap ? n_cap : c);
-  const Choice ch = auto_choice(c, V, static_cast<int>(gridDim.x));
-  if (ch.cg == 2 && ch.bn == BN)
-    lmhead_run<2, BN, kMode>(smem_raw, &tmA, &tmB128, count_ptr, true, n_cap, V, d,
-                             Cfg<2>::kGroupM, part, part_cap, unit_ctr, out, dbg_logits, status);
-  else if (ch.cg == 2)
-    lmhead_run<2, BN_NARROW, kMode>(smem_raw, &tmA, &tmB64, count_ptr, true, n_cap, V, d,
-                                    Cfg<2>::kGroupM, part, part_cap, unit_ctr, out, dbg_logits,
-                                    status);
-  else if (ch.bn == BN)
-    lmhead_run<1, BN, kMode>(smem_raw, &tmA, &tmB256, count_ptr, true, n_cap, V, d,
-                             Cfg<1>::kGroupM, part, part_cap, unit_ctr, out, dbg_logits, status);
+  const int c = *count_ptr;
+  if (auto_variant(c) == 2)
+    lmhead_run<2, kMode>(smem_raw, &tmA, &tmB2, count_ptr, true, n_cap, V, d, Cfg<2>::kGroupM,
+                         part, part_cap, unit_ctr, out, dbg_logits, status);
   else
-    lmhead_run<1, BN_NARROW, kMode>(smem_raw, &tmA, &tmB128, count_ptr, true, n_cap, V, d,
-                                    Cfg<1>::kGroupM, part, part_cap, unit_ctr, out, dbg_logits,
-                                    status);
+    lmhead_run<1, kMode>(smem_raw, &tmA, &tmB1, count_ptr, true, n_cap, V, d, Cfg<1>::kGroupM,
+                         part, part_cap, unit_ctr, out, dbg_logits, status);
 }
 
 }  // namespace lm

@@ -35,7 +35,7 @@ def _draw(seed):
     k = int(rng.choice([1, 2, 8, 33, 128]))
     r = float(rng.choice([0.0, 0.05, 0.5, 0.9, 1.0]))
     windows = int(rng.integers(0, 3))          # 0 none, 1 selection windows, 2 block-only
-    variant = int(rng.integers(0, 5))          # default, single, pair, single narrow, pair narrow
+    variant = int(rng.integers(0, 3))
     stats = int(rng.integers(0, 4))
     return rng, B, L, d, V, k, r, windows, variant, stats
 

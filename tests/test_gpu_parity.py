@@ -202,19 +202,6 @@ def test_single_sm_variant(dl, name):
         dl.debug_set_gemm_variant(0)
 
 
-@pytest.mark.parametrize("variant", [3, 4], ids=["single_narrow", "pair_narrow"])
-@pytest.mark.parametrize("name", ["cfg0", "cfg1", "cfg1_m64", "cfg4_block"])
-def test_narrow_tile_variants(dl, variant, name):
-    """The 128-column vocabulary tiles (forced) meet the same bar end to end: the workloads
-    the device picks them for (cfg1_m64, cfg4_block) and two it does not."""
-    dl.debug_set_gemm_variant(variant)
-    try:
-        inp = WL.make_inputs(WL.CONFIGS[name], seed=0)
-        check_step(dl, inp, all_rows=True, window_rows=inp["cfg"].block_only)
-    finally:
-        dl.debug_set_gemm_variant(0)
-
-
 def test_pair_variant_large(dl):
     """The paired-SM (cta_group::2) GEMM on a large workload (default there: single SMs)."""
     dl.debug_set_gemm_variant(2)

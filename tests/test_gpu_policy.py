@@ -25,8 +25,7 @@ def dl():
     return dl
 
 
-@pytest.fixture(params=[0, 1, 2, 3, 4],
-                ids=["default", "single", "pair", "single_narrow", "pair_narrow"])
+@pytest.fixture(params=[0, 1, 2], ids=["default", "single", "pair"])
 def variant(request, dl):
     dl.debug_set_gemm_variant(request.param)
     yield request.param

@@ -34,7 +34,7 @@ def _p(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
-@pytest.mark.parametrize("variant", [1, 2, 3, 4], ids=["single", "pair", "single_narrow", "pair_narrow"])
+@pytest.mark.parametrize("variant", [1, 2], ids=["single", "pair"])
 def test_unarmed_stage_times_out_and_context_survives(injected, variant):
     import mask_only_logits_b200 as dl
     inp = WL.make_inputs(WL.CONFIGS["cfg0"], seed=0)
