@@ -206,8 +206,9 @@ WsLayout ws_layout(int B, int L, int d, int V, long long rows) {
   if (r2 > cap) cap = r2;
   if (cap < 1) cap = 1;
   w.part_cap = cap;
-  // one counter per (m-tile, CTA of the pair): ceil(rows / 128) + 2 covers both variants
-  w.n_ctr = static_cast<int>((rows + 127) / 128 + 2);
+  // one counter per (m-tile, CTA of the pair): ceil(rows / 128) + 2 covers both variants;
+  // then one progress word per work holder (the pair body's pacing), zeroed with them
+  w.n_ctr = static_cast<int>((rows + 127) / 128 + 2 + lm::kMaxCtas);
   size_t off = 0;
   w.tiles_off = off; off = round_up(off + sizeof(int) * ntiles, 256);
   w.ctr_off = off;   off = round_up(off + sizeof(int) * static_cast<size_t>(w.n_ctr), 256);

@@ -68,6 +68,9 @@
 #ifndef DLLM_PAIR_W_HINT
 #define DLLM_PAIR_W_HINT 0        // CTA-pair body: L2 hint of the W loads (0 none, 2 evict_first)
 #endif
+#ifndef DLLM_PAIR_PACE
+#define DLLM_PAIR_PACE 0          // CTA-pair body: lead a holder may take over its stream, in
+#endif                            // tiles (0 = no pacing)
 #ifndef DLLM_EPI_PACKED
 #define DLLM_EPI_PACKED 0         // epilogue: 3-input max and packed fp32x2 fma / add
 #endif
@@ -595,7 +598,55 @@ __device__ __forceinline__ void lmhead_run(uint8_t* smem_raw, const CUtensorMap*
       const uint64_t a_policy =
           (CG == 1 ? DLLM_A_EVICT_LAST : DLLM_PAIR_A_HINT) ? policy_evict_last() : 0ull;
       const uint64_t w_policy = DLLM_PAIR_W_HINT ? policy_evict_first() : 0ull;
+      // Pacing of the CTA-pair body (full groups): the holders of one stream read the same W
+      // tiles, and W comes from HBM about once per group only while they stay within a few
+      // tiles of each other; pairs drift apart over a long stream (measured: 182-421 GB of
+      // DRAM reads per launch on B1 L131072 at r_m = 0.9 without pacing).  Each pair
+      // publishes how many tiles it has started (the pairs of a stream start the same number
+      // per full group); before a tile, a pair that is more than kPace tiles ahead of a
+      // stream-mate waits for it.  The mates' progress is read one tile ahead, so the check
+      // costs the producer nothing unless it really has to wait; the slowest pair never
+      // waits, so every wait ends (it is bounded all the same).
+      constexpr int kPace = CG == 2 ? DLLM_PAIR_PACE : 0;
+      constexpr int kMates = 40;                 // at least the pair body's group size
+      int* const progress = unit_ctr + ((n_cap + 127) / 128 + 2);
+      int started = 0;
+      int seen[kMates];                          // the mates' progress as of the last tile
+#pragma unroll
+      for (int j = 0; j < kMates; ++j) seen[j] = 0;
+      auto pace = [&](int m_tile) -> bool {
+        if (kPace <= 0 || pl.ngroups < 2 || pl.rem || pl.gmax > kMates) return true;
+        const int g = m_tile / pl.gmax;
+        if (pl.group_size(g) != pl.gmax) return true;          // the last, smaller group
+        if (rank == 0) st_relaxed_gpu(progress + holder, started);
+        const int first = (holder / pl.gmax) * pl.gmax;        // the stream's first holder
+        const int need = started - kPace;
+        bool behind = false;
+#pragma unroll
+        for (int j = 0; j < kMates; ++j) behind |= j < pl.gmax && seen[j] < need;
+        if (behind) {                                          // really ahead: fresh reads
+          const unsigned long long t0 = globaltimer_ns();
+          for (;;) {
+            bool lag = false;
+            for (int j = 0; j < pl.gmax; ++j) lag |= ld_relaxed_gpu(progress + first + j) < need;
+            if (!lag) break;
+            if (*abort_flag) return false;
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+              atomicOr(status, kStatusTimeout);
+              *abort_flag = 1;
+              return false;
+            }
+            __nanosleep(128);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < kMates; ++j)                       // for the next tile's check
+          if (j < pl.gmax) seen[j] = ld_relaxed_gpu(progress + first + j);
+        return true;
+      };
       auto load_tile = [&](int m_tile, int n) -> bool {
+        if (!pace(m_tile)) return false;
+        ++started;
         const int a_row = m_tile * C::BM + static_cast<int>(rank) * C::BM_CTA;
         const int b_row = n * BN + static_cast<int>(rank) * C::B_ROWS;
         for (int kb = 0; kb < KB; ++kb, ++it) {

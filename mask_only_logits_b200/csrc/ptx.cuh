@@ -136,6 +136,16 @@ __device__ __forceinline__ bool mbar_wait_until(uint32_t bar, uint32_t parity,
   return true;
 }
 
+// Relaxed GPU-scope load / store of an int (progress words that other CTAs poll).
+__device__ __forceinline__ int ld_relaxed_gpu(const int* p) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_relaxed_gpu(int* p, int v) {
+  asm volatile("st.relaxed.gpu.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // ---------------------------------------------------------------------------------------
 // Clusters of two CTAs (the CTA pair of a cta_group::2 MMA)
 // ---------------------------------------------------------------------------------------
