@@ -99,8 +99,8 @@ def roofline_s(cfg, M: int, peaks: dict) -> float:
 
 def gemm_paired(variant: int, count: int) -> bool:
     """Whether the GEMM runs on CTA pairs: forced (1, 2), or the library's choice from the
-    masked count (pairs for 129..16384 rows)."""
-    return variant == 2 or (variant == 0 and 128 < count <= 16384)
+    masked count (pairs above 128 rows)."""
+    return variant == 2 or (variant == 0 and count > 128)
 
 
 # A timed region at least this long runs in the regime of the measured sustained bf16 rate

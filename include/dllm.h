@@ -488,7 +488,7 @@ dllm_status dllm_debug_lse_merge(const float* part_m, const float* part_s,
  * Test hook: choose the tensor-core GEMM variant used by later calls in this process:
  * 2 = CTA pairs (tcgen05 cta_group::2, 256x256 tiles over two SMs), 1 = single CTAs
  * (cta_group::1, 128x256 tiles), 0 = the default: one launch that picks on the device,
- * from the masked count, pairs for 129..16384 rows and single CTAs otherwise.  Results
+ * from the masked count, single CTAs for at most 128 rows and pairs above.  Results
  * agree to fp32 rounding; the variants differ in speed.  Returns DLLM_ERR_SHAPE for other
  * values.
  */

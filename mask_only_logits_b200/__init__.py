@@ -437,7 +437,7 @@ def debug_lse_merge(part_m, part_s, part_a, tok, conf, lse, stream=None) -> None
 
 def debug_set_gemm_variant(cta_group: int) -> None:
     """Test hook: 2 = paired-SM GEMM, 1 = single-SM GEMM, 0 = default (chosen on the device
-    from the masked count: pairs for 129..16384 rows, single SMs otherwise)."""
+    from the masked count: single SMs for at most 128 rows, pairs above)."""
     _check(lib().dllm_debug_set_gemm_variant(cta_group), "dllm_debug_set_gemm_variant")
 
 

@@ -51,10 +51,9 @@ struct DeviceState {
 
 // GEMM variant: 2 = CTA pairs (cta_group::2, 256x256 tiles), 1 = single CTAs
 // (cta_group::1, 128x256 tiles), both forced (test hook).  0 = default: chosen on the
-// device from the masked count (lm::auto_variant): pairs for 129..16384 rows (the larger
-// tile does more work per clock), single CTAs for one m-tile (a pair would compute 128
-// empty rows) and for long GEMMs (measured under the 1 kW power cap, the single-CTA kernel
-// does more work per joule and sustains a higher clock).
+// device from the masked count (lm::auto_variant): single CTAs for one m-tile of at most
+// 128 rows (a pair would compute 128 empty rows), CTA pairs above (per SM a third fewer
+// bytes staged from L2 per flop, which sets the clock under the 1 kW power cap).
 std::atomic<int> g_gemm_variant{0};
 
 std::mutex g_mu;

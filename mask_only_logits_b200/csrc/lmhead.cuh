@@ -59,21 +59,9 @@
 #ifndef DLLM_EPI_BACKOFF_NS
 #define DLLM_EPI_BACKOFF_NS 0     // epilogue: sleep between polls of the accumulator barrier
 #endif
-#ifndef DLLM_A_EVICT_LAST
-#define DLLM_A_EVICT_LAST 0       // single-CTA body: load Hm tiles with the L2 evict_last hint
-#endif
-#ifndef DLLM_PAIR_A_HINT
-#define DLLM_PAIR_A_HINT 0        // CTA-pair body: L2 hint of the Hm loads (0 none, 1 evict_last)
-#endif
-#ifndef DLLM_PAIR_W_HINT
-#define DLLM_PAIR_W_HINT 0        // CTA-pair body: L2 hint of the W loads (0 none, 2 evict_first)
-#endif
 #ifndef DLLM_PAIR_PACE
-#define DLLM_PAIR_PACE 0          // CTA-pair body: lead a holder may take over its stream, in
+#define DLLM_PAIR_PACE 1          // CTA-pair body: lead a holder may take over its stream, in
 #endif                            // tiles (0 = no pacing)
-#ifndef DLLM_EPI_PACKED
-#define DLLM_EPI_PACKED 0         // epilogue: 3-input max and packed fp32x2 fma / add
-#endif
 
 namespace dllm {
 namespace lm {
@@ -315,21 +303,9 @@ __device__ __forceinline__ void fold_chunk(float (&v)[32], int col0, int V, RowS
     for (int j = 0; j < 32; ++j)
       if (col0 + j >= V) v[j] = -INFINITY;
   }
-  float mx;
-  if constexpr (DLLM_EPI_PACKED) {
-    // 32 -> 11 -> 4 -> 1 with three-input maxima (17 instructions instead of 31)
-    float t[11];
+  float mx = v[0];
 #pragma unroll
-    for (int i = 0; i < 10; ++i) t[i] = max3f(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
-    t[10] = fmaxf(v[30], v[31]);
-    const float u0 = max3f(t[0], t[1], t[2]), u1 = max3f(t[3], t[4], t[5]);
-    const float u2 = max3f(t[6], t[7], t[8]), u3 = fmaxf(t[9], t[10]);
-    mx = fmaxf(max3f(u0, u1, u2), u3);
-  } else {
-    mx = v[0];
-#pragma unroll
-    for (int j = 1; j < 32; ++j) mx = fmaxf(mx, v[j]);
-  }
+  for (int j = 1; j < 32; ++j) mx = fmaxf(mx, v[j]);
   if (mx == -INFINITY) return;                 // the whole chunk is past the vocabulary
   float c2 = -INFINITY;                        // chunk's second largest (= mx on a tie)
   if constexpr (kExt) {
@@ -373,21 +349,6 @@ __device__ __forceinline__ void fold_chunk(float (&v)[32], int col0, int V, RowS
       t1 += e1 > 0.f ? e1 * (v[j + 1] - st.m) : 0.f;
     }
     st.t += t0 + t1;
-  } else if constexpr (DLLM_EPI_PACKED) {
-    // the same arithmetic as the scalar loop below (same four accumulators, same order and
-    // roundings), with fma and add two lanes per instruction
-    const uint64_t scale = pack2f(kLog2e, kLog2e), shift = pack2f(-mb, -mb);
-    uint64_t acc01 = pack2f(0.f, 0.f), acc23 = pack2f(0.f, 0.f);
-#pragma unroll
-    for (int j = 0; j < 32; j += 4) {
-      float a0, a1, a2, a3;
-      unpack2f(fma2f(pack2f(v[j + 0], v[j + 1]), scale, shift), a0, a1);
-      unpack2f(fma2f(pack2f(v[j + 2], v[j + 3]), scale, shift), a2, a3);
-      acc01 = add2f(acc01, pack2f(ex2_approx(a0), ex2_approx(a1)));
-      acc23 = add2f(acc23, pack2f(ex2_approx(a2), ex2_approx(a3)));
-    }
-    unpack2f(acc01, s0, s1);
-    unpack2f(acc23, s2, s3);
   } else {
 #pragma unroll
     for (int j = 0; j < 32; j += 4) {
@@ -595,9 +556,6 @@ __device__ __forceinline__ void lmhead_run(uint8_t* smem_raw, const CUtensorMap*
       // completion is counted on the leader's full barrier (the address with the peer bit
       // cleared), which the leader arms for the bytes of both CTAs.
       uint32_t it = 0;
-      const uint64_t a_policy =
-          (CG == 1 ? DLLM_A_EVICT_LAST : DLLM_PAIR_A_HINT) ? policy_evict_last() : 0ull;
-      const uint64_t w_policy = DLLM_PAIR_W_HINT ? policy_evict_first() : 0ull;
       // Pacing of the CTA-pair body (full groups): the holders of one stream read the same W
       // tiles, and W comes from HBM about once per group only while they stay within a few
       // tiles of each other; pairs drift apart over a long stream (measured: 182-421 GB of
@@ -663,24 +621,13 @@ __device__ __forceinline__ void lmhead_run(uint8_t* smem_raw, const CUtensorMap*
           armed_parity = (armed_parity & ~(1u << s)) | (ph << s);
           if constexpr (CG == 1) {
             mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
-            if (DLLM_A_EVICT_LAST)
-              tma_load_2d_hint(smem_u32(sm.a + s * C::A_BYTES), tmA, fb, kb * BK, a_row, a_policy);
-            else
-              tma_load_2d(smem_u32(sm.a + s * C::A_BYTES), tmA, fb, kb * BK, a_row);
+            tma_load_2d(smem_u32(sm.a + s * C::A_BYTES), tmA, fb, kb * BK, a_row);
             tma_load_2d(smem_u32(sm.b + s * C::B_BYTES), tmB, fb, kb * BK, b_row);
           } else {
             if (leader) mbar_arrive_expect_tx(fb, CG * C::STAGE_BYTES);
             const uint32_t fb_leader = fb & kPeerBitMask;
-            if (DLLM_PAIR_A_HINT)
-              tma_load_2d_pair_hint(smem_u32(sm.a + s * C::A_BYTES), tmA, fb_leader, kb * BK, a_row,
-                                    a_policy);
-            else
-              tma_load_2d_pair(smem_u32(sm.a + s * C::A_BYTES), tmA, fb_leader, kb * BK, a_row);
-            if (DLLM_PAIR_W_HINT)
-              tma_load_2d_pair_hint(smem_u32(sm.b + s * C::B_BYTES), tmB, fb_leader, kb * BK, b_row,
-                                    w_policy);
-            else
-              tma_load_2d_pair(smem_u32(sm.b + s * C::B_BYTES), tmB, fb_leader, kb * BK, b_row);
+            tma_load_2d_pair(smem_u32(sm.a + s * C::A_BYTES), tmA, fb_leader, kb * BK, a_row);
+            tma_load_2d_pair(smem_u32(sm.b + s * C::B_BYTES), tmB, fb_leader, kb * BK, b_row);
           }
         }
         return true;
@@ -983,15 +930,13 @@ lmhead_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
 
 // The variant chosen on the device from the masked count, which the host does not know:
 // one m-tile of 128 rows or fewer runs on single CTAs (a pair would compute 128 empty
-// rows), up to kPairMaxRows rows on CTA pairs (per SM half the W bytes staged per flop),
-// more on single CTAs (longer GEMMs, where the pairs' higher power draw costs clock under
-// the power cap).  Launched in clusters of two CTAs with the shared memory of the larger
-// variant; the count is read first, so the set-up follows griddepcontrol.wait.
+// rows), more on CTA pairs: per SM a third fewer bytes staged from L2 per flop, which under
+// the 1 kW power cap is what sets the clock (measured on B1 L131072 at r_m = 0.9: the paced
+// pair ran the GEMM in 89.8 ms at 1320 MHz where single CTAs took 99-100 ms at 1170 MHz).
+// Launched in clusters of two CTAs with the shared memory of the larger variant; the count
+// is read first, so the set-up follows griddepcontrol.wait.
 constexpr int kSingleMaxRows = 128;
-constexpr int kPairMaxRows = 16384;
-__host__ __device__ inline int auto_variant(int count) {
-  return count > kSingleMaxRows && count <= kPairMaxRows ? 2 : 1;
-}
+__host__ __device__ inline int auto_variant(int count) { return count > kSingleMaxRows ? 2 : 1; }
 constexpr int kAutoSmemBytes = Cfg<1>::SMEM_BYTES > Cfg<2>::SMEM_BYTES ? Cfg<1>::SMEM_BYTES
                                                                         : Cfg<2>::SMEM_BYTES;
 

@@ -90,9 +90,9 @@ def test_bound_switches_at_the_ridge_point():
 def test_gemm_variant_rule_matches_the_kernel():
     text = open(os.path.join(ROOT, "mask_only_logits_b200", "csrc", "lmhead.cuh")).read()
     single = int(re.search(r"kSingleMaxRows\s*=\s*(\d+)", text).group(1))
-    pair = int(re.search(r"kPairMaxRows\s*=\s*(\d+)", text).group(1))
-    for c in (1, single, single + 1, 1024, pair, pair + 1, 117961):
-        assert bench.gemm_paired(0, c) == (single < c <= pair), c
+    assert re.search(r"auto_variant\(int count\) \{ return count > kSingleMaxRows \? 2 : 1; \}", text)
+    for c in (1, single, single + 1, 1024, 16384, 16385, 117961):
+        assert bench.gemm_paired(0, c) == (c > single), c
     assert not bench.gemm_paired(1, 1024) and bench.gemm_paired(2, 10)
 
 
