@@ -22,6 +22,10 @@
 #include "select.cuh"
 #include "arena.cuh"
 
+#ifndef DLLM_GATHER_HOST_CTAS
+#define DLLM_GATHER_HOST_CTAS 1   // gather CTAs per SM when the rows come from host memory
+#endif
+
 namespace dllm {
 
 // An NVTX range around each entry point of the ABI, named after it, so that a timeline
@@ -246,8 +250,9 @@ WsLayout ws_layout_for(int B, int L, int d, int V, size_t ws_bytes) {
 // device can read over PCIe (zero-copy: only the bytes the kernels touch cross the bus,
 // e.g. just the masked rows of H).  Resolves the pointer the kernels use; pageable host
 // memory is rejected (DLLM_ERR_MEMORY) because the device cannot read it.
-dllm_status resolve_input(const void* p, const void** dev) {
+dllm_status resolve_input(const void* p, const void** dev, bool* on_host = nullptr) {
   cudaPointerAttributes at{};
+  if (on_host) *on_host = false;
   if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
     cudaGetLastError();                       // clear the sticky-free error of the query
     return DLLM_ERR_MEMORY;
@@ -258,6 +263,7 @@ dllm_status resolve_input(const void* p, const void** dev) {
   }
   if (at.type == cudaMemoryTypeHost && at.devicePointer != nullptr) {
     *dev = at.devicePointer;
+    if (on_host) *on_host = true;
     return aligned16(*dev) ? DLLM_OK : DLLM_ERR_ALIGN;
   }
   return DLLM_ERR_MEMORY;
@@ -350,7 +356,8 @@ dllm_status validate_logits(const LogitsArgs& a, bool debug, bool prepared = fal
 dllm_status prepare_rows(const LogitsArgs& a, const DeviceState& ds, const WsLayout& w) {
   const void* Hd = nullptr;
   const void* Md = nullptr;
-  dllm_status st = resolve_input(a.H, &Hd);
+  bool host_rows = false;
+  dllm_status st = resolve_input(a.H, &Hd, &host_rows);
   if (st != DLLM_OK) return st;
   if ((st = resolve_input(a.M, &Md)) != DLLM_OK) return st;
   uint8_t* ws = static_cast<uint8_t*>(a.ws);
@@ -361,7 +368,12 @@ dllm_status prepare_rows(const LogitsArgs& a, const DeviceState& ds, const WsLay
   if ((st = launch_compact(static_cast<const uint8_t*>(Md), a.B, a.L, a.win_lo, a.win_hi, a.row_idx,
                            a.seq_off, a.count, tiles, ds.status, a.s)) != DLLM_OK)
     return st;
-  if (launch_pdl(gather_rows_kernel, dim3(ds.sms * 4), dim3(kGatherThreads), 0, a.s,
+  // Rows read from device memory: 4 CTAs per SM.  Rows read over the bus from page-locked
+  // host memory: the bus, not the SMs, bounds the copy (about 20 ms for cfg3's 0.97 GB), and
+  // one CTA per SM keeps enough reads in flight while leaving each SM room for the next
+  // GEMM's persistent CTA, which this staging overlaps.
+  if (launch_pdl(gather_rows_kernel, dim3(ds.sms * (host_rows ? DLLM_GATHER_HOST_CTAS : 4)),
+                 dim3(kGatherThreads), 0, a.s,
                  static_cast<const uint16_t*>(Hd), (const int*)a.row_idx, (const int*)a.count, n,
                  w.rows, a.d, Hm, ctr, w.n_ctr, ds.status) != cudaSuccess)
     return DLLM_ERR_CUDA;
