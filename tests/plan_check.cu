@@ -8,6 +8,8 @@
 //     epilogue's merge waits for;
 //   - without remainder holders, the streams of a group differ by at most one tile; with
 //     them, no holder runs more tiles than the busiest stream would without them;
+//   - in every full group of a problem with several groups, the holders of one stream run
+//     the same number of tiles (what the pair body's pacing compares);
 //   - part_entries() fits the partial region the workspace reserves: groups x holders x
 //     rows per m-tile, or (holders + gmax^2) x rows per m-tile when the problem fits one
 //     group (remainder holders), for any masked count up to the capacity.
@@ -89,6 +91,23 @@ bool check_case(int count, int V, int ctas, int cg) {
     if (pl.rem) pl.leftovers_of(m - g * pl.gmax, G, j_lo, j_hi);
     const int units = Plan::streams(G, ctas, pl.numN) + (j_hi >= j_lo ? j_hi - j_lo + 1 : 0);
     if (writers[m] != units) return fail("writer count", count, V, ctas, cg);
+  }
+  // pacing compares the tiles started by the holders of one stream: in every full group all
+  // holders of a stream run the same number of tiles, and the same in every full group
+  if (!pl.rem && pl.ngroups > 1) {
+    std::vector<int> per_stream_tiles;
+    for (int g = 0; g < pl.ngroups; ++g) {
+      if (pl.group_size(g) != pl.gmax) continue;
+      for (int h = 0; h < ctas; ++h) {
+        Unit u;
+        if (!unit_of(pl, g, h, u) || u.leftover) continue;
+        if (u.G != pl.gmax || u.p != h / pl.gmax) return fail("stream of a full group", count, V, ctas, cg);
+        const int t = u.n1 - u.n0;
+        if (static_cast<int>(per_stream_tiles.size()) <= u.p) per_stream_tiles.resize(u.p + 1, -1);
+        if (per_stream_tiles[u.p] < 0) per_stream_tiles[u.p] = t;
+        if (per_stream_tiles[u.p] != t) return fail("pacing: unequal tiles in a stream", count, V, ctas, cg);
+      }
+    }
   }
   if (!pl.rem) {
     for (int g = 0; g < pl.ngroups; ++g) {
