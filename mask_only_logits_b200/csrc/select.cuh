@@ -66,6 +66,8 @@ select_unmask_kernel(const float* __restrict__ conf, const int* __restrict__ row
   __shared__ unsigned int hist[256];
   __shared__ int sh_lo, sh_hi, sh_n, sh_digit, sh_krem, sh_taken, sh_q;
   __shared__ int warp_cnt[32];
+  __shared__ int blk_cnt[kSelUnroll * 32];      // collect: equal keys per (block of rows, warp)
+  __shared__ int blk_tot[kSelUnroll];
 
   pdl_wait();
   pdl_launch_dependents();
@@ -157,11 +159,21 @@ select_unmask_kernel(const float* __restrict__ conf, const int* __restrict__ row
     // 2'. every candidate is selected
     for (int r = c0 + tid; r < c1; r += kSelThreads) keys[r - c0] = sel_key(key_of(r), r);
   } else if (k_eff > 0) {
-    // 2. radix select of the k_eff-th largest key
+    // 2. radix select of the k_eff-th largest key.  Candidates not staged in shared memory
+    // use that buffer for one 16-bit histogram per warp instead: confidences crowd into a
+    // few bins, and one shared counter per bin had all 32 warps adding to the same words
+    // (a warp sees at most 32 keys per 1024 candidates a pass: 32768 at 2^20 candidates,
+    // within 16 bits).
     uint32_t prefix = 0, pmask = 0;
     int krem = k_eff;
+    const bool warp_hist = !staged && n <= (1 << 20);
+    uint16_t (*whist)[256] = reinterpret_cast<uint16_t (*)[256]>(skey);
+    static_assert(sizeof(skey) >= 32 * 256 * sizeof(uint16_t), "per-warp histograms fit");
     for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
+      if (warp_hist)
+        for (int i = tid; i < 32 * 256 / 2; i += kSelThreads) skey[i] = 0u;
+      else
+        for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
       __syncthreads();
       // warp-aggregated histogram: confidences crowd into few bins (most share their top
       // bits), so lanes with the same bin add their count once
@@ -178,10 +190,24 @@ select_unmask_kernel(const float* __restrict__ conf, const int* __restrict__ row
           uint32_t bin = 0xFFFFFFFFu;
           if (r < c1 && (u[j] & pmask) == prefix) bin = (u[j] >> shift) & 255u;
           const unsigned peers = __match_any_sync(0xffffffffu, bin);
-          if (bin != 0xFFFFFFFFu && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+          if (bin != 0xFFFFFFFFu && lane == __ffs(peers) - 1) {
+            if (warp_hist)
+              whist[warp][bin] = static_cast<uint16_t>(whist[warp][bin] + __popc(peers));
+            else
+              atomicAdd(&hist[bin], __popc(peers));
+          }
         }
       }
       __syncthreads();
+      if (warp_hist) {
+        for (int i = tid; i < 256; i += kSelThreads) {
+          unsigned tot = 0;
+#pragma unroll 8
+          for (int w = 0; w < 32; ++w) tot += whist[w][i];
+          hist[i] = tot;
+        }
+        __syncthreads();
+      }
       if (warp == 0) {
         // lane l owns bins 255-8l down to 248-8l (descending order of digits)
         int own = 0;
@@ -208,38 +234,60 @@ select_unmask_kernel(const float* __restrict__ conf, const int* __restrict__ row
       krem = sh_krem;
       __syncthreads();
     }
-    // 3. collect: all above T, and the first krem equal to T in row order
+    // 3. collect: all above T, and the first krem equal to T in row order.  Rows are taken
+    // kSelUnroll blocks of kSelThreads at a time; the equal keys are counted per (block,
+    // warp) and scanned in that order, which is row order, with four barriers per chunk.
     const uint32_t T = prefix;
     if (tid == 0) sh_taken = 0;
     __syncthreads();
     for (int base = c0; base < c1; base += kSelThreads * kSelUnroll) {
       uint32_t uu[kSelUnroll];
+      unsigned bal[kSelUnroll];
 #pragma unroll
       for (int j = 0; j < kSelUnroll; ++j) {
         const int r = base + j * kSelThreads + tid;
         uu[j] = r < c1 ? key_of(r) : 0u;
       }
-      // blocks of kSelThreads rows in ascending order, so "first in row order" holds
-      for (int j = 0; j < kSelUnroll && base + j * kSelThreads < c1; ++j) {
+#pragma unroll
+      for (int j = 0; j < kSelUnroll; ++j) {
         const int r = base + j * kSelThreads + tid;
-        const uint32_t u = uu[j];
-        const bool gt = r < c1 && u > T;
-        const bool eq = r < c1 && u == T;
-        if (gt) keys[atomicAdd(&sh_n, 1)] = sel_key(u, r);
-        const unsigned bal = __ballot_sync(0xffffffffu, eq);
-        if (lane == 0) warp_cnt[warp] = __popc(bal);
-        __syncthreads();
-        int before = sh_taken;
-        for (int w = 0; w < warp; ++w) before += warp_cnt[w];
-        before += __popc(bal & ((1u << lane) - 1u));
-        if (eq && before < krem) keys[atomicAdd(&sh_n, 1)] = sel_key(u, r);
-        __syncthreads();
-        if (tid == 0) {
-          int tot = 0;
-          for (int w = 0; w < kSelThreads / 32; ++w) tot += warp_cnt[w];
-          sh_taken += tot;
+        if (r < c1 && uu[j] > T) keys[atomicAdd(&sh_n, 1)] = sel_key(uu[j], r);
+        bal[j] = __ballot_sync(0xffffffffu, r < c1 && uu[j] == T);
+        if (lane == 0) blk_cnt[j * 32 + warp] = __popc(bal[j]);
+      }
+      __syncthreads();
+      // exclusive scan of blk_cnt in (block, warp) order: warps 0..kSelUnroll-1 scan one
+      // block each, then each block adds the totals of the blocks before it
+      int v = 0, incl = 0;
+      if (tid < kSelUnroll * 32) {
+        v = blk_cnt[tid];
+        incl = v;
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
         }
-        __syncthreads();
+        if (lane == 31) blk_tot[warp] = incl;
+      }
+      __syncthreads();
+      if (tid < kSelUnroll * 32) {
+        int before_blocks = sh_taken;
+        for (int b2 = 0; b2 < warp; ++b2) before_blocks += blk_tot[b2];
+        blk_cnt[tid] = before_blocks + incl - v;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int j = 0; j < kSelUnroll; ++j) {
+        const int r = base + j * kSelThreads + tid;
+        if (r < c1 && uu[j] == T) {
+          const int before = blk_cnt[j * 32 + warp] + __popc(bal[j] & ((1u << lane) - 1u));
+          if (before < krem) keys[atomicAdd(&sh_n, 1)] = sel_key(uu[j], r);
+        }
+      }
+      __syncthreads();
+      if (tid == 0) {
+        int tot = 0;
+        for (int b2 = 0; b2 < kSelUnroll; ++b2) tot += blk_tot[b2];
+        sh_taken += tot;
       }
     }
   }
