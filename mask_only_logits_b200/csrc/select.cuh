@@ -65,7 +65,6 @@ select_unmask_kernel(const float* __restrict__ conf, const int* __restrict__ row
   __shared__ uint32_t skey[kSelStage];
   __shared__ unsigned int hist[256];
   __shared__ int sh_lo, sh_hi, sh_n, sh_digit, sh_krem, sh_taken, sh_q;
-  __shared__ int warp_cnt[32];
   __shared__ int blk_cnt[kSelUnroll * 32];      // collect: equal keys per (block of rows, warp)
   __shared__ int blk_tot[kSelUnroll];
 

@@ -131,7 +131,13 @@ def variant(request, dl):
                                        (1, 2048, 64, 3000, 1.0),       # 8 m-tiles of 256
                                        (1, 2300, 64, 2000, 1.0),       # 9 of 256 / 18 of 128: streams
                                        (1, 1000, 64, 20000, 1.0),      # 8 m-tiles of 128
-                                       (1, 1000, 64, 37800, 1.0)])     # remainder holders
+                                       (1, 1000, 64, 37800, 1.0),      # remainder holders
+                                       # one m-tile whose vocabulary tiles do not divide
+                                       # evenly among the 74 pairs / 148 CTAs
+                                       (1, 100, 128, 40000, 1.0),      # 157 tiles, 2 K blocks
+                                       (1, 128, 192, 75000, 0.9),      # 3 K blocks, V tail
+                                       (2, 128, 1024, 40000, 1.0),     # 16 K blocks, 256 rows
+                                       (1, 256, 128, 19044, 0.95)])    # 75 tiles over 74 pairs
 def test_lmhead_raw_logits(dl, variant, B, L, d, V, p):
     rng = np.random.default_rng(d + V)
     H = _rand_bf16(rng, (B * L, d), 1.0)
