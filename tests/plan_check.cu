@@ -10,6 +10,8 @@
 //     them, no holder runs more tiles than the busiest stream would without them;
 //   - in every full group of a problem with several groups, the holders of one stream run
 //     the same number of tiles (what the pair body's pacing compares);
+//   - a problem of one m-tile uses the fewest streams that keep the busiest stream's tile
+//     count (the other holders stay idle);
 //   - part_entries() fits the partial region the workspace reserves: groups x holders x
 //     rows per m-tile, or (holders + gmax^2) x rows per m-tile when the problem fits one
 //     group (remainder holders), for any masked count up to the capacity.
@@ -91,6 +93,16 @@ bool check_case(int count, int V, int ctas, int cg) {
     if (pl.rem) pl.leftovers_of(m - g * pl.gmax, G, j_lo, j_hi);
     const int units = Plan::streams(G, ctas, pl.numN) + (j_hi >= j_lo ? j_hi - j_lo + 1 : 0);
     if (writers[m] != units) return fail("writer count", count, V, ctas, cg);
+  }
+  // one m-tile: the fewest streams that keep the busiest stream's tile count of an even
+  // split over min(holders, tiles) streams
+  if (pl.numM == 1 && pl.ngroups == 1) {
+    const int P = Plan::streams(1, ctas, pl.numN);
+    const int P0 = std::max(1, std::min(ctas, pl.numN));
+    const int busiest = (pl.numN + P0 - 1) / P0;
+    if ((pl.numN + P - 1) / P != busiest) return fail("fewest streams: busiest count", count, V, ctas, cg);
+    if (P > 1 && (pl.numN + P - 2) / (P - 1) == busiest)
+      return fail("fewest streams: not the fewest", count, V, ctas, cg);
   }
   // pacing compares the tiles started by the holders of one stream: in every full group all
   // holders of a stream run the same number of tiles, and the same in every full group
